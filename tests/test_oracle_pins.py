@@ -1,0 +1,406 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself:
+the OCP E4M3 encoding table, library routines (torch's fp8 cast, scipy's
+Sylvester Hadamard matrix, numpy's stable argsort), closed forms, invariants
+and brute force on tiny inputs.  CPU only."""
+import math
+import os
+import struct
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.retriever as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --------------------------------------------------------------------- e4m3
+
+
+def test_e4m3_ocp_points():
+    rows = []
+    with open(os.path.join(GOLDEN, "e4m3_ocp_points.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                c, v = line.split()
+                rows.append((int(c, 16), float(v)))
+    codes = np.array([c for c, _ in rows], np.uint8)
+    got = O.e4m3_decode(codes)
+    for (c, v), g in zip(rows, got):
+        if math.isnan(v):
+            assert math.isnan(g), hex(c)
+        else:
+            assert g == v and math.copysign(1, g) == math.copysign(1, v), (hex(c), g, v)
+
+
+def test_e4m3_exhaustive_vs_torch_cast():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = O.e4m3_decode(codes)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).float().numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    # round trip through torch's encoder for every finite code
+    back = torch.from_numpy(ours[~nan].copy()).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    fin = codes[~nan]
+    # -0 and +0 both decode to zero; the encoder keeps the sign
+    assert np.array_equal(back, fin)
+
+
+# ------------------------------------------------------------ record parsing
+
+
+def _record(codes, scale):
+    return np.frombuffer(bytes(codes) + struct.pack("<f", scale), np.uint8).copy()
+
+
+def test_record_scale_is_little_endian_fp32_after_the_codes():
+    rng = np.random.default_rng(0)
+    codes = rng.integers(0, 0x7E, 128).astype(np.uint8)
+    rec = _record(codes, 0.0123)
+    c, s = O.split_records(rec[None])
+    assert np.array_equal(c[0], codes)
+    assert s[0] == np.float32(struct.unpack("<f", struct.pack("<f", 0.0123))[0])
+    k = O.dequant(rec[None])[0]
+    assert np.array_equal(k, (O.e4m3_decode(codes) * np.float32(0.0123)).astype(np.float32))
+
+
+def test_zero_scale_gives_zero_key():
+    rec = _record(np.full(128, 0x7E, np.uint8), 0.0)
+    assert np.all(O.dequant(rec[None]) == 0)
+
+
+def test_dequant_known_bytes():
+    codes = np.zeros(128, np.uint8)
+    codes[0], codes[1], codes[127] = 0x38, 0xC0, 0x01  # 1.0, -2.0, 2^-9
+    k = O.dequant(_record(codes, 4.0)[None])[0]
+    assert k[0] == 4.0 and k[1] == -8.0 and k[127] == 4.0 * 2.0 ** -9
+    assert np.all(k[2:127] == 0)
+
+
+# ---------------------------------------------------------------- linear maps
+
+
+def test_linear_orientation_with_selection_matrix():
+    # W [out=3, in=5] picks inputs 4, 0, 2: a transposed W cannot pass.
+    W = np.zeros((3, 5))
+    W[0, 4] = W[1, 0] = W[2, 2] = 1.0
+    x = np.array([[10., 11., 12., 13., 14.], [1., 2., 3., 4., 5.]])
+    assert np.array_equal(O.linear(W, x), [[14., 10., 12.], [5., 1., 3.]])
+
+
+def test_linear_is_linear():
+    rng = np.random.default_rng(1)
+    W, x, y = rng.normal(size=(7, 9)), rng.normal(size=9), rng.normal(size=9)
+    np.testing.assert_allclose(O.linear(W, 2 * x - 3 * y),
+                               2 * O.linear(W, x) - 3 * O.linear(W, y), atol=1e-12)
+
+
+# -------------------------------------------------------------------- RMSNorm
+
+
+def test_rmsnorm_constant_input_closed_form():
+    c, eps = 0.003, 1e-6
+    g = np.linspace(0.5, 1.5, 16)
+    out = O.rms_norm(np.full(16, c), g, eps)
+    np.testing.assert_allclose(out, g * c / math.sqrt(c * c + eps), rtol=1e-14)
+
+
+def test_rmsnorm_unit_rms_and_gain():
+    rng = np.random.default_rng(2)
+    x = rng.normal(size=(3, 1024)) * 5
+    out = O.rms_norm(x, np.ones(1024))
+    ms = np.mean(x * x, -1)
+    np.testing.assert_allclose(np.sqrt(np.mean(out * out, -1)), np.sqrt(ms / (ms + 1e-6)), rtol=1e-12)
+    g = rng.normal(size=1024)
+    np.testing.assert_allclose(O.rms_norm(x, g), out * g, rtol=1e-12)
+
+
+# ----------------------------------------------------------------- YaRN RoPE
+
+
+def test_yarn_band_edges():
+    # dim(32) = 64 ln(65536/(64 pi)) / (2 ln 160000) = 15.45..,
+    # dim(1)  = 64 ln(65536/(2 pi))  / (2 ln 160000) = 24.71..
+    low, high = O.yarn_correction_range(64, 160000.0, 65536.0, 32.0, 1.0)
+    assert (low, high) == (15, 25)
+
+
+def test_yarn_frequencies_closed_form():
+    f = O.yarn_inv_freq()
+    assert f.shape == (32,)
+    for j in range(32):
+        inv = 160000.0 ** (-j / 32.0)
+        if j <= 15:
+            assert f[j] == pytest.approx(inv, rel=1e-15)
+        elif j >= 25:
+            assert f[j] == pytest.approx(inv / 16.0, rel=1e-15)
+    # middle of the band: ramp = (20 - 15) / 10 = 1/2
+    inv20 = 160000.0 ** (-20 / 32.0)
+    assert f[20] == pytest.approx(0.5 * inv20 + 0.5 * inv20 / 16.0, rel=1e-15)
+    assert f[0] == 1.0
+
+
+def test_rotary_pairing_and_sign():
+    # a quarter turn sends e_{64+j} to e_{96+j} and e_{96+j} to -e_{64+j}
+    for j in (0, 7, 31):
+        q = np.zeros((1, 1, 128))
+        q[0, 0, 64 + j] = 1.0
+        theta = np.zeros((1, 32))
+        theta[0, j] = math.pi / 2
+        out = O.apply_rotary(q, theta)[0, 0]
+        expect = np.zeros(128)
+        expect[96 + j] = 1.0
+        np.testing.assert_allclose(out, expect, atol=1e-15)
+        q2 = np.zeros((1, 1, 128))
+        q2[0, 0, 96 + j] = 1.0
+        out2 = O.apply_rotary(q2, theta)[0, 0]
+        expect2 = np.zeros(128)
+        expect2[64 + j] = -1.0
+        np.testing.assert_allclose(out2, expect2, atol=1e-15)
+
+
+def test_rope_angle_is_position_times_frequency():
+    f = O.yarn_inv_freq()
+    pos = np.array([1 << 20, 12345])
+    th = O.rope_angles(pos, f)
+    assert th.shape == (2, 32)
+    q = np.zeros((2, 1, 128))
+    q[:, 0, 64 + 3] = 1.0
+    out = O.apply_rotary(q, th)
+    for b in range(2):
+        a = float(pos[b]) * (160000.0 ** (-3 / 32.0))
+        assert out[b, 0, 64 + 3] == pytest.approx(math.cos(a), abs=1e-12)
+        assert out[b, 0, 96 + 3] == pytest.approx(math.sin(a), abs=1e-12)
+
+
+def test_rope_identity_norm_untouched_and_composition():
+    rng = np.random.default_rng(3)
+    q = rng.normal(size=(2, 64, 128))
+    f = O.yarn_inv_freq()
+    zero = O.apply_rotary(q, O.rope_angles(np.zeros(2), f))
+    np.testing.assert_array_equal(zero, q)
+    pos = np.array([16384, 1 << 20])
+    r = O.apply_rotary(q, O.rope_angles(pos, f))
+    np.testing.assert_array_equal(r[..., :64], q[..., :64])
+    np.testing.assert_allclose(np.linalg.norm(r, axis=-1), np.linalg.norm(q, axis=-1), rtol=1e-12)
+    two = O.apply_rotary(O.apply_rotary(q, O.rope_angles(np.array([100, 7]), f)),
+                         O.rope_angles(np.array([23, 1000]), f))
+    one = O.apply_rotary(q, O.rope_angles(np.array([123, 1007]), f))
+    np.testing.assert_allclose(two, one, atol=1e-11)
+
+
+# ------------------------------------------------------------------ Hadamard
+
+
+def test_hadamard_matches_scipy_sylvester():
+    import scipy.linalg
+    np.testing.assert_array_equal(O.hadamard_matrix(128), scipy.linalg.hadamard(128))
+
+
+def test_hadamard_kron_construction():
+    H2 = np.array([[1., 1.], [1., -1.]])
+    H = np.ones((1, 1))
+    for _ in range(7):
+        H = np.kron(H, H2)
+    np.testing.assert_array_equal(O.hadamard_matrix(128), H)
+
+
+def test_wht_orthonormal_involution():
+    H = O.hadamard_matrix(128)
+    np.testing.assert_array_equal(H @ H, 128 * np.eye(128))
+    rng = np.random.default_rng(4)
+    x = rng.normal(size=(5, 128))
+    y = O.hadamard_transform(x)
+    np.testing.assert_allclose(O.hadamard_transform(y), x, atol=1e-12)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-13)
+    e0 = np.zeros(128)
+    e0[0] = 1
+    np.testing.assert_allclose(O.hadamard_transform(e0), np.full(128, 128 ** -0.5), rtol=1e-15)
+    e1 = np.zeros(128)
+    e1[1] = 1
+    np.testing.assert_allclose(O.hadamard_transform(e1) * math.sqrt(128),
+                               np.tile([1., -1.], 64), rtol=1e-15)
+
+
+# ------------------------------------------------------- query prep, composed
+
+
+def _tiny_layer(rng, hid=48, rank=32, H=3, D=128):
+    return dict(wq_a=rng.normal(size=(rank, hid)) * 0.1,
+                q_norm=1 + rng.normal(size=rank) * 0.1,
+                wq_b=rng.normal(size=(H * D, rank)) * 0.1,
+                weights_proj=rng.normal(size=(H, hid)) * 0.1)
+
+
+def test_query_prep_order_of_steps():
+    rng = np.random.default_rng(5)
+    layer = _tiny_layer(rng)
+    h = rng.normal(size=(2, 48))
+    pos = np.array([0, 4096])
+    q, w = O.query_prep(layer, h, pos, n_heads=3, head_dim=128)
+    # undo the (involutive) Hadamard: the heads before rotation
+    pre = O.hadamard_transform(q)
+    a = h @ layer["wq_a"].T
+    r = a / np.sqrt(np.mean(a * a, -1, keepdims=True) + 1e-6) * layer["q_norm"]
+    qf = (r @ layer["wq_b"].T).reshape(2, 3, 128)
+    # row 0 has position 0: no rotation at all
+    np.testing.assert_allclose(pre[0], qf[0], atol=1e-12)
+    # row 1: rotation leaves dims 0..63 and the rotated half's norm alone
+    np.testing.assert_allclose(pre[1, :, :64], qf[1, :, :64], atol=1e-12)
+    np.testing.assert_allclose(np.linalg.norm(pre[1, :, 64:], axis=-1),
+                               np.linalg.norm(qf[1, :, 64:], axis=-1), rtol=1e-12)
+    assert not np.allclose(pre[1, :, 64:], qf[1, :, 64:])
+    # the head-weight branch: constant HEAD_DIM^-1/2 * N_HEADS^-1/2
+    np.testing.assert_allclose(w, (h @ layer["weights_proj"].T) / math.sqrt(128 * 3), rtol=1e-13)
+
+
+def test_head_weight_scale_constant():
+    layer = dict(wq_a=np.eye(4), q_norm=np.ones(4), wq_b=np.zeros((64 * 128, 4)),
+                 weights_proj=np.ones((64, 4)))
+    _, w = O.query_prep(layer, np.array([[1., 0., 0., 0.]]), np.array([0]))
+    np.testing.assert_allclose(w, np.full((1, 64), 0.011048543456039806), rtol=1e-15)
+
+
+# --------------------------------------------------------------------- score
+
+
+def _records_from_keys(k):
+    """Exactly representable keys: k = codes * scale with scale 1."""
+    codes = torch.from_numpy(np.asarray(k, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    return np.stack([_record(c, 1.0) for c in codes])
+
+
+def test_score_hand_example():
+    # two heads, D = 128; q_h = e_h so dot_h = k[h]
+    q = np.zeros((2, 128))
+    q[0, 0] = q[1, 1] = 1.0
+    k = np.zeros((3, 128))
+    k[0, :2] = [1.0, -2.0]    # relu -> (1, 0):  logit = 0.5
+    k[1, :2] = [-1.0, 2.0]    # relu -> (0, 2):  logit = 2 * (-0.25) = -0.5
+    k[2, :2] = [3.0, 4.0]     # logit = 1.5 - 1.0 = 0.5
+    w = np.array([0.5, -0.25])
+    s = O.score_chunks(_records_from_keys(k), q, w)
+    np.testing.assert_allclose(s, [0.6224593312018546, 0.3775406687981454, 0.6224593312018546],
+                               rtol=1e-15)
+
+
+def test_score_scale_applies_inside_relu():
+    q = np.zeros((1, 128))
+    q[0, 0] = 1.0
+    codes = np.zeros(128, np.uint8)
+    codes[0] = 0x38  # 1.0
+    rec = np.stack([_record(codes, 0.5), _record(codes, 0.0)])
+    s = O.score_chunks(rec, q, np.array([2.0]))
+    np.testing.assert_allclose(s, [1 / (1 + math.exp(-1.0)), 0.5], rtol=1e-15)
+
+
+def test_score_degenerate_cases_and_range():
+    rng = np.random.default_rng(6)
+    q = rng.normal(size=(64, 128))
+    w = rng.normal(size=64)
+    # zero scale -> k = 0 -> sigma(0) = 1/2 exactly
+    zero = np.stack([_record(rng.integers(0, 0x7E, 128).astype(np.uint8), 0.0) for _ in range(3)])
+    assert np.all(O.score_chunks(zero, q, w) == 0.5)
+    # a key anti-aligned with every head -> every relu is 0
+    qpos = np.abs(q)
+    neg = _records_from_keys(-np.ones((1, 128)))
+    assert O.score_chunks(neg, qpos, w)[0] == 0.5
+    recs = np.stack([_record(rng.integers(0, 0x7E, 128).astype(np.uint8), float(s))
+                     for s in rng.uniform(0, 1, 64)])
+    s = O.score_chunks(recs, q * 10, w * 10)
+    assert np.all((s >= 0) & (s <= 1))
+
+
+def test_score_brute_force_tiny():
+    rng = np.random.default_rng(7)
+    H, N = 4, 8
+    q = rng.normal(size=(H, 128))
+    w = rng.normal(size=H)
+    recs = np.stack([_record(rng.integers(0, 0x7E, 128).astype(np.uint8),
+                             float(rng.uniform(0.001, 0.01))) for _ in range(N)])
+    got = O.score_chunks(recs, q, w)
+    for n in range(N):
+        scale = struct.unpack("<f", bytes(recs[n, 128:132]))[0]
+        kv = [float(torch.tensor([int(b)], dtype=torch.uint8).view(torch.float8_e4m3fn).float()) * scale
+              for b in recs[n, :128]]
+        logit = 0.0
+        for h in range(H):
+            d = sum(kv[i] * q[h, i] for i in range(128))
+            logit += max(d, 0.0) * w[h]
+        assert got[n] == pytest.approx(1.0 / (1.0 + math.exp(-logit)), rel=1e-6, abs=1e-7)
+
+
+def test_score_layer_pads_with_zero():
+    rng = np.random.default_rng(8)
+    ck = np.zeros((2, 6, 132), np.uint8)
+    for b in range(2):
+        for n in range(6):
+            ck[b, n] = _record(rng.integers(0, 0x7E, 128).astype(np.uint8), 0.01)
+    s = O.score_layer(ck, np.array([6, 2]), rng.normal(size=(2, 64, 128)), rng.normal(size=(2, 64)))
+    assert np.all(s[1, 2:] == 0) and np.all(s[1, :2] > 0) and np.all(s[0] > 0)
+
+
+# ------------------------------------------------------------------ ensemble
+
+
+def test_ensemble_values():
+    s = np.array([[[0.1, 0.9]], [[0.4, 0.2]], [[0.7, 0.3]]])
+    np.testing.assert_allclose(O.ensemble(s, "max"), [[0.7, 0.9]])
+    np.testing.assert_allclose(O.ensemble(s, "mean"), [[0.4, 1.4 / 3]], rtol=1e-15)
+
+
+def test_ensemble_max_ge_mean_and_identical_layers():
+    rng = np.random.default_rng(9)
+    s = rng.uniform(size=(3, 4, 50))
+    assert np.all(O.ensemble(s, "max") >= O.ensemble(s, "mean") - 1e-15)
+    same = np.stack([s[0]] * 3)
+    np.testing.assert_allclose(O.ensemble(same, "mean"), s[0], rtol=1e-15)
+    np.testing.assert_array_equal(O.ensemble(same, "max"), s[0])
+
+
+# ----------------------------------------------------------------- selection
+
+
+def test_topk_matches_stable_argsort():
+    rng = np.random.default_rng(10)
+    ens = rng.integers(0, 20, size=(3, 200)).astype(np.float32) / 20  # many ties
+    nv = np.array([200, 150, 7])
+    keep = O.select_topk(ens, nv, 30)
+    for b in range(3):
+        n = nv[b]
+        order = np.argsort(-ens[b, :n].astype(np.float64), kind="stable")
+        expect = np.zeros(200, bool)
+        expect[order[:min(30, n)]] = True
+        np.testing.assert_array_equal(keep[b], expect)
+        assert keep[b].sum() == min(30, n)
+
+
+def test_topk_brute_force_and_ties():
+    ens = np.array([[0.5, 0.7, 0.7, 0.2, 0.7, 0.9]])
+    keep = O.select_topk(ens, np.array([6]), 3)
+    # 0.9 first, then the two lowest-index 0.7s
+    np.testing.assert_array_equal(keep[0], [False, True, True, False, False, True])
+    keep = O.select_topk(ens, np.array([6]), 10)
+    assert keep.all()
+    keep = O.select_topk(ens, np.array([3]), 10)
+    np.testing.assert_array_equal(keep[0], [True, True, True, False, False, False])
+    dup = np.full((1, 40), 0.25)
+    np.testing.assert_array_equal(O.select_topk(dup, np.array([40]), 9)[0], np.arange(40) < 9)
+
+
+def test_topk_keeps_everything_above_kth():
+    rng = np.random.default_rng(11)
+    ens = rng.uniform(size=(2, 1000))
+    keep = O.select_topk(ens, np.array([1000, 1000]), 100)
+    for b in range(2):
+        kth = np.sort(ens[b])[::-1][99]
+        assert np.all(keep[b][ens[b] > kth]) and not np.any(keep[b][ens[b] < kth])
+
+
+def test_threshold_is_strict_and_respects_length():
+    ens = np.array([[0.5, 0.50000006, 0.4, 0.9, 0.9]], np.float32)
+    keep = O.select_threshold(ens, np.array([4]), 0.5)
+    np.testing.assert_array_equal(keep[0], [False, True, False, True, False])
