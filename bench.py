@@ -1,0 +1,375 @@
+#!/usr/bin/env python
+"""Throughput of the FlashMemory DS-V4 retriever hot path on B200.
+
+One step = the whole path for one batch of decode rows: query prep for all
+three CSA layers, the fused scoring pass (3 layers + ensemble), and the top-K
+keep-mask.  Default workload: B=64 rows x N=262144 chunks per layer (6.6 GB of
+fp8 keys, larger than L2), max ensemble, top-4096, query prep timed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I]
+    python bench.py --impl reference ...   # the CPU oracle on host cores
+
+Multi-GPU (torchrun): every rank scores its own batch (weak scaling, no
+collective on the data path); the time is the max over ranks.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gen import synthetic as G  # noqa: E402
+
+METRIC = "retriever chunks scored/sec (3-layer ensemble + top-K)"
+UNIT = "chunks/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=4)
+    ap.add_argument("--q-pieces", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[device_index]) if vis else device_index
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((mhz, reasons, util))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        nv = self.nv
+        names = {
+            "gpu_idle": nv.nvmlClocksEventReasonGpuIdle,
+            "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap,
+            "hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+            "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+            "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+            "hw_power_brake_slowdown": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown,
+            "applications_clocks_setting": nv.nvmlClocksEventReasonApplicationsClocksSetting,
+        }
+        loaded = [s for s in self.samples if s[2] > 0] or self.samples
+        seen = set()
+        for _, r, _ in loaded:
+            for n, bit in names.items():
+                if r & bit and n != "gpu_idle":
+                    seen.add(n)
+        return {"sm_mhz": float(statistics.median(s[0] for s in loaded)),
+                "sm_max_mhz": float(self.max_mhz), "reasons": sorted(seen),
+                "samples": len(loaded)}
+
+
+# -------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    from learned_kv_chunk_b200 import fm
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = G.WORKLOADS[args.workload]
+    inp = G.make_query_inputs(wl)
+    B, N, L = wl.B, wl.N, G.N_LAYERS
+    r = fm.Retriever(inp.weights, device=local_rank, max_batch=max(64, B), q_pieces=args.q_pieces)
+    hidden = inp.hidden.to(dev)
+    positions = inp.positions.to(dev)
+    n_valid = inp.n_valid.to(dev)
+    q, w = r.fm_query_prep(hidden, positions)
+    plant = q[:, :, 0, :].permute(1, 0, 2).contiguous().cpu()
+    keys = G.make_keys(wl.seed(G.SEED_KEYS) + 7919 * rank, [int(x) for x in inp.n_valid], N, L,
+                       plant, device=dev)
+    torch.cuda.synchronize()
+    decisions = int(inp.n_valid.sum())          # valid (row, chunk) pairs per step
+    key_bytes = L * decisions * G.RECORD_BYTES  # valid records only
+
+    ens = torch.empty(B, N, device=dev, dtype=torch.float32)
+    keep = torch.empty(B, N, device=dev, dtype=torch.bool)
+    keep_thr = torch.empty(B, N, device=dev, dtype=torch.bool) if wl.threshold is not None else None
+    ws = torch.empty(fm.fm_topk_workspace_bytes(B, N), device=dev, dtype=torch.uint8)
+    qb = torch.empty(B, L, 64, 128, device=dev)
+    wb = torch.empty(B, L, 64, device=dev)
+    stream = torch.cuda.current_stream()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = key_bytes < 4 * l2
+    flush_buf = torch.empty(max(2 * l2, 1 << 28) // 4, device=dev, dtype=torch.float32) if flush else None
+
+    ev_sc = []
+
+    def step(timed=False):
+        r.fm_query_prep(hidden, positions, q=qb, fused_w=wb)
+        if timed:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+        r.fm_score_fused(keys, qb, wb, mode=wl.mode, threshold=wl.threshold, n_valid=n_valid, N=N,
+                         ens=ens, keep_thr=keep_thr)
+        if timed:
+            b.record(stream)
+            ev_sc.append((a, b))
+        fm.fm_select_topk(ens, wl.top_k, n_valid, out=keep, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    r.fm_sync_status()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    sampler = ClockSampler(local_rank)
+    launches0 = fm.fm_launch_count()
+    with sampler:
+        barrier()
+        if not flush:
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(args.steps):
+                step(timed=True)
+            t1.record(stream)
+            torch.cuda.synchronize()
+            elapsed_ms = t0.elapsed_time(t1)
+        else:
+            elapsed_ms = 0.0
+            for _ in range(args.steps):
+                flush_buf.fill_(1.0)
+                t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                t0.record(stream)
+                step(timed=True)
+                t1.record(stream)
+                torch.cuda.synchronize()
+                elapsed_ms += t0.elapsed_time(t1)
+        barrier()
+    launches = fm.fm_launch_count() - launches0
+    r.fm_sync_status()
+    score_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_sc]))
+
+    t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    elapsed_max = float(t.item())
+    ms_per_step = elapsed_max / args.steps
+    value = decisions * world * args.steps / (elapsed_max / 1e3)
+
+    hbm_peak, peak_kind = peaks()
+    alg_bytes = decisions * (L * G.RECORD_BYTES + 4)  # keys + ensembled score per decision
+    achieved = alg_bytes / (score_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                "kernel": "score_kernel (fused scoring pass, via fm_score_fused)",
+                "kernel_ms": round(score_ms, 4), "peak_kind": peak_kind,
+                "alg_bytes_per_launch": alg_bytes}
+
+    # end to end through the host-buffer API: H2D of the step's inputs, D2H of the mask
+    e2e = None
+    if not args.no_e2e:
+        hk = [k.cpu().pin_memory() for k in keys]
+        hh, hp, hn = hidden.cpu().pin_memory(), positions.cpu().pin_memory(), inp.n_valid.pin_memory()
+        bufs = {}
+        r.retrieve_from_host(hh, hp, hk, hn, wl.mode, wl.top_k, wl.threshold, N, bufs)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            kt, kh = r.retrieve_from_host(hh, hp, hk, hn, wl.mode, wl.top_k, wl.threshold, N, bufs)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        et = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+        if world > 1:
+            torch.distributed.all_reduce(et, op=torch.distributed.ReduceOp.MAX)
+        h2d = sum(k.numel() for k in hk) + hh.numel() * 4 + hp.numel() * 8 + hn.numel() * 4
+        d2h = B * N * (2 if wl.threshold is not None else 1)
+        e2e = {"value": decisions * world * args.e2e_steps / (float(et.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": args.e2e_steps}
+        del hk
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_sample(inp, keys, wl, q_row=0)
+
+    r.close()
+    return dict(value=value, ms_per_step=ms_per_step, roofline=roofline, e2e=e2e, cpu=cpu,
+                clocks=sampler.summary(), launches=launches, decisions=decisions, flush=flush,
+                key_bytes=key_bytes)
+
+
+def _oracle_threads():
+    try:
+        import threadpoolctl
+        return max(i["num_threads"] for i in threadpoolctl.threadpool_info()) or os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline_sample(inp, keys, wl, q_row=0):
+    """The CPU oracle, as it stands, on one row of the workload (all chunks,
+    3 layers, query prep, ensemble, top-K)."""
+    import oracle.retriever as O
+    b = q_row
+    n = int(inp.n_valid[b])
+    layers = [{k: v.numpy().astype(np.float64) for k, v in w_.items()} for w_ in inp.weights]
+    host = [k[b, :n].cpu().numpy() for k in keys]
+    h = inp.hidden[b:b + 1].numpy().astype(np.float64)
+    pos = inp.positions[b:b + 1].numpy()
+    t0 = time.perf_counter()
+    qw = [O.query_prep(l, h, pos) for l in layers]
+    s = np.stack([O.score_chunks(host[l], qw[l][0][0], qw[l][1][0]) for l in range(len(layers))])
+    e = O.ensemble(s, wl.mode)[None]
+    O.select_topk(e, np.array([n]), wl.top_k)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"row {b} of the workload: {n} chunks x 3 layers, query prep, ensemble, "
+                      f"top-{wl.top_k} ({dt:.1f} s)"}
+
+
+# ---------------------------------------------------------- reference arm
+def run_reference(args):
+    """The CPU oracle on the host cores: each step scores a bounded sample
+    (one row's query prep + 8192 chunks x 3 layers + ensemble + top-K)."""
+    import oracle.retriever as O
+    wl = G.WORKLOADS[args.workload]
+    inp = G.make_query_inputs(wl)
+    layers = [{k: v.numpy().astype(np.float64) for k, v in w_.items()} for w_ in inp.weights]
+    M = min(8192, wl.N)
+    samples = []
+    for s in range(2):
+        b = s % wl.B
+        h = inp.hidden[b:b + 1].numpy().astype(np.float64)
+        pos = inp.positions[b:b + 1].numpy()
+        keys = [G.make_key_slab(wl.seed(G.SEED_KEYS), l, b, M, None).numpy() for l in range(3)]
+        samples.append((h, pos, keys))
+
+    def step(i):
+        h, pos, keys = samples[i % len(samples)]
+        qw = [O.query_prep(l, h, pos) for l in layers]
+        sc = np.stack([O.score_chunks(keys[l], qw[l][0][0], qw[l][1][0]) for l in range(3)])
+        e = O.ensemble(sc, wl.mode)[None]
+        O.select_topk(e, np.array([M]), min(wl.top_k, M))
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    value = M * args.steps / dt
+    cores = _oracle_threads()
+    sample = f"per step: one row's query prep + {M} chunks x 3 layers + ensemble + top-{min(wl.top_k, M)}"
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(wl, args.gpus),
+            "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample, "value": value,
+                             "unit": UNIT},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def config_of(wl, gpus, flush=None, key_bytes=None):
+    c = {"workload": wl.name, "global_batch": wl.B * gpus, "chunks_per_row": wl.N, "layers": 3,
+         "ensemble": wl.mode, "top_k": wl.top_k, "threshold": wl.threshold,
+         "query_prep_in_step": True, "parallelism": f"rows sharded over {gpus} GPU(s), no collective"}
+    if flush is not None:
+        c["l2"] = ("flushed between steps (256 MB write)" if flush
+                   else f"inputs larger than L2 ({key_bytes / 1e9:.2f} GB of keys per step)")
+    return c
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    wl = G.WORKLOADS[args.workload]
+    out = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "e4m3 x e4m3 tensor-core products, f32 accumulate/epilogue; f32 query prep",
+           "data": "synthetic (seeded generator, random-init weights)",
+           "config": config_of(wl, world, res["flush"], res["key_bytes"]),
+           "roofline": res["roofline"], "e2e": res["e2e"], "gpu_launches": res["launches"],
+           "clocks": res["clocks"], "cpu_baseline": res["cpu"]}
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,211 @@
+/*
+ * fm.h -- C ABI of libfm, a B200 (sm_100a) implementation of the FlashMemory
+ * DS-V4 retriever's hot path: the Memory Indexer that scores every
+ * fp8-compressed CSA KV chunk against a decode token's indexer query for three
+ * CSA layers (l10, l12, l20), ensembles the layers and selects a keep-mask.
+ *
+ * Source of the operations: the FlashMemory DS-V4 Retriever README
+ * (libertywing/FlashMemory-Deepseek-V4, translated copy on
+ * bittide.aicompass.dev): "Usage" (the calls and their shapes),
+ * "compressed_k format" (the 132-byte record), "Architecture" (the query
+ * chain and the score formula), "Joint checkpoint + ensemble" (max / mean),
+ * and the decode-loop figure of "Toy inference reference" (top-K or
+ * sigmoid > thresh keep-mask).
+ *
+ * Conventions shared by every call
+ *   - Pointers marked "device" are CUDA device pointers owned by the caller;
+ *     the library never frees them.  Pointers marked "host or device" may be
+ *     either (copied with cudaMemcpyDefault).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and returns an fm_status.  Argument errors are
+ *     detected on the host before anything is launched, and nothing is
+ *     written in that case.  Errors raised inside a kernel (a bounded wait
+ *     that ran out) are recorded in the context and reported by
+ *     fm_sync_status.
+ *   - No call allocates device memory except fm_create (and fm_destroy frees).
+ *     Calls on one context must not run concurrently on different streams:
+ *     they share the context's packed-query workspace.
+ *   - Shapes: L = n_layers (1..4), H = n_heads = 64, D = head_dim = 128,
+ *     HID = hidden, R = q_lora_rank.  B rows (decode tokens), N chunks per row.
+ *   - A keep mask is one byte per chunk, 0 or 1 (the layout of torch.bool).
+ *     Entries past a row's valid length n_valid[b] score 0.0f and are never
+ *     kept.
+ */
+#ifndef FM_H_
+#define FM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cudaStream_t;
+
+typedef int fm_status;
+enum {
+  FM_OK = 0,
+  FM_ERR_INVALID_ARG = 1,  /* a size, pointer or option is out of range          */
+  FM_ERR_ALIGNMENT = 2,    /* a pointer or stride breaks the alignment rule      */
+  FM_ERR_UNSUPPORTED = 3,  /* shape the kernels are not built for                */
+  FM_ERR_CUDA = 4,         /* a CUDA runtime call failed (see fm_last_cuda_error) */
+  FM_ERR_OOM = 5,          /* cudaMalloc failed in fm_create                     */
+  FM_ERR_DEVICE = 6        /* a kernel recorded an error (bounded wait ran out)  */
+};
+
+enum { FM_ENSEMBLE_MAX = 0, FM_ENSEMBLE_MEAN = 1 };
+
+/* Model constants.  README "Architecture" fixes HEAD_DIM = 128, ROPE_DIM = 64,
+ * base 160000, eps 1e-6 and hidden 4096; the hyper-parameter table that would
+ * give Q_LORA_RANK and N_HEADS is missing from the pages, so they are inputs
+ * (1024 and 64 in every shipped workload).  Supported: hidden % 128 == 0,
+ * q_lora_rank % 128 == 0, n_heads == 64, head_dim == 128, rope_dim == 64,
+ * 1 <= n_layers <= 4, 1 <= max_batch <= 4096, q_pieces in {2, 3}. */
+typedef struct fm_config {
+  int hidden;             /* 4096 */
+  int q_lora_rank;        /* 1024 */
+  int n_heads;            /* 64 */
+  int head_dim;           /* 128 */
+  int n_layers;           /* 3: l10, l12, l20 */
+  int rope_dim;           /* 64: the last 64 dims of each head */
+  double rope_base;       /* 160000 */
+  double rope_factor;     /* YaRN scaling factor, 16 */
+  double rope_orig_max_pos; /* YaRN original context, 65536 */
+  double rope_beta_fast;  /* 32 */
+  double rope_beta_slow;  /* 1 */
+  float rms_eps;          /* 1e-6 */
+  int max_batch;          /* largest B any call on this context will pass */
+  int q_pieces;           /* e4m3 pieces per query element in the tensor-core
+                             product: 3 (default, ~2^-12 relative) or 2 (~2^-8) */
+} fm_config;
+
+/* One layer's weights, fp32, row-major [out, in], no biases (README
+ * "Architecture": wq_a 4096 -> Q_LORA_RANK, RMSNorm weight, wq_b
+ * Q_LORA_RANK -> N_HEADS*HEAD_DIM, weights_proj 4096 -> N_HEADS).
+ * Host or device pointers; fm_create copies them. */
+typedef struct fm_layer_weights {
+  const float* wq_a;         /* [R, HID]   */
+  const float* q_norm;       /* [R]        */
+  const float* wq_b;         /* [H*D, R]   */
+  const float* weights_proj; /* [H, HID]   */
+} fm_layer_weights;
+
+typedef struct fm_ctx fm_ctx;
+
+/* Fills *cfg with the shipped constants (hidden 4096, rank 1024, 64 heads,
+ * head_dim 128, 3 layers, YaRN 160000/16/65536/32/1, eps 1e-6, max_batch 64,
+ * q_pieces 3). */
+void fm_config_default(fm_config* cfg);
+
+/* Creates a context on `device`: uploads the weights (cfg->n_layers entries of
+ * `weights`) and allocates the packed-query workspace for cfg->max_batch rows.
+ * Synchronous.  FM_ERR_INVALID_ARG / FM_ERR_UNSUPPORTED for a bad config,
+ * FM_ERR_OOM, FM_ERR_CUDA.  *out is NULL on failure. */
+fm_status fm_create(const fm_config* cfg, const fm_layer_weights* weights, int device,
+                    fm_ctx** out);
+
+/* Frees everything fm_create allocated (synchronises the device first). */
+fm_status fm_destroy(fm_ctx* ctx);
+
+/* Query side of every layer (README "Architecture", upper two chains):
+ *   q[b,l]       = Hadamard(RoPE_YaRN(reshape(wq_b . RMSNorm(wq_a . hidden[b]))))
+ *   fused_w[b,l] = (weights_proj . hidden[b]) * HEAD_DIM^-1/2 * N_HEADS^-1/2
+ * hidden    [B, HID] fp32 device, row-major.
+ * positions [B] int64 device (token position of each row, >= 0).
+ * q         [B, L, H, D] fp32 device (written).
+ * fused_w   [B, L, H] fp32 device (written).
+ * 1 <= B <= max_batch.  All fp32 arithmetic; the RoPE angles pos * f_j and
+ * their cos/sin are taken in fp64 and rounded once. */
+fm_status fm_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* positions, int B,
+                        float* q, float* fused_w, cudaStream_t stream);
+
+/* Per-layer chunk scores (README "Architecture", score line):
+ *   scores[l,b,n] = sigmoid( sum_h relu(k[l,b,n] . q[b,l,h]) * fused_w[b,l,h] )
+ *   k[l,b,n]      = e4m3(comp_k[l][b,n,0:128]) * f32le(comp_k[l][b,n,128:132])
+ * comp_k    array of L device pointers (host array); layer l's keys are
+ *           [B, N_pad, 132] uint8 with row b starting at
+ *           comp_k[l] + b * row_stride_bytes.  Each pointer 16-byte aligned,
+ *           row_stride_bytes a multiple of 16 and >= N * 132 rounded up to a
+ *           multiple of 528 (i.e. N_pad >= N rounded up to 4) -- the tile
+ *           copy reads whole 4-record groups.  Otherwise FM_ERR_ALIGNMENT.
+ * n_valid   [B] int32 device, 0 <= n_valid[b] <= N, or NULL (= N for all).
+ * q, fused_w as written by fm_query_prep (any producer is fine).
+ * scores    [L, B, N] fp32 device (written; 0.0f past n_valid).
+ * The product k.q runs on the tensor cores with q split into q_pieces e4m3
+ * terms (per-head power-of-two scaling) and the keys used as stored. */
+fm_status fm_score(fm_ctx* ctx, const uint8_t* const* comp_k, int64_t row_stride_bytes,
+                   const int32_t* n_valid, int B, int N, const float* q, const float* fused_w,
+                   float* scores, cudaStream_t stream);
+
+/* Cross-layer ensemble (README "Joint checkpoint + ensemble"):
+ *   mode FM_ENSEMBLE_MAX:  ens[b,n] = max_l scores[l,b,n]   (union, default)
+ *   mode FM_ENSEMBLE_MEAN: ens[b,n] = (((s0 + s1) + s2) ...) / L   in fp32
+ * scores [L, B, N] fp32 device; ens [B, N] fp32 device (written). */
+fm_status fm_ensemble(const float* scores, int L, int B, int N, int mode, float* ens,
+                      cudaStream_t stream);
+
+/* One pass that scores all L layers, ensembles them and (optionally) applies
+ * the threshold rule, writing one fp32 per chunk instead of L.
+ * Inputs as fm_score.  mode as fm_ensemble.
+ * scores_or_null [L, B, N] fp32 device or NULL (per-layer scores not written).
+ * ens            [B, N] fp32 device (written).
+ * keep_thr_or_null [B, N] uint8 device or NULL: keep = (ens > thr) for valid
+ *                chunks (strict, README toy loop "sigmoid > thresh"); thr is
+ *                ignored when this pointer is NULL. */
+fm_status fm_score_fused(fm_ctx* ctx, const uint8_t* const* comp_k, int64_t row_stride_bytes,
+                         const int32_t* n_valid, int B, int N, const float* q,
+                         const float* fused_w, int mode, float thr, float* scores_or_null,
+                         float* ens, uint8_t* keep_thr_or_null, cudaStream_t stream);
+
+/* Bytes of device workspace fm_select_topk needs for B rows of N chunks. */
+size_t fm_topk_workspace_bytes(int B, int N);
+
+/* Top-K keep mask (README "Usage" select_topk(top_k=K); toy loop "top-K"):
+ * keep[b,n] = 1 for the min(k, n_b) largest ens[b, 0:n_b], equal scores taken
+ * in increasing chunk index; 0 elsewhere.  Scores must be >= 0 (sigmoid
+ * outputs); NaN ranks below every number.
+ * ens [B, N] fp32 device; n_valid [B] int32 device or NULL; k >= 1;
+ * keep [B, N] uint8 device (written);
+ * ws device workspace of at least fm_topk_workspace_bytes(B, N) bytes,
+ * 16-byte aligned, owned by the caller; its contents on entry do not matter. */
+fm_status fm_select_topk(const float* ens, const int32_t* n_valid, int B, int N, int k,
+                         uint8_t* keep, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Threshold keep mask (README "Usage" select_topk(threshold=t)):
+ * keep[b,n] = (n < n_b) && (ens[b,n] > thr).  Shapes as fm_select_topk. */
+fm_status fm_select_threshold(const float* ens, const int32_t* n_valid, int B, int N, float thr,
+                              uint8_t* keep, cudaStream_t stream);
+
+/* Synchronises `stream` and returns FM_ERR_DEVICE if a kernel launched on this
+ * context recorded an error since the last call (the record is cleared),
+ * FM_ERR_CUDA if the stream reports a CUDA error, FM_OK otherwise. */
+fm_status fm_sync_status(fm_ctx* ctx, cudaStream_t stream);
+
+/* Static text for a status code. */
+const char* fm_strerror(fm_status status);
+
+/* The last CUDA runtime error code seen by any call of this thread (0 = none). */
+int fm_last_cuda_error(void);
+
+/* Number of kernel launches issued by this process since load (all calls). */
+uint64_t fm_launch_count(void);
+
+/* Diagnostic: the raw tensor-core dot products of one 128-chunk tile of layer
+ * `layer`, row b, tile t (chunks t*128 .. t*128+127), before the per-chunk
+ * scale, the per-head power-of-two scale and the epilogue:
+ *   out[r, p*64 + h] = sum_d e4m3(comp_k[layer][b, t*128 + r, d]) * piece_p(q[b,layer,h])[d]
+ * where the query pieces satisfy
+ *   q[b,layer,h,d] ~= 2^-pow2_exp[h] * sum_p 16^-p * piece_p[d].
+ * out [128, q_pieces*64] fp32 device (written), pow2_exp [64] int32 device
+ * (written).  Rows of the tile past N hold unspecified values.  Used by the
+ * tests to check the tensor-core operand layouts in isolation. */
+fm_status fm_debug_tile_dots(fm_ctx* ctx, const uint8_t* const* comp_k, int64_t row_stride_bytes,
+                             int B, int N, const float* q, const float* fused_w, int layer, int b,
+                             int t, float* out, int32_t* pow2_exp, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FM_H_ */

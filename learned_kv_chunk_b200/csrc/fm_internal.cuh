@@ -1,0 +1,280 @@
+// fm_internal.cuh -- shared declarations and PTX wrappers of libfm (sm_100a).
+//
+// Everything here is written for Blackwell (sm_100a): mbarrier-tracked bulk
+// copies (the TMA engine's 1-D form), tcgen05 tensor-core MMA with TMEM
+// accumulators, and bounded waits that record an error instead of hanging.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fm.h"
+
+namespace fm {
+
+// ---------------------------------------------------------------- constants
+constexpr int kHeads = 64;        // N_HEADS (the shipped value; checked at create)
+constexpr int kHeadDim = 128;     // HEAD_DIM (README "Architecture")
+constexpr int kRopeDim = 64;      // ROPE_DIM (README "Architecture")
+constexpr int kRecord = 132;      // bytes per compressed chunk (README "compressed_k format")
+constexpr int kTile = 128;        // chunks per tensor-core tile (MMA M)
+constexpr int kMaxLayers = 4;
+constexpr int kMaxBatch = 4096;
+
+// device error codes written into the context's error word
+enum : int { kDevErrNone = 0, kDevErrTimeout = 1 };
+
+}  // namespace fm
+
+// The context behind the opaque fm_ctx handle.
+struct fm_ctx {
+  fm_config cfg;
+  int device;
+  int num_sms;
+  // weights (device)
+  float* w_down;    // [L*(R+H), HID]: per layer wq_a rows then weights_proj rows
+  float* q_norm;    // [L, R]
+  float* w_up;      // [L, H*D, R]
+  double* rope_freq;  // [rope_dim/2] YaRN frequencies (fp64)
+  // workspace (device), sized for cfg.max_batch rows
+  int splitk_max;
+  float* a_part;    // [splitk_max, max_batch, L*(R+H)] partial sums of the down projection
+  float* r_norm;    // [max_batch, L, R] RMSNorm output
+  float* rope_cs;   // [max_batch, rope_dim/2, 2] cos, sin
+  uint8_t* qpack;   // [max_batch, L, q_pieces*64*128] e4m3 query pieces (MMA operand image)
+  float* wprime;    // [max_batch, L, 64] fused_w * 2^-e per head
+  int32_t* qexp;    // [max_batch, L, 64] the exponent e of each head's scaling
+  int* d_err;       // device error word
+};
+
+namespace fm {
+
+// launch helpers (fm_api.cu)
+void note_launch();
+fm_status check_launch();
+
+// kernels' host entry points
+fm_status launch_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* positions, int B,
+                            float* q, float* fused_w, cudaStream_t stream);
+fm_status launch_qpack(fm_ctx* ctx, const float* q, const float* fused_w, int B,
+                       cudaStream_t stream);
+
+struct ScoreArgs {
+  const uint8_t* comp_k[kMaxLayers];
+  int64_t row_stride;      // bytes between rows of one layer
+  const int32_t* n_valid;  // [B] or null
+  int B, N, L;
+  const uint8_t* qpack;    // [B, L, P*64*128]
+  const float* wprime;     // [B, L, 64]
+  float* scores;           // [L, B, N] or null
+  float* ens;              // [B, N] or null
+  uint8_t* keep_thr;       // [B, N] or null
+  float thr;
+  int mode;                // FM_ENSEMBLE_*
+  int* err;
+  // diagnostic dump of one tile's raw accumulators
+  float* dbg_out;          // [128, P*64] or null
+  int dbg_layer, dbg_b, dbg_t;
+};
+fm_status launch_score(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t stream);
+
+fm_status launch_ensemble(const float* scores, int L, int B, int N, int mode, float* ens,
+                          cudaStream_t stream);
+fm_status launch_threshold(const float* ens, const int32_t* n_valid, int B, int N, float thr,
+                           uint8_t* keep, cudaStream_t stream);
+size_t topk_workspace_bytes(int B, int N);
+fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, int k, uint8_t* keep,
+                      void* ws, size_t ws_bytes, cudaStream_t stream);
+
+// ------------------------------------------------------------ PTX wrappers
+#if defined(__CUDACC__)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits until the phase with the given parity of `bar` has completed.  Gives
+// up after `limit_ns` of wall time or as soon as *abort becomes non-zero; on
+// a timeout it records kDevErrTimeout in *err and sets *abort.  Returns true
+// when the phase completed.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort, int* err,
+                                                  uint64_t limit_ns = 2000000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        atomicExch(err, kDevErrTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// 1-D bulk copy global -> shared through the TMA engine, completing on `bar`
+// (transaction bytes).  dst, src and bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+      "[%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// Makes this thread's generic-proxy shared-memory writes visible to the async
+// proxy (tensor-core operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------- tcgen05
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, fp8 (kind::f8f6f4) inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrives on `bar` once every tcgen05.mma this thread issued before has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// 32 lanes x 32 consecutive fp32 columns; thread i gets lane (base_lane + i).
+__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major operand stored in the
+// canonical 128-byte-swizzled layout: rows of 128 bytes, groups of 8 rows
+// 1024 bytes apart, the 16-byte chunk c of row r stored at chunk c ^ (r % 8).
+// `addr` is the shared address of the first element used (1024-aligned tile
+// base plus a k offset of a multiple of 32 bytes inside the row).
+__device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr & 0x3FFFFu) >> 4);  // start address, 16-byte units
+  d |= static_cast<uint64_t>(1) << 16;                 // leading byte offset (unused here)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;         // stride byte offset: 8-row groups
+  d |= static_cast<uint64_t>(1) << 46;                 // descriptor version (sm_100)
+  d |= static_cast<uint64_t>(2) << 61;                 // layout: 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: kind::f8f6f4, A = B = E4M3, D = F32, both K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                                    // D format F32
+         | (0u << 7) | (0u << 10)                     // A, B format E4M3
+         | (0u << 15) | (0u << 16)                    // A, B K-major
+         | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
+// Byte offset of element (row, k) inside a K-major 128B-swizzled tile of
+// 128-byte rows (one fp8 element per byte).
+__host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t kbyte) {
+  return (row >> 3) * 1024u + (row & 7u) * 128u + ((((kbyte >> 4) ^ (row & 7u)) & 7u) << 4) +
+         (kbyte & 15u);
+}
+
+#endif  // __CUDACC__
+
+}  // namespace fm

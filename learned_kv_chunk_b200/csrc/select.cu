@@ -1,0 +1,326 @@
+// select.cu -- cross-layer ensemble and keep-mask selection.
+//
+// README "Joint checkpoint + ensemble": per-chunk max (union, default) or mean
+// over the layers.  README "Usage" / toy decode loop: keep = top-K of the
+// ensembled scores, or sigmoid > thresh.
+//
+// Top-K is an exact radix select on order-preserving 32-bit keys of the fp32
+// scores: three histogram passes (11 + 11 + 10 bits, most significant first)
+// fix the K-th largest key T and how many keys equal to T are kept; a mask
+// pass then keeps every key > T and the first `need` keys == T in chunk-index
+// order (only when the keys equal to T outnumber `need` does it rank them,
+// with a per-block count pass and an in-block ordered scan).  Each histogram
+// pass ends in its last-arriving block (atomic ticket, no waiting), which
+// chooses the digit for the row; no kernel waits on another block.
+#include "fm_internal.cuh"
+
+namespace fm {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kPerThread = 16;
+constexpr int kChunk = kThreads * kPerThread;  // elements per block slice
+constexpr int kBins0 = 2048, kBins1 = 2048, kBins2 = 1024;
+constexpr int kHistWords = kBins0 + kBins1 + kBins2;
+constexpr int kShift[3] = {21, 10, 0};
+constexpr int kBits[3] = {11, 11, 10};
+
+enum : int { kModeEmpty = 0, kModeAll = 1, kModeSelect = 2 };
+
+// Per-row state (in the workspace).
+struct RowState {
+  int nv;          // valid chunks
+  int mode;        // kMode*
+  uint32_t prefix; // key digits chosen so far
+  int remaining;   // how many of the keys matching `prefix` are still to keep
+  int need_eq;     // after the last pass: keys == T to keep
+  int cnt_eq;      // after the last pass: keys == T present
+  int tickets[3];  // arrival counters of the three histogram passes
+  int pad[7];
+};
+static_assert(sizeof(RowState) == 64, "row state is 64 bytes");
+
+struct Workspace {
+  RowState* state;  // [B]
+  uint32_t* hist;   // [B, kHistWords]
+  int* eqcnt;       // [B, nblk]
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+__host__ __device__ inline Workspace carve(void* ws, int B, int nblk) {
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  Workspace w;
+  w.state = reinterpret_cast<RowState*>(p);
+  p += align256(sizeof(RowState) * (size_t)B);
+  w.hist = reinterpret_cast<uint32_t*>(p);
+  p += align256(sizeof(uint32_t) * (size_t)B * kHistWords);
+  w.eqcnt = reinterpret_cast<int*>(p);
+  return w;
+}
+
+__host__ __device__ inline size_t ws_bytes(int B, int nblk) {
+  return align256(sizeof(RowState) * (size_t)B) + align256(sizeof(uint32_t) * (size_t)B * kHistWords) +
+         align256(sizeof(int) * (size_t)B * nblk);
+}
+
+// Order-preserving key: larger float -> larger key; +0 and -0 equal; NaN lowest.
+__device__ __forceinline__ uint32_t order_key(float x) {
+  if (x != x) return 0u;
+  uint32_t u = (x == 0.f) ? 0u : __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ int row_nvalid(const int32_t* n_valid, int b, int N) {
+  int v = n_valid ? n_valid[b] : N;
+  return max(0, min(v, N));
+}
+
+// ------------------------------------------------------------ ensemble
+__global__ void ensemble_kernel(const float* __restrict__ scores, int L, int64_t BN, int mode,
+                                float* __restrict__ ens) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < BN;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float e = scores[i];
+    if (mode == FM_ENSEMBLE_MAX) {
+      for (int l = 1; l < L; ++l) e = fmaxf(e, scores[(int64_t)l * BN + i]);
+    } else {
+      for (int l = 1; l < L; ++l) e = e + scores[(int64_t)l * BN + i];
+      e = e / (float)L;
+    }
+    ens[i] = e;
+  }
+}
+
+// ----------------------------------------------------------- threshold
+__global__ void threshold_kernel(const float* __restrict__ ens, const int32_t* __restrict__ n_valid,
+                                 int N, float thr, uint8_t* __restrict__ keep) {
+  const int b = blockIdx.y;
+  const int nv = row_nvalid(n_valid, b, N);
+  for (int n = blockIdx.x * blockDim.x + threadIdx.x; n < N; n += gridDim.x * blockDim.x) {
+    const float e = ens[(int64_t)b * N + n];
+    keep[(int64_t)b * N + n] = (n < nv && e > thr) ? 1 : 0;
+  }
+}
+
+// --------------------------------------------------------------- top-K
+__global__ void topk_init_kernel(Workspace w, const int32_t* __restrict__ n_valid, int N, int k) {
+  const int b = blockIdx.x;
+  uint32_t* h = w.hist + (size_t)b * kHistWords;
+  for (int i = threadIdx.x; i < kHistWords; i += blockDim.x) h[i] = 0u;
+  if (threadIdx.x == 0) {
+    RowState s = {};
+    s.nv = row_nvalid(n_valid, b, N);
+    s.mode = s.nv == 0 ? kModeEmpty : (k >= s.nv ? kModeAll : kModeSelect);
+    s.prefix = 0u;
+    s.remaining = min(k, s.nv);
+    w.state[b] = s;
+  }
+}
+
+template <int PASS>
+__global__ void __launch_bounds__(kThreads) topk_hist_kernel(Workspace w, const float* __restrict__ ens,
+                                                             int N) {
+  constexpr int bins = PASS == 0 ? kBins0 : (PASS == 1 ? kBins1 : kBins2);
+  constexpr int shift = kShift[PASS];
+  constexpr int hi_shift = shift + kBits[PASS];  // digits above this pass
+  __shared__ uint32_t sh[bins];
+  __shared__ int s_last;
+  __shared__ uint32_t s_suffix[kThreads];
+  const int b = blockIdx.y;
+  RowState* st = w.state + b;
+  if (st->mode != kModeSelect) return;  // uniform across the block
+  const int nv = st->nv;
+  const uint32_t prefix = st->prefix;
+  for (int i = threadIdx.x; i < bins; i += kThreads) sh[i] = 0u;
+  __syncthreads();
+  const int64_t base = (int64_t)blockIdx.x * kChunk;
+  const float* row = ens + (int64_t)b * N;
+#pragma unroll 4
+  for (int i = 0; i < kPerThread; ++i) {
+    const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
+    if (n < nv) {
+      const uint32_t key = order_key(row[n]);
+      const bool match = (hi_shift >= 32) || ((key >> (hi_shift & 31)) == (prefix >> (hi_shift & 31)));
+      if (match) atomicAdd(&sh[(key >> shift) & (bins - 1)], 1u);
+    }
+  }
+  __syncthreads();
+  uint32_t* gh = w.hist + (size_t)b * kHistWords + (PASS == 0 ? 0 : (PASS == 1 ? kBins0 : kBins0 + kBins1));
+  for (int i = threadIdx.x; i < bins; i += kThreads)
+    if (sh[i]) atomicAdd(&gh[i], sh[i]);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&st->tickets[PASS], 1) == (int)gridDim.x - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // Last block of the row: pick the digit holding the remaining-th largest key.
+  // Thread t owns bins [t*per, (t+1)*per) in descending order of value.
+  constexpr int per = bins / kThreads;
+  uint32_t cnt[per];
+  uint32_t mine = 0;
+#pragma unroll
+  for (int j = 0; j < per; ++j) {
+    const int d = bins - 1 - (threadIdx.x * per + j);  // descending digit
+    cnt[j] = __ldcg(&gh[d]);
+    mine += cnt[j];
+  }
+  s_suffix[threadIdx.x] = mine;
+  __syncthreads();
+  // inclusive scan over threads (descending digit order)
+  for (int off = 1; off < kThreads; off <<= 1) {
+    const uint32_t v = threadIdx.x >= off ? s_suffix[threadIdx.x - off] : 0u;
+    __syncthreads();
+    s_suffix[threadIdx.x] += v;
+    __syncthreads();
+  }
+  const uint32_t before = s_suffix[threadIdx.x] - mine;  // keys with a larger digit
+  const uint32_t want = (uint32_t)st->remaining;
+  if (before < want && before + mine >= want) {
+    uint32_t acc = before;
+#pragma unroll
+    for (int j = 0; j < per; ++j) {
+      if (acc + cnt[j] >= want) {
+        const int d = bins - 1 - (threadIdx.x * per + j);
+        st->prefix = prefix | ((uint32_t)d << shift);
+        st->remaining = (int)(want - acc);
+        if (PASS == 2) {
+          st->need_eq = (int)(want - acc);
+          st->cnt_eq = (int)cnt[j];
+        }
+        break;
+      }
+      acc += cnt[j];
+    }
+  }
+}
+
+// Per-block count of keys equal to T, only for rows whose tie at T is split.
+__global__ void __launch_bounds__(kThreads) topk_eqcount_kernel(Workspace w, const float* __restrict__ ens,
+                                                                int N, int nblk) {
+  const int b = blockIdx.y;
+  const RowState* st = w.state + b;
+  if (st->mode != kModeSelect || st->need_eq == st->cnt_eq) return;
+  const uint32_t T = st->prefix;
+  const int nv = st->nv;
+  const int64_t base = (int64_t)blockIdx.x * kChunk;
+  const float* row = ens + (int64_t)b * N;
+  int c = 0;
+  for (int i = 0; i < kPerThread; ++i) {
+    const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
+    if (n < nv && order_key(row[n]) == T) ++c;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  __shared__ int red[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int i = 0; i < kThreads / 32; ++i) t += red[i];
+    w.eqcnt[(size_t)b * nblk + blockIdx.x] = t;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) topk_mask_kernel(Workspace w, const float* __restrict__ ens,
+                                                             int N, int nblk, uint8_t* __restrict__ keep) {
+  const int b = blockIdx.y;
+  const RowState* st = w.state + b;
+  const int mode = st->mode, nv = st->nv;
+  const uint32_t T = st->prefix;
+  const bool split_tie = mode == kModeSelect && st->need_eq != st->cnt_eq;
+  const int need = st->need_eq;
+  const int64_t base = (int64_t)blockIdx.x * kChunk;
+  const float* row = ens + (int64_t)b * N;
+  uint8_t* out = keep + (int64_t)b * N;
+  if (!split_tie) {
+    for (int i = 0; i < kPerThread; ++i) {
+      const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
+      if (n >= N) break;
+      uint8_t k = 0;
+      if (n < nv) k = (mode == kModeAll) ? 1 : (order_key(row[n]) >= T ? 1 : 0);
+      out[n] = k;
+    }
+    return;
+  }
+  // ordered rank among keys == T: blocks before this one, then in-block order
+  __shared__ int s_prefix;
+  __shared__ int s_warp[kThreads / 32];
+  if (threadIdx.x == 0) {
+    int p = 0;
+    for (int j = 0; j < (int)blockIdx.x; ++j) p += w.eqcnt[(size_t)b * nblk + j];
+    s_prefix = p;
+  }
+  __syncthreads();
+  int running = s_prefix;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = 0; i < kPerThread; ++i) {
+    const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
+    uint32_t key = 0;
+    if (n < nv) key = order_key(row[n]);
+    const int eq = (n < nv && key == T) ? 1 : 0;
+    // block-wide exclusive scan of eq in index order
+    const unsigned ball = __ballot_sync(0xffffffffu, eq);
+    const int in_warp = __popc(ball & ((1u << lane) - 1u));
+    if (lane == 0) s_warp[warp] = __popc(ball);
+    __syncthreads();
+    int before_warp = 0, total = 0;
+    for (int j = 0; j < kThreads / 32; ++j) {
+      if (j < warp) before_warp += s_warp[j];
+      total += s_warp[j];
+    }
+    const int rank = running + before_warp + in_warp;
+    if (n < N) {
+      uint8_t k = 0;
+      if (n < nv) k = (key > T || (eq && rank < need)) ? 1 : 0;
+      out[n] = k;
+    }
+    running += total;
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+fm_status launch_ensemble(const float* scores, int L, int B, int N, int mode, float* ens,
+                          cudaStream_t st) {
+  const int64_t BN = (int64_t)B * N;
+  int64_t g = (BN + 255) / 256;
+  const int grid = (int)(g < 148 * 16 ? g : 148 * 16);
+  ensemble_kernel<<<grid, 256, 0, st>>>(scores, L, BN, mode, ens);
+  note_launch();
+  return check_launch();
+}
+
+fm_status launch_threshold(const float* ens, const int32_t* n_valid, int B, int N, float thr,
+                           uint8_t* keep, cudaStream_t st) {
+  const int64_t gx = ((int64_t)N + 1023) / 1024;
+  dim3 grid((unsigned)(gx < 1024 ? gx : 1024), B);
+  threshold_kernel<<<grid, 256, 0, st>>>(ens, n_valid, N, thr, keep);
+  note_launch();
+  return check_launch();
+}
+
+size_t topk_workspace_bytes(int B, int N) {
+  const int nblk = (int)(((int64_t)N + kChunk - 1) / kChunk);
+  return ws_bytes(B, nblk);
+}
+
+fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, int k, uint8_t* keep,
+                      void* ws, size_t ws_size, cudaStream_t st) {
+  const int nblk = (int)(((int64_t)N + kChunk - 1) / kChunk);
+  if (ws_size < ws_bytes(B, nblk)) return FM_ERR_INVALID_ARG;
+  Workspace w = carve(ws, B, nblk);
+  topk_init_kernel<<<B, 256, 0, st>>>(w, n_valid, N, k);
+  dim3 grid(nblk, B);
+  topk_hist_kernel<0><<<grid, kThreads, 0, st>>>(w, ens, N);
+  topk_hist_kernel<1><<<grid, kThreads, 0, st>>>(w, ens, N);
+  topk_hist_kernel<2><<<grid, kThreads, 0, st>>>(w, ens, N);
+  topk_eqcount_kernel<<<grid, kThreads, 0, st>>>(w, ens, N, nblk);
+  topk_mask_kernel<<<grid, kThreads, 0, st>>>(w, ens, N, nblk, keep);
+  for (int i = 0; i < 6; ++i) note_launch();
+  return check_launch();
+}
+
+}  // namespace fm

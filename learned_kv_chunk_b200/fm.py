@@ -1,0 +1,322 @@
+"""Thin Python binding of libfm (ctypes).  Argument marshalling only: every
+step of the retriever path runs in the library's CUDA kernels.  torch is used
+for device memory and the current stream.
+
+The functions carry the C ABI's names (include/fm.h); `Retriever` bundles a
+context with its weights for convenience.  If libfm.so is missing, importing
+this module raises: there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libfm.so")
+
+FM_OK, FM_ERR_INVALID_ARG, FM_ERR_ALIGNMENT, FM_ERR_UNSUPPORTED = 0, 1, 2, 3
+FM_ERR_CUDA, FM_ERR_OOM, FM_ERR_DEVICE = 4, 5, 6
+FM_ENSEMBLE_MAX, FM_ENSEMBLE_MEAN = 0, 1
+MODES = {"max": FM_ENSEMBLE_MAX, "mean": FM_ENSEMBLE_MEAN}
+
+
+class fm_config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("q_lora_rank", ctypes.c_int),
+                ("n_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("n_layers", ctypes.c_int), ("rope_dim", ctypes.c_int),
+                ("rope_base", ctypes.c_double), ("rope_factor", ctypes.c_double),
+                ("rope_orig_max_pos", ctypes.c_double), ("rope_beta_fast", ctypes.c_double),
+                ("rope_beta_slow", ctypes.c_double), ("rms_eps", ctypes.c_float),
+                ("max_batch", ctypes.c_int), ("q_pieces", ctypes.c_int)]
+
+
+class fm_layer_weights(ctypes.Structure):
+    _fields_ = [("wq_a", ctypes.c_void_p), ("q_norm", ctypes.c_void_p),
+                ("wq_b", ctypes.c_void_p), ("weights_proj", ctypes.c_void_p)]
+
+
+class FMError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.fm_strerror(status).decode() if _lib is not None else str(status)
+        extra = ""
+        if status == FM_ERR_CUDA:
+            extra = f" (cudaError {_lib.fm_last_cuda_error()})"
+        super().__init__(f"{where}: {msg}{extra}")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libfm.so not built at {LIB_PATH}; run `python -m learned_kv_chunk_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "fm_config_default": (None, [ctypes.POINTER(fm_config)]),
+        "fm_create": (I, [ctypes.POINTER(fm_config), ctypes.POINTER(fm_layer_weights), I,
+                          ctypes.POINTER(P)]),
+        "fm_destroy": (I, [P]),
+        "fm_query_prep": (I, [P, P, P, I, P, P, P]),
+        "fm_score": (I, [P, P, I64, P, I, I, P, P, P, P]),
+        "fm_ensemble": (I, [P, I, I, I, I, P, P]),
+        "fm_score_fused": (I, [P, P, I64, P, I, I, P, P, I, F, P, P, P, P]),
+        "fm_topk_workspace_bytes": (S, [I, I]),
+        "fm_select_topk": (I, [P, P, I, I, I, P, P, S, P]),
+        "fm_select_threshold": (I, [P, P, I, I, F, P, P]),
+        "fm_sync_status": (I, [P, P]),
+        "fm_strerror": (ctypes.c_char_p, [I]),
+        "fm_last_cuda_error": (I, []),
+        "fm_launch_count": (ctypes.c_uint64, []),
+        "fm_debug_tile_dots": (I, [P, P, I64, I, I, P, P, I, I, I, P, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != FM_OK:
+        raise FMError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def fm_config_default() -> fm_config:
+    c = fm_config()
+    _lib.fm_config_default(ctypes.byref(c))
+    return c
+
+
+def fm_launch_count() -> int:
+    return int(_lib.fm_launch_count())
+
+
+def fm_topk_workspace_bytes(B: int, N: int) -> int:
+    return int(_lib.fm_topk_workspace_bytes(B, N))
+
+
+def _comp_k_array(comp_k: Sequence[torch.Tensor]):
+    for i, t in enumerate(comp_k):
+        _need(t, torch.uint8, f"comp_k[{i}]")
+    return (ctypes.c_void_p * len(comp_k))(*[t.data_ptr() for t in comp_k])
+
+
+def _keys_shape(comp_k: Sequence[torch.Tensor], N: Optional[int]):
+    B, N_pad, rec = comp_k[0].shape
+    if rec != 132:
+        raise ValueError("compressed keys must be [B, N, 132] uint8")
+    for t in comp_k:
+        if tuple(t.shape) != (B, N_pad, rec):
+            raise ValueError("every layer's keys must have the same shape")
+    N = N_pad if N is None else N
+    return B, N, N_pad * 132
+
+
+def fm_ensemble(scores: torch.Tensor, mode: str = "max", out: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    _need(scores, torch.float32, "scores")
+    L, B, N = scores.shape
+    ens = out if out is not None else torch.empty(B, N, device=scores.device, dtype=torch.float32)
+    _check(_lib.fm_ensemble(_ptr(scores), L, B, N, MODES[mode], _ptr(ens), _stream(stream)),
+           "fm_ensemble")
+    return ens
+
+
+def fm_select_topk(ens: torch.Tensor, k: int, n_valid: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    _need(ens, torch.float32, "ens")
+    B, N = ens.shape
+    if n_valid is not None:
+        _need(n_valid, torch.int32, "n_valid")
+    keep = out if out is not None else torch.empty(B, N, device=ens.device, dtype=torch.bool)
+    nbytes = fm_topk_workspace_bytes(B, N)
+    ws = workspace if workspace is not None else torch.empty(nbytes, device=ens.device, dtype=torch.uint8)
+    _check(_lib.fm_select_topk(_ptr(ens), _ptr(n_valid), B, N, int(k), _ptr(keep), _ptr(ws),
+                               ws.numel(), _stream(stream)), "fm_select_topk")
+    return keep
+
+
+def fm_select_threshold(ens: torch.Tensor, thr: float, n_valid: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _need(ens, torch.float32, "ens")
+    B, N = ens.shape
+    if n_valid is not None:
+        _need(n_valid, torch.int32, "n_valid")
+    keep = out if out is not None else torch.empty(B, N, device=ens.device, dtype=torch.bool)
+    _check(_lib.fm_select_threshold(_ptr(ens), _ptr(n_valid), B, N, float(thr), _ptr(keep),
+                                    _stream(stream)), "fm_select_threshold")
+    return keep
+
+
+class Retriever:
+    """A libfm context: the three CSA layers' weights on one device.
+
+    weights: list (one per layer) of dicts with fp32 tensors wq_a [R, HID],
+    q_norm [R], wq_b [H*D, R], weights_proj [H, HID] (CPU or CUDA)."""
+
+    def __init__(self, weights: List[dict], device: int = 0, max_batch: int = 64,
+                 q_pieces: int = 3, **overrides):
+        cfg = fm_config_default()
+        cfg.n_layers = len(weights)
+        cfg.max_batch = max_batch
+        cfg.q_pieces = q_pieces
+        for k, v in overrides.items():
+            setattr(cfg, k, v)
+        self.cfg = cfg
+        self.device = device
+        keep = []
+        arr = (fm_layer_weights * len(weights))()
+        for i, w in enumerate(weights):
+            ts = {k: w[k].detach().to(torch.float32).contiguous() for k in
+                  ("wq_a", "q_norm", "wq_b", "weights_proj")}
+            keep.append(ts)
+            arr[i] = fm_layer_weights(*[ts[k].data_ptr() for k in ("wq_a", "q_norm", "wq_b", "weights_proj")])
+        h = ctypes.c_void_p()
+        _check(_lib.fm_create(ctypes.byref(cfg), arr, device, ctypes.byref(h)), "fm_create")
+        self._h = h
+        self.L = cfg.n_layers
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.fm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def handle(self):
+        return self._h
+
+    def fm_query_prep(self, hidden: torch.Tensor, positions: torch.Tensor, q=None, fused_w=None,
+                      stream=None):
+        _need(hidden, torch.float32, "hidden")
+        _need(positions, torch.int64, "positions")
+        B = hidden.shape[0]
+        dev = hidden.device
+        q = q if q is not None else torch.empty(B, self.L, 64, 128, device=dev, dtype=torch.float32)
+        fused_w = fused_w if fused_w is not None else torch.empty(B, self.L, 64, device=dev, dtype=torch.float32)
+        _check(_lib.fm_query_prep(self._h, _ptr(hidden), _ptr(positions), B, _ptr(q), _ptr(fused_w),
+                                  _stream(stream)), "fm_query_prep")
+        return q, fused_w
+
+    def fm_score(self, comp_k: Sequence[torch.Tensor], q: torch.Tensor, fused_w: torch.Tensor,
+                 n_valid: Optional[torch.Tensor] = None, N: Optional[int] = None, out=None,
+                 stream=None) -> torch.Tensor:
+        B, N, stride = _keys_shape(comp_k, N)
+        arr = _comp_k_array(comp_k)
+        _need(q, torch.float32, "q")
+        _need(fused_w, torch.float32, "fused_w")
+        if n_valid is not None:
+            _need(n_valid, torch.int32, "n_valid")
+        scores = out if out is not None else torch.empty(self.L, B, N, device=q.device, dtype=torch.float32)
+        _check(_lib.fm_score(self._h, arr, stride, _ptr(n_valid), B, N, _ptr(q), _ptr(fused_w),
+                             _ptr(scores), _stream(stream)), "fm_score")
+        return scores
+
+    def fm_score_fused(self, comp_k: Sequence[torch.Tensor], q: torch.Tensor, fused_w: torch.Tensor,
+                       mode: str = "max", threshold: Optional[float] = None,
+                       n_valid: Optional[torch.Tensor] = None, N: Optional[int] = None,
+                       want_layers: bool = False, ens=None, keep_thr=None, scores=None, stream=None):
+        B, N, stride = _keys_shape(comp_k, N)
+        arr = _comp_k_array(comp_k)
+        _need(q, torch.float32, "q")
+        _need(fused_w, torch.float32, "fused_w")
+        if n_valid is not None:
+            _need(n_valid, torch.int32, "n_valid")
+        dev = q.device
+        ens = ens if ens is not None else torch.empty(B, N, device=dev, dtype=torch.float32)
+        if threshold is not None and keep_thr is None:
+            keep_thr = torch.empty(B, N, device=dev, dtype=torch.bool)
+        if want_layers and scores is None:
+            scores = torch.empty(self.L, B, N, device=dev, dtype=torch.float32)
+        thr = 0.0 if threshold is None else float(threshold)
+        _check(_lib.fm_score_fused(self._h, arr, stride, _ptr(n_valid), B, N, _ptr(q), _ptr(fused_w),
+                                   MODES[mode], thr, _ptr(scores), _ptr(ens),
+                                   _ptr(keep_thr if threshold is not None else None),
+                                   _stream(stream)), "fm_score_fused")
+        return ens, keep_thr, scores
+
+    def fm_sync_status(self, stream=None):
+        _check(_lib.fm_sync_status(self._h, _stream(stream)), "fm_sync_status")
+
+    def fm_debug_tile_dots(self, comp_k, q, fused_w, layer: int, b: int, t: int, N=None):
+        B, N, stride = _keys_shape(comp_k, N)
+        arr = _comp_k_array(comp_k)
+        P = self.cfg.q_pieces
+        out = torch.full((128, P * 64), float("nan"), device=q.device, dtype=torch.float32)
+        e = torch.zeros(64, device=q.device, dtype=torch.int32)
+        _check(_lib.fm_debug_tile_dots(self._h, arr, stride, B, N, _ptr(q), _ptr(fused_w), layer, b, t,
+                                       _ptr(out), _ptr(e), _stream()), "fm_debug_tile_dots")
+        return out, e
+
+    def retrieve_from_host(self, hidden, positions, comp_k, n_valid=None, mode="max", top_k=None,
+                           threshold=None, N=None, device_buffers: Optional[dict] = None):
+        """The whole path for inputs that live in (pinned) host memory: copies
+        them to device buffers, runs retrieve() and copies the keep masks back.
+        Returns (keep_topk, keep_thr) as host tensors (either may be None)."""
+        dev = torch.device("cuda", self.device)
+        buf = device_buffers if device_buffers is not None else {}
+        def stage(name, t):
+            d = buf.get(name)
+            if d is None or d.shape != t.shape or d.dtype != t.dtype:
+                d = buf[name] = torch.empty(t.shape, dtype=t.dtype, device=dev)
+            d.copy_(t, non_blocking=True)
+            return d
+        h = stage("hidden", hidden)
+        p = stage("positions", positions)
+        keys = [stage(f"keys{l}", t) for l, t in enumerate(comp_k)]
+        nv = stage("n_valid", n_valid) if n_valid is not None else None
+        ens, keep_topk, keep_thr = self.retrieve(h, keys, p, nv, mode, top_k, threshold, N)
+        out = []
+        for name, t in (("out_topk", keep_topk), ("out_thr", keep_thr)):
+            if t is None:
+                out.append(None)
+                continue
+            o = buf.get(name)
+            if o is None or o.shape != t.shape:
+                o = buf[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            o.copy_(t, non_blocking=True)
+            out.append(o)
+        torch.cuda.current_stream().synchronize()
+        return out[0], out[1]
+
+    # the pages' calls, composed (README "Usage")
+    def retrieve(self, hidden, comp_k, positions, n_valid=None, mode="max", top_k=None,
+                 threshold=None, N=None):
+        q, w = self.fm_query_prep(hidden, positions)
+        ens, keep_thr, _ = self.fm_score_fused(comp_k, q, w, mode=mode, threshold=threshold,
+                                               n_valid=n_valid, N=N)
+        keep_topk = fm_select_topk(ens, top_k, n_valid) if top_k is not None else None
+        return ens, keep_topk, keep_thr

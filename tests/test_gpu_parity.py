@@ -1,0 +1,199 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on small
+cases that span several 128-chunk tiles and ragged tails."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.retriever as O
+from gen import synthetic as G
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from learned_kv_chunk_b200 import fm  # noqa: E402  (loads libfm.so; raises if missing)
+
+DEV = torch.device("cuda", 0)
+
+
+@pytest.fixture(scope="module")
+def weights():
+    return G.make_weights(4242, 3)
+
+
+@pytest.fixture(scope="module", params=[3, 2], ids=["pieces3", "pieces2"])
+def retr(request, weights):
+    r = fm.Retriever(weights, device=0, max_batch=64, q_pieces=request.param)
+    yield r
+    r.close()
+
+
+def _dev(ts):
+    return [t.to(DEV) for t in ts]
+
+
+def _run_query(r, case):
+    q, w = r.fm_query_prep(case.hidden.to(DEV), case.positions.to(DEV))
+    torch.cuda.synchronize()
+    return q, w
+
+
+def test_query_prep_matches_oracle(retr, weights):
+    case = H.make_case(5, 256, [256] * 5, seed=11, weights=weights,
+                       positions=[0, 1, 16384, 1 << 18, 1 << 20])
+    q, w = _run_query(retr, case)
+    q = q.cpu().numpy().astype(np.float64)
+    w = w.cpu().numpy().astype(np.float64)
+    nrm = np.linalg.norm(case.q_o, axis=-1, keepdims=True)
+    err = np.linalg.norm(q - case.q_o, axis=-1, keepdims=True) / nrm
+    assert err.max() < 2e-5, err.max()
+    np.testing.assert_allclose(w, case.w_o, rtol=1e-4, atol=1e-6)
+    retr.fm_sync_status()
+
+
+def test_tile_dot_products_layout(retr, weights):
+    """Raw tensor-core dots of one tile against exact fp64 dots of the e4m3
+    codes with the query: checks the A/B operand layouts and the pieces."""
+    case = H.make_case(2, 640, [640, 640], seed=12, weights=weights)
+    keys = _dev(case.comp_k)
+    q, w = _run_query(retr, case)
+    P = retr.cfg.q_pieces
+    qh = q.cpu().numpy().astype(np.float64)
+    for (l, b, t) in [(0, 0, 0), (2, 1, 3), (1, 0, 4)]:
+        out, e = retr.fm_debug_tile_dots(keys, q, w, l, b, t)
+        torch.cuda.synchronize()
+        out = out.cpu().numpy().astype(np.float64)
+        e = e.cpu().numpy()
+        codes = case.comp_k[l][b, t * 128:(t + 1) * 128, :128].numpy()
+        kv = O.e4m3_decode(codes).astype(np.float64)             # [128, 128]
+        exact = kv @ qh[b, l].T                                    # [128, 64]
+        rec = np.zeros((128, 64))
+        for p in range(P):
+            rec += out[:, p * 64:(p + 1) * 64] * 16.0 ** (-p)
+        rec *= 2.0 ** (-e[None, :].astype(np.float64))
+        # split error: 2^-4P relative per query element, plus the e4m3
+        # subnormal floor of the last piece; doubled for fp32 accumulation
+        floor = 2.0 ** (-10 - 4 * (P - 1)) * 2.0 ** (-e.astype(np.float64))
+        bound = (np.abs(kv) @ np.abs(qh[b, l]).T * 2.0 ** (-4 * P)
+                 + np.abs(kv).sum(1, keepdims=True) * floor[None, :]) * 2 + 1e-6
+        assert np.all(np.abs(rec - exact) <= bound), np.abs(rec - exact).max()
+
+
+@pytest.mark.parametrize("shape", [
+    dict(B=1, N=4096, nv=[4096]),
+    dict(B=3, N=1001, nv=[1001, 517, 0]),
+    dict(B=4, N=700, nv=[1, 127, 128, 700]),
+])
+def test_scores_match_oracle(retr, weights, shape):
+    case = H.make_case(shape["B"], shape["N"], shape["nv"], seed=13, weights=weights)
+    keys = _dev(case.comp_k)
+    q, w = _run_query(retr, case)
+    nv = case.n_valid.to(DEV)
+    scores = retr.fm_score(keys, q, w, n_valid=nv, N=case.N)
+    torch.cuda.synchronize()
+    s_gpu = scores.cpu().numpy().astype(np.float64)
+    s_o = H.oracle_scores(case)
+    err = np.abs(s_gpu - s_o)
+    assert err.max() <= H.SCORE_TOL, err.max()
+    # exact zeros past each row's valid length
+    for b in range(shape["B"]):
+        assert np.all(s_gpu[:, b, int(case.n_valid[b]):] == 0.0)
+    assert np.all((s_gpu >= 0) & (s_gpu <= 1))
+    retr.fm_sync_status()
+
+
+@pytest.mark.parametrize("mode,thr", [("max", None), ("mean", 0.5)])
+def test_fused_pass_ensemble_and_masks(retr, weights, mode, thr):
+    case = H.make_case(3, 2000, [2000, 1500, 333], seed=14, weights=weights)
+    keys = _dev(case.comp_k)
+    q, w = _run_query(retr, case)
+    nv = case.n_valid.to(DEV)
+    ens, keep_thr, scores = retr.fm_score_fused(keys, q, w, mode=mode, threshold=thr, n_valid=nv,
+                                                N=case.N, want_layers=True)
+    keep = fm.fm_select_topk(ens, 100, nv)
+    torch.cuda.synchronize()
+    s_o = H.oracle_scores(case)
+    e_o = O.ensemble(s_o, mode)
+    e_gpu = ens.cpu().numpy()
+    assert np.abs(e_gpu - e_o).max() <= H.SCORE_TOL
+    assert np.abs(scores.cpu().numpy() - s_o).max() <= H.SCORE_TOL
+    # the fused ensemble equals the standalone ensemble of the same per-layer scores
+    ens2 = fm.fm_ensemble(scores, mode)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(ens2.cpu().numpy(), e_gpu)
+    H.check_topk_against_rule(keep.cpu().numpy(), e_gpu, case.n_valid.numpy(), 100)
+    H.check_topk_near_oracle(keep.cpu().numpy(), e_o, case.n_valid.numpy(), 100)
+    if thr is not None:
+        expect = O.select_threshold(e_gpu, case.n_valid.numpy(), thr)
+        np.testing.assert_array_equal(keep_thr.cpu().numpy(), expect)
+    if mode == "max":
+        assert np.all(e_gpu[None] >= scores.cpu().numpy())
+
+
+def test_zero_scale_records_score_one_half(retr, weights):
+    case = H.make_case(1, 300, [300], seed=15, weights=weights)
+    for t in case.comp_k:
+        t[0, 5:40, 128:132] = 0      # scale 0.0f -> k = 0 -> sigmoid(0)
+    keys = _dev(case.comp_k)
+    q, w = _run_query(retr, case)
+    s = retr.fm_score(keys, q, w).cpu().numpy()
+    assert np.all(s[:, 0, 5:40] == 0.5)
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_topk_exact_rule(ties):
+    g = torch.Generator().manual_seed(5)
+    B, N = 6, 50000
+    if ties:
+        ens = torch.randint(0, 40, (B, N), generator=g).float() / 40.0
+    else:
+        ens = torch.rand(B, N, generator=g)
+    nv = torch.tensor([N, 49999, 1, 0, 20000, 4096], dtype=torch.int32)
+    for k in (1, 7, 4096, 30000, 60000):
+        keep = fm.fm_select_topk(ens.to(DEV), k, nv.to(DEV))
+        torch.cuda.synchronize()
+        H.check_topk_against_rule(keep.cpu().numpy(), ens.numpy(), nv.numpy(), k)
+
+
+def test_topk_all_equal_and_no_n_valid():
+    ens = torch.full((2, 10000), 0.5)
+    keep = fm.fm_select_topk(ens.to(DEV), 333).cpu().numpy()
+    assert keep[0, :333].all() and not keep[0, 333:].any() and keep.sum() == 666
+
+
+def test_threshold_and_ensemble_kernels():
+    g = torch.Generator().manual_seed(6)
+    s = (torch.randint(0, 9, (3, 4, 777), generator=g).float() / 8.0)
+    nv = torch.tensor([777, 0, 5, 400], dtype=torch.int32)
+    for mode in ("max", "mean"):
+        e = fm.fm_ensemble(s.to(DEV), mode).cpu().numpy()
+        np.testing.assert_allclose(e, O.ensemble(s.numpy(), mode), rtol=1e-6, atol=1e-7)
+        keep = fm.fm_select_threshold(torch.from_numpy(e).to(DEV), 0.5, nv.to(DEV)).cpu().numpy()
+        np.testing.assert_array_equal(keep, O.select_threshold(e, nv.numpy(), 0.5))
+
+
+def test_argument_errors(retr, weights):
+    case = H.make_case(2, 256, [256, 256], seed=16, weights=weights)
+    keys = _dev(case.comp_k)
+    q, w = _run_query(retr, case)
+    lib = fm.lib()
+    import ctypes
+    arr = (ctypes.c_void_p * 3)(*[k.data_ptr() for k in keys])
+    bad = (ctypes.c_void_p * 3)(*[k.data_ptr() + 4 for k in keys])
+    out = torch.empty(3, 2, 256, device=DEV)
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    assert lib.fm_score(retr.handle, bad, 256 * 132, None, 2, 256, P(q), P(w), P(out), st) == fm.FM_ERR_ALIGNMENT
+    assert lib.fm_score(retr.handle, arr, 255 * 132, None, 2, 256, P(q), P(w), P(out), st) != fm.FM_OK
+    assert lib.fm_score(retr.handle, arr, 256 * 132, None, 65, 256, P(q), P(w), P(out), st) == fm.FM_ERR_INVALID_ARG
+    assert lib.fm_score(retr.handle, arr, 256 * 132, None, 2, 0, P(q), P(w), P(out), st) == fm.FM_ERR_INVALID_ARG
+    ens = torch.zeros(2, 256, device=DEV)
+    keep = torch.zeros(2, 256, device=DEV, dtype=torch.uint8)
+    ws = torch.zeros(fm.fm_topk_workspace_bytes(2, 256), device=DEV, dtype=torch.uint8)
+    assert lib.fm_select_topk(P(ens), None, 2, 256, 0, P(keep), P(ws), ws.numel(), st) == fm.FM_ERR_INVALID_ARG
+    assert lib.fm_select_topk(P(ens), None, 2, 256, 5, P(keep), P(ws), 16, st) == fm.FM_ERR_INVALID_ARG
+    assert lib.fm_score_fused(retr.handle, arr, 256 * 132, None, 2, 256, P(q), P(w), 7, 0.0, None,
+                              P(ens), None, st) == fm.FM_ERR_INVALID_ARG
+    retr.fm_sync_status()
