@@ -71,6 +71,7 @@ struct ScoreArgs {
   uint8_t* keep_thr;       // [B, N] or null
   float thr;
   int mode;                // FM_ENSEMBLE_*
+  int prefetch_units;      // (row, tile) units the key loader prefetches into L2 ahead
   int* err;
   // diagnostic dump of one tile's raw accumulators
   float* dbg_out;          // [128, P*64] or null
@@ -148,6 +149,23 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Waits for a phase that an asynchronous operation this CTA issued will
+// complete (a bulk copy landing, an MMA commit arriving) before the CTA may
+// exit.  Ignores the abort flag -- the operation is in flight whatever else
+// failed -- and gives up only after `limit_ns`, recording kDevErrTimeout.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int* err,
+                                           uint64_t limit_ns = 200000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0 && global_timer_ns() - t0 > limit_ns) {
+      atomicExch(err, kDevErrTimeout);
+      return false;
+    }
+  }
+}
+
 // 1-D bulk copy global -> shared through the TMA engine, completing on `bar`
 // (transaction bytes).  dst, src and bytes must be multiples of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
@@ -166,6 +184,12 @@ __device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32
       "[%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+
+// Prefetch [src, src + bytes) from global memory into L2 (bulk, no shared
+// memory involved).  src and bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {
@@ -224,24 +248,112 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
       : "memory");
 }
 
-// 32 lanes x 32 consecutive fp32 columns; thread i gets lane (base_lane + i).
-__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, float* v) {
-  uint32_t r[32];
+// tcgen05.ld writes its destination registers asynchronously: they hold the
+// data only after tcgen05.wait::ld.  The loads and the wait are therefore
+// issued in ONE asm statement, so the compiler never sees the registers as
+// defined (and never copies or reuses them) before the data has landed.
+#define FM_TMEM_REGS32(p)                                                                   \
+  "=r"(p[0]), "=r"(p[1]), "=r"(p[2]), "=r"(p[3]), "=r"(p[4]), "=r"(p[5]), "=r"(p[6]),     \
+      "=r"(p[7]), "=r"(p[8]), "=r"(p[9]), "=r"(p[10]), "=r"(p[11]), "=r"(p[12]),          \
+      "=r"(p[13]), "=r"(p[14]), "=r"(p[15]), "=r"(p[16]), "=r"(p[17]), "=r"(p[18]),       \
+      "=r"(p[19]), "=r"(p[20]), "=r"(p[21]), "=r"(p[22]), "=r"(p[23]), "=r"(p[24]),       \
+      "=r"(p[25]), "=r"(p[26]), "=r"(p[27]), "=r"(p[28]), "=r"(p[29]), "=r"(p[30]),       \
+      "=r"(p[31])
+
+// 32 lanes x 32 consecutive fp32 columns at taddr (thread i gets lane base+i), waited.
+__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t* a) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : FM_TMEM_REGS32(a)
+      : "r"(taddr)
+      : "memory");
 }
-__device__ __forceinline__ void tmem_ld_wait() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+
+// Two 32-column loads (taddr0, taddr1) and one wait.
+__device__ __forceinline__ void tmem_ld32x2_wait(uint32_t t0, uint32_t t1, uint32_t* a,
+                                                 uint32_t* b) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : FM_TMEM_REGS32(a), FM_TMEM_REGS32(b)
+      : "r"(t0), "r"(t1)
+      : "memory");
+}
+
+// Three 32-column loads and one wait.
+__device__ __forceinline__ void tmem_ld32x3_wait(uint32_t t0, uint32_t t1, uint32_t t2,
+                                                 uint32_t* a, uint32_t* b, uint32_t* c) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%96];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%97];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
+      "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95}, [%98];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : FM_TMEM_REGS32(a), FM_TMEM_REGS32(b), FM_TMEM_REGS32(c)
+      : "r"(t0), "r"(t1), "r"(t2)
+      : "memory");
+}
+
+// 16-column variants: P loads of 32 lanes x 16 fp32 columns, then one wait.
+#define FM_TMEM_REGS16(p)                                                                  \
+  "=r"(p[0]), "=r"(p[1]), "=r"(p[2]), "=r"(p[3]), "=r"(p[4]), "=r"(p[5]), "=r"(p[6]),    \
+      "=r"(p[7]), "=r"(p[8]), "=r"(p[9]), "=r"(p[10]), "=r"(p[11]), "=r"(p[12]),         \
+      "=r"(p[13]), "=r"(p[14]), "=r"(p[15])
+
+__device__ __forceinline__ void tmem_ld16x2_wait(uint32_t t0, uint32_t t1, uint32_t* a,
+                                                 uint32_t* b) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : FM_TMEM_REGS16(a), FM_TMEM_REGS16(b)
+      : "r"(t0), "r"(t1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16x3_wait(uint32_t t0, uint32_t t1, uint32_t t2,
+                                                 uint32_t* a, uint32_t* b, uint32_t* c) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%48];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%49];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47}, [%50];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : FM_TMEM_REGS16(a), FM_TMEM_REGS16(b), FM_TMEM_REGS16(c)
+      : "r"(t0), "r"(t1), "r"(t2)
+      : "memory");
+}
+
+// Packed fp32x2 arithmetic (sm_100): one instruction for two lanes of data.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
 }
 
 // Shared-memory matrix descriptor for a K-major operand stored in the

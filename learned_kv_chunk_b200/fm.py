@@ -15,7 +15,7 @@ from typing import List, Optional, Sequence
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "lib", "libfm.so")
+LIB_PATH = os.environ.get("FM_LIBRARY_PATH") or os.path.join(_PKG, "lib", "libfm.so")
 
 FM_OK, FM_ERR_INVALID_ARG, FM_ERR_ALIGNMENT, FM_ERR_UNSUPPORTED = 0, 1, 2, 3
 FM_ERR_CUDA, FM_ERR_OOM, FM_ERR_DEVICE = 4, 5, 6
