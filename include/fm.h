@@ -172,6 +172,31 @@ size_t fm_topk_workspace_bytes(int B, int N);
 fm_status fm_select_topk(const float* ens, const int32_t* n_valid, int B, int N, int k,
                          uint8_t* keep, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Size of the scratch array fm_select_topk_static uses: 4 MiB, compiled into
+ * the library, one per GPU that loads it, held until the process exits.  It
+ * covers fm_topk_workspace_bytes(B, N) up to about 200 rows of 262144 chunks. */
+#define FM_TOPK_STATIC_SCRATCH_BYTES (4u << 20)
+
+/* fm_select_topk for callers that cannot allocate device memory: the same
+ * keep mask, with the scratch taken from a fixed array inside the library
+ * instead of a caller workspace.  The paper has no counterpart; this is an
+ * integration entry point.  Callers that need it: a serving process whose
+ * device memory is all handed to its KV-cache pool at start-up, a plugin that
+ * must leave device memory to its host framework's allocator, a decode loop
+ * that cannot afford the device synchronisation cudaMalloc/cudaFree may cause.
+ * Allocates nothing; the caller passes inputs and outputs as for
+ * fm_select_topk (ens, n_valid, keep: device; same shapes and rules).
+ * Runs on the calling thread's current device, which must own `stream`; the
+ * first call on each device looks up the array's device address (with
+ * cudaGetSymbolAddress) and caches it, so make that first call before any
+ * stream capture.  Every call on a device shares the one array and the call's
+ * first kernel re-initialises what it uses: calls whose kernels overlap on the
+ * GPU (different streams or threads) race and give wrong masks; order them.
+ * Returns FM_ERR_UNSUPPORTED, launching nothing, when
+ * fm_topk_workspace_bytes(B, N) > FM_TOPK_STATIC_SCRATCH_BYTES. */
+fm_status fm_select_topk_static(const float* ens, const int32_t* n_valid, int B, int N, int k,
+                                uint8_t* keep, cudaStream_t stream);
+
 /* Threshold keep mask (README "Usage" select_topk(threshold=t)):
  * keep[b,n] = (n < n_b) && (ens[b,n] > thr).  Shapes as fm_select_topk. */
 fm_status fm_select_threshold(const float* ens, const int32_t* n_valid, int B, int N, float thr,

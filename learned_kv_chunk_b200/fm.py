@@ -65,6 +65,7 @@ def _load():
         "fm_topk_workspace_bytes": (S, [I, I]),
         "fm_select_topk": (I, [P, P, I, I, I, P, P, S, P]),
         "fm_select_threshold": (I, [P, P, I, I, F, P, P]),
+        "fm_select_topk_static": (I, [P, P, I, I, I, P, P]),
         "fm_sync_status": (I, [P, P]),
         "fm_strerror": (ctypes.c_char_p, [I]),
         "fm_last_cuda_error": (I, []),
@@ -161,6 +162,21 @@ def fm_select_topk(ens: torch.Tensor, k: int, n_valid: Optional[torch.Tensor] = 
     ws = workspace if workspace is not None else torch.empty(nbytes, device=ens.device, dtype=torch.uint8)
     _check(_lib.fm_select_topk(_ptr(ens), _ptr(n_valid), B, N, int(k), _ptr(keep), _ptr(ws),
                                ws.numel(), _stream(stream)), "fm_select_topk")
+    return keep
+
+
+def fm_select_topk_static(ens: torch.Tensor, k: int, n_valid: Optional[torch.Tensor] = None,
+                          out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """fm_select_topk without a workspace: the library's fixed scratch array
+    is used, so the C call allocates nothing (for callers that cannot
+    allocate device memory).  Pass `out` to allocate nothing here either."""
+    _need(ens, torch.float32, "ens")
+    B, N = ens.shape
+    if n_valid is not None:
+        _need(n_valid, torch.int32, "n_valid")
+    keep = out if out is not None else torch.empty(B, N, device=ens.device, dtype=torch.bool)
+    _check(_lib.fm_select_topk_static(_ptr(ens), _ptr(n_valid), B, N, int(k), _ptr(keep),
+                                      _stream(stream)), "fm_select_topk_static")
     return keep
 
 
