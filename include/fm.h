@@ -216,14 +216,16 @@ int fm_last_cuda_error(void);
 /* Number of kernel launches issued by this process since load (all calls). */
 uint64_t fm_launch_count(void);
 
-/* Diagnostic: the raw tensor-core dot products of one 128-chunk tile of layer
- * `layer`, row b, tile t (chunks t*128 .. t*128+127), before the per-chunk
- * scale, the per-head power-of-two scale and the epilogue:
- *   out[r, p*64 + h] = sum_d e4m3(comp_k[layer][b, t*128 + r, d]) * piece_p(q[b,layer,h])[d]
+/* Diagnostic: the raw tensor-core dot products of one 96-chunk tile of layer
+ * `layer`, row b, tile t (chunks t*96 .. t*96+95), before the per-chunk
+ * scale, the per-head power-of-two scale and the epilogue, for r < 96 and
+ * p < q_pieces:
+ *   out[r, p*64 + h] = sum_d e4m3(comp_k[layer][b, t*96 + r, d]) * piece_p(q[b,layer,h])[d]
  * where the query pieces satisfy
  *   q[b,layer,h,d] ~= 2^-pow2_exp[h] * sum_p 16^-p * piece_p[d].
- * out [128, q_pieces*64] fp32 device (written), pow2_exp [64] int32 device
- * (written).  Rows of the tile past N hold unspecified values.  Used by the
+ * out [128, 192] fp32 device (the entries above written, the rest untouched),
+ * pow2_exp [64] int32 device (written).  Rows of the tile past N
+ * hold unspecified values.  Used by the
  * tests to check the tensor-core operand layouts in isolation. */
 fm_status fm_debug_tile_dots(fm_ctx* ctx, const uint8_t* const* comp_k, int64_t row_stride_bytes,
                              int B, int N, const float* q, const float* fused_w, int layer, int b,

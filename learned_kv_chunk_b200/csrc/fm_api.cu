@@ -236,8 +236,6 @@ static fm_status score_common(fm_ctx* c, const uint8_t* const* comp_k, int64_t r
   a.keep_thr = keep_thr;
   a.thr = thr;
   a.mode = mode;
-  a.prefetch_units = 0;
-  if (const char* e = std::getenv("FM_PREFETCH_UNITS")) a.prefetch_units = std::atoi(e);
   a.err = c->d_err;
   a.dbg_out = dbg_out;
   a.dbg_layer = dbg_layer;

@@ -17,7 +17,9 @@ constexpr int kHeads = 64;        // N_HEADS (the shipped value; checked at crea
 constexpr int kHeadDim = 128;     // HEAD_DIM (README "Architecture")
 constexpr int kRopeDim = 64;      // ROPE_DIM (README "Architecture")
 constexpr int kRecord = 132;      // bytes per compressed chunk (README "compressed_k format")
-constexpr int kTile = 128;        // chunks per tensor-core tile (MMA M)
+constexpr int kTile = 96;         // chunks per scored tile: TMEM lanes 0-31 and 64-127 of an
+                                  // M = 128 MMA (lanes 32-63, the quarter that only warps on the
+                                  // MMA issuer's scheduler can reach, stay unused)
 constexpr int kMaxLayers = 4;
 constexpr int kMaxBatch = 4096;
 
@@ -71,10 +73,9 @@ struct ScoreArgs {
   uint8_t* keep_thr;       // [B, N] or null
   float thr;
   int mode;                // FM_ENSEMBLE_*
-  int prefetch_units;      // (row, tile) units the key loader prefetches into L2 ahead
   int* err;
   // diagnostic dump of one tile's raw accumulators
-  float* dbg_out;          // [128, P*64] or null
+  float* dbg_out;          // [128, 128] or null
   int dbg_layer, dbg_b, dbg_t;
 };
 fm_status launch_score(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t stream);
@@ -237,6 +238,35 @@ __device__ __forceinline__ void umma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, ui
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, fp8 (kind::f8f6f4) inputs, fp32
+// accumulate.  A (M = 128 rows, K = 32 bytes) sits in TMEM: row r in lane r,
+// its 32 bytes in 8 consecutive 32-bit columns starting at a_tmem.
+__device__ __forceinline__ void umma_f8f6f4_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns from registers into TMEM at taddr
+// (thread i writes lane base+i), then waits until the store has completed.
+__device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
 

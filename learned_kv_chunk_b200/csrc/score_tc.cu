@@ -7,33 +7,43 @@
 // threshold keep rule (toy decode loop, "sigmoid > thresh").
 //
 // Design (sm_100a):
-//  * one persistent CTA per SM walks a contiguous range of (row, 128-chunk
-//    tile) units; each unit is scored for all L layers back to back (one
-//    "item" per layer) so the ensemble stays in registers and one fp32 per
-//    chunk is written;
+//  * one persistent CTA per SM walks a contiguous range of (row, 96-chunk
+//    tile) units; each unit is scored for all L layers (one "item" per layer)
+//    so the ensemble stays in registers and one fp32 per chunk is written;
 //  * the keys go to the tensor cores as stored: kind::f8f6f4 MMA with A = the
-//    128 e4m3 bytes of 128 records (M = 128 chunks, K = 128 dims) and B = the
-//    query split into P e4m3 pieces per head (N = P*64), fp32 accumulators in
-//    TMEM.  The per-chunk fp32 scale, the per-head power-of-two scale of the
-//    pieces, relu, the head-weighted sum and the sigmoid run in the epilogue;
+//    128 e4m3 bytes of each record (K = 128 dims) and B = the query split into
+//    P e4m3 pieces (N = P * 64: piece p of head h in column p*64 + h), fp32
+//    accumulators in TMEM -- four MMAs (the K steps) per item.  A tile holds
+//    96 chunks in TMEM lanes 0-31 and 64-127 of an M = 128 MMA; lanes 32-63
+//    stay unused (see the warp roles).  The per-chunk fp32 scale, the
+//    per-head power-of-two scale of the pieces, relu, the head-weighted sum
+//    and the sigmoid run in the epilogue;
 //  * the 132-byte records are not 16-byte aligned, so a tile is fetched with
-//    one 1-D bulk copy (TMA engine) of 128 * 132 bytes and re-laid in place,
-//    inside the same shared-memory stage, into the 128B-swizzled K-major
-//    operand layout by four transform warps (every warp reads all its rows
-//    before any warp writes: row r's destination [128r, 128r+128) overlaps
-//    only rows <= r of the source).  The stage goes back to the key loader
-//    when the MMA that read it retires, so the whole ring holds keys in
-//    flight -- about 170 KB per SM;
+//    one 1-D bulk copy (TMA engine) of 96 * 132 bytes into a shared-memory
+//    stage; three transform warps (one TMEM lane quarter each, one chunk row
+//    per thread) read each row with conflict-free 4-byte loads (row stride 33
+//    words) and store it into TMEM, where the MMA takes A from.  A stage goes
+//    back to the key loader as soon as it has been read, so the ring holds
+//    little besides keys in flight from HBM;
+//  * one thread issues every MMA, and its issue rate bounds the pass: each
+//    tcgen05.mma, commit or mbarrier probe it executes costs tens of cycles.
+//    So an item is four MMAs with descriptors advanced by constant adds, and
+//    the thread's scheduler is left to it alone: warp w runs on scheduler
+//    w % 4 and may only touch TMEM lanes 32*(w % 4) .. +31, and a warp
+//    issuing back-to-back FP32 work on the issuer's scheduler (1) starves
+//    tcgen05.mma issue (measured: 8 MMAs went from ~400 to ~1700 cycles; on
+//    the other schedulers such warps cost nothing).  Hence no chunk lives in
+//    lane quarter 1;
 //  * warp roles (16 warps): 0 key loader, 1 MMA issuer, 2 TMEM owner + query
-//    loader, 4-7 transform, 8-11 and 12-15 two epilogue groups (one TMEM lane
-//    quarter per warp, all 64 heads of a chunk row) that take alternate
-//    units.  Each group owns half of the accumulator stages, so every stage's
-//    phases are consumed in order by one group (a parity wait cannot tell
-//    phases two apart).  Each item crosses four mbarrier hand-offs (copy
-//    landed, operand ready, accumulator ready, accumulator free); every ring
-//    index is advanced incrementally, and the epilogue reads each chunk's
-//    scale from global memory (an L2 hit: the tile was fetched moments
-//    earlier) instead of through another ring.
+//    loader, 4, 6, 7 transform, {8, 10, 11} and {12, 14, 15} two epilogue
+//    groups (one lane quarter per warp, all 64 heads of a chunk row), each
+//    with one accumulator stage.  Units are taken in pairs from the same row,
+//    the first for group 0 and the second for group 1, and their items are
+//    issued layer by layer alternately, (u0,l0) (u1,l0) (u0,l1) (u1,l1) ...,
+//    so each group has a whole MMA to drain its stage before it is needed
+//    again.  Every ring index is advanced incrementally (no runtime division
+//    in any loop), and the epilogue reads each chunk's scale from global
+//    memory (an L2 hit: the tile was fetched moments earlier).
 #include <cstdlib>
 
 #include "fm_internal.cuh"
@@ -43,41 +53,51 @@ namespace {
 
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kRawBytes = kTile * kRecord;    // 16896
-constexpr int kStageBytes = 17408;           // one key stage: 16896 B rounded to 1 KB
-constexpr int kBarXform = 1;                 // named barrier id of the transform warps
+constexpr int kRawBytes = kTile * kRecord;  // 12672, a multiple of 128
+constexpr int kMmaM = 128;                  // MMA rows (TMEM lanes); chunks use lanes 0-31, 64-127
+constexpr int kQuarters = 3;                // TMEM lane quarters holding chunks: 0, 2, 3
 constexpr int kWarpLoader = 0, kWarpMma = 1, kWarpQ = 2;
-constexpr int kWarpXform0 = 4, kWarpEpi0 = 8;
+constexpr int kWarpXform0 = 4, kWarpEpi0 = 8;  // + 0, 2, 3 (scheduler 1 is left to the MMA issuer)
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kACols = 32;  // 128 e4m3 bytes per row = 32 columns per key tile
+constexpr uint32_t kPieceBytes = kHeads * kHeadDim;  // one query piece of one layer
+
+// TMEM columns: accumulator of group g at [g * P*64, (g+1) * P*64), key tiles after them.
+template <int P>
+constexpr uint32_t acc_cols() { return (uint32_t)P * kHeads; }
+template <int P>
+constexpr uint32_t a_col_base() { return 2u * acc_cols<P>(); }
+template <int P>
+constexpr uint32_t a_stages() { return (kTmemCols - a_col_base<P>()) / kACols; }  // 8 (P=2), 4 (P=3)
+
+// TMEM lane quarter q in {0, 2, 3} -> block of 32 tile rows (0, 1, 2).
+__device__ __forceinline__ int quarter_block(int q) { return q == 0 ? 0 : q - 1; }
 
 struct Layout {
-  int L, P, NR, NACC;
   uint32_t q_off, raw_off, wp_off, bar_off, misc_off, total;
 };
 
-__host__ __device__ inline Layout make_layout(int L, int P, int NR) {
+__host__ __device__ inline Layout make_layout(int L, int P, int NR, int NA) {
   Layout s;
-  s.L = L; s.P = P; s.NR = NR;
-  s.NACC = (P == 3) ? 2 : 4;  // accumulator stages of P*64 TMEM columns (<= 512)
   uint32_t o = 0;
-  s.q_off = o;    o += (uint32_t)L * P * kHeads * kHeadDim;           // multiple of 1024
-  s.raw_off = o;  o += (uint32_t)NR * kStageBytes;                     // 1024-aligned stages
-  s.wp_off = o;   o += 8u * (uint32_t)L * kHeads * 4;                 // per epilogue warp
+  s.q_off = o;    o += (uint32_t)L * P * kPieceBytes;                  // multiple of 1024
+  s.raw_off = o;  o += (uint32_t)NR * kRawBytes;                       // 128-aligned stages
+  s.wp_off = o;   o += 2u * kQuarters * (uint32_t)L * kHeads * 4;     // per epilogue warp
   o = (o + 7u) & ~7u;
-  s.bar_off = o;  o += (uint32_t)(3 * NR + 2 * s.NACC + 3) * 8;
+  s.bar_off = o;  o += (uint32_t)(2 * NR + 2 * NA + 4 + 3) * 8;
   s.misc_off = o; o += 64;
   s.total = o + 1024;  // slack to align the base to 1024
   return s;
 }
 
 struct Bars {
-  uint64_t *raw_full, *raw_empty, *a_full, *acc_full, *acc_empty, *q_full, *q_empty, *done;
+  uint64_t *raw_full, *raw_empty, *a_full, *a_empty, *acc_full, *acc_empty, *q_full, *q_empty,
+      *done;
 };
 
 // Position in a ring of n stages: the stage index and the parity of the
 // stage's mbarrier phase for the current pass.  Advanced once per item, so no
-// role ever divides by a runtime ring size (an integer division is a long
-// dependent instruction sequence on the GPU, and it sat in every role's loop).
+// role ever divides by a runtime ring size.
 struct Ring {
   uint32_t stage, phase, n;
   __device__ explicit Ring(uint32_t n_) : stage(0), phase(0), n(n_) {}
@@ -109,6 +129,38 @@ struct UnitWalk {
       do { ++b; nv = nvalid_of(b); tiles = (nv + kTile - 1) / kTile; } while (tiles == 0);
     }
   }
+};
+
+struct Unit {
+  int b, t, nv;
+};
+
+// The walk in pairs of units of the same row: u[0] for epilogue group 0 and,
+// when the row has a next unit in this CTA's range, u[1] for group 1.  Every
+// role derives the same pairs from the same range.
+struct PairWalk {
+  UnitWalk w;
+  Unit u[2];
+  bool has0, has1;
+  __device__ void fill() {
+    has0 = w.valid();
+    has1 = false;
+    if (!has0) return;
+    u[0] = Unit{w.b, w.t, w.nv};
+    w.next();
+    if (w.valid() && w.b == u[0].b) {
+      u[1] = Unit{w.b, w.t, w.nv};
+      has1 = true;
+      w.next();
+    }
+  }
+  __device__ void start(const int32_t* n_valid, int N, int B, int b0, int t0, int64_t count) {
+    w.n_valid = n_valid; w.N = N; w.B = B;
+    w.start(b0, t0, count);
+    fill();
+  }
+  __device__ bool valid() const { return has0; }
+  __device__ void next() { fill(); }
 };
 
 // 32 lanes x 32 heads x P pieces of one accumulator stage, read in one load+wait.
@@ -168,36 +220,40 @@ __device__ __forceinline__ float head_sum32(const HeadCols<P>& c, const float* _
 template <int P, bool DUMP>
 __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int NR) {
   extern __shared__ uint8_t smem_raw[];
-  const Layout lay = make_layout(args.L, P, NR);
+  constexpr uint32_t ACCW = acc_cols<P>();
+  constexpr uint32_t ABASE = a_col_base<P>();
+  constexpr uint32_t NA = a_stages<P>();
+  const Layout lay = make_layout(args.L, P, NR, NA);
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int L = args.L;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NQ = P * kHeads;
-  constexpr uint32_t kQLayerBytes = (uint32_t)P * kHeads * kHeadDim;
+  constexpr uint32_t kQLayerBytes = (uint32_t)P * kPieceBytes;
 
   uint8_t* sQ = smem + lay.q_off;
   uint8_t* sRaw = smem + lay.raw_off;
   float* sWp = reinterpret_cast<float*>(smem + lay.wp_off);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + lay.bar_off);
   Bars B_;
-  B_.raw_full = bar;                      B_.raw_empty = B_.raw_full + NR;
-  B_.a_full = B_.raw_empty + NR;
-  B_.acc_full = B_.a_full + NR;           B_.acc_empty = B_.acc_full + lay.NACC;
-  B_.q_full = B_.acc_empty + lay.NACC;
-  B_.q_empty = B_.q_full + 1;             B_.done = B_.q_empty + 1;
+  B_.raw_full = bar;                B_.raw_empty = B_.raw_full + NR;
+  B_.a_full = B_.raw_empty + NR;    B_.a_empty = B_.a_full + NA;
+  B_.acc_full = B_.a_empty + NA;    B_.acc_empty = B_.acc_full + 2;
+  B_.q_full = B_.acc_empty + 2;
+  B_.q_empty = B_.q_full + 1;       B_.done = B_.q_empty + 1;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + lay.misc_off);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + lay.misc_off + 4);
   int* sRange = reinterpret_cast<int*>(smem + lay.misc_off + 8);  // b0, t0, count lo, count hi
-  volatile int* sXStatus = reinterpret_cast<volatile int*>(smem + lay.misc_off + 24);
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
     for (int i = 0; i < NR; ++i) {
-      mbar_init(&B_.raw_full[i], 1);   // bulk copy landed
-      mbar_init(&B_.a_full[i], 4);     // re-laid in place (one arrival per transform warp)
-      mbar_init(&B_.raw_empty[i], 1);  // the MMA that read the stage retired
+      mbar_init(&B_.raw_full[i], 1);           // bulk copy landed
+      mbar_init(&B_.raw_empty[i], kQuarters);  // read by all transform warps
     }
-    for (int i = 0; i < lay.NACC; ++i) { mbar_init(&B_.acc_full[i], 1); mbar_init(&B_.acc_empty[i], 4); }
+    for (uint32_t i = 0; i < NA; ++i) {
+      mbar_init(&B_.a_full[i], kQuarters);     // key tile stored in TMEM (one arrival per warp)
+      mbar_init(&B_.a_empty[i], 1);            // the MMA that read it retired
+    }
+    for (int g = 0; g < 2; ++g) { mbar_init(&B_.acc_full[g], 1); mbar_init(&B_.acc_empty[g], kQuarters); }
     mbar_init(B_.q_full, 1);
     mbar_init(B_.q_empty, 1);
     mbar_init(B_.done, 1);
@@ -205,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kWarpMma && lane == 0) {
-    // this CTA's share of the valid units: rows contribute ceil(n_b / 128) tiles
+    // this CTA's share of the valid units: rows contribute ceil(n_b / 96) tiles
     int64_t total = 0;
     for (int b = 0; b < args.B; ++b) {
       int v = args.n_valid ? __ldg(args.n_valid + b) : args.N;
@@ -236,45 +292,32 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
   const uint32_t tmem_base = *sTmem;
   const int b_start = sRange[0], t_start = sRange[1];
   const int64_t count = (int64_t)(uint32_t)sRange[2] | ((int64_t)sRange[3] << 32);
-
-  UnitWalk walk;
-  walk.n_valid = args.n_valid; walk.N = args.N; walk.B = args.B;
+  PairWalk pw;
 
   if (warp == kWarpLoader) {
     // ------------------------------------------------------- key tile loader
     if (lane == 0) {
-      // a second walker runs `prefetch_units` units ahead and pulls their
-      // records into L2, so far more bytes are in flight from HBM than the
-      // shared-memory ring holds; the ring's bulk copies then hit L2
-      UnitWalk pf = walk;
-      pf.start(b_start, t_start, count);
-      auto prefetch_unit = [&]() {
-        const int nrem = min(kTile, pf.nv - pf.t * kTile);
-        const uint32_t bytes = (uint32_t)((nrem + 3) & ~3) * kRecord;
-        for (int l = 0; l < L; ++l)
-          bulk_prefetch_l2(args.comp_k[l] + (int64_t)pf.b * args.row_stride +
-                               (int64_t)pf.t * kRawBytes, bytes);
-        pf.next();
-      };
-      for (int u = 0; u < args.prefetch_units && pf.valid(); ++u) prefetch_unit();
       uint32_t item = 0;
       Ring raw(NR);
-      for (walk.start(b_start, t_start, count); walk.valid() && !*sAbort; walk.next()) {
-        if (args.prefetch_units > 0 && pf.valid()) prefetch_unit();
-        const int nrem = min(kTile, walk.nv - walk.t * kTile);
-        const uint32_t bytes = (uint32_t)((nrem + 3) & ~3) * kRecord;
-        bool ok = true;
-        for (int l = 0; l < L; ++l) {
-          ok = mbar_wait_bounded(&B_.raw_empty[raw.stage], raw.phase ^ 1, sAbort, args.err);
-          if (!ok) break;
-          mbar_arrive_expect_tx(&B_.raw_full[raw.stage], bytes);
-          const uint8_t* src = args.comp_k[l] + (int64_t)walk.b * args.row_stride +
-                               (int64_t)walk.t * kRawBytes;
-          bulk_g2s(sRaw + (size_t)raw.stage * kStageBytes, src, bytes, &B_.raw_full[raw.stage]);
-          ++item;
-          raw.advance();
+      bool ok = true;
+      for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); ok && pw.valid() && !*sAbort;
+           pw.next()) {
+        for (int l = 0; l < L && ok; ++l) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (j == 1 && !pw.has1) break;
+            const Unit U = j == 0 ? pw.u[0] : pw.u[1];
+            const int nrem = min(kTile, U.nv - U.t * kTile);
+            const uint32_t bytes = (uint32_t)((nrem + 3) & ~3) * kRecord;
+            ok = mbar_wait_bounded(&B_.raw_empty[raw.stage], raw.phase ^ 1, sAbort, args.err);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&B_.raw_full[raw.stage], bytes);
+            const uint8_t* src = args.comp_k[l] + (int64_t)U.b * args.row_stride + (int64_t)U.t * kRawBytes;
+            bulk_g2s(sRaw + (size_t)raw.stage * kRawBytes, src, bytes, &B_.raw_full[raw.stage]);
+            ++item;
+            raw.advance();
+          }
         }
-        if (!ok) break;
       }
       // every copy issued must land before the CTA can exit (runs once: the
       // divisions here are off the hot loop)
@@ -289,14 +332,15 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
     if (lane == 0) {
       int cur = -1;
       uint32_t loads = 0;
-      for (walk.start(b_start, t_start, count); walk.valid() && !*sAbort; walk.next()) {
-        if (walk.b == cur) continue;
+      for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); pw.valid() && !*sAbort; pw.next()) {
+        const int b = pw.u[0].b;
+        if (b == cur) continue;
         if (loads > 0 && !mbar_wait_bounded(B_.q_empty, (loads - 1) & 1, sAbort, args.err)) break;
         mbar_arrive_expect_tx(B_.q_full, (uint32_t)L * kQLayerBytes);
         for (int l = 0; l < L; ++l)
-          bulk_g2s(sQ + (size_t)l * kQLayerBytes,
-                   args.qpack + ((size_t)walk.b * L + l) * kQLayerBytes, kQLayerBytes, B_.q_full);
-        cur = walk.b;
+          bulk_g2s(sQ + (size_t)l * kQLayerBytes, args.qpack + ((size_t)b * L + l) * kQLayerBytes,
+                   kQLayerBytes, B_.q_full);
+        cur = b;
         ++loads;
       }
       if (loads > 0) mbar_drain(B_.q_full, (loads - 1) & 1, args.err);
@@ -304,110 +348,110 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(kTile, NQ);
-      uint32_t item = 0, rows = 0;
-      const uint32_t nacc_g = (uint32_t)lay.NACC / 2;
-      Ring ast(NR), acc0(nacc_g), acc1(nacc_g);  // key stages; accumulator stages of group 0 / 1
-      uint32_t unit = 0;                         // CTA-local unit index: unit & 1 = group
+      constexpr uint32_t idesc = idesc_e4m3_f32(kMmaM, (int)ACCW);
+      // B descriptors: the start-address field counts 16-byte units, so the
+      // layer and K-step offsets are plain adds (the field cannot carry: the
+      // query image lies in the first 256 KB of shared memory)
+      const uint64_t bdesc0 = sdesc_kmajor_sw128(smem_u32(sQ));
+      constexpr uint64_t kLayerStep = kQLayerBytes >> 4, kKStep = 32 >> 4;
+      uint32_t item = 0, rows = 0, ph0 = 0, ph1 = 0;
+      Ring ast(NA);
       int cur = -1;
       bool ok = true;
-      walk.start(b_start, t_start, count);
-      while (ok && walk.valid() && !*sAbort) {
-        const int b = walk.b;
+      for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); ok && pw.valid() && !*sAbort;) {
+        const int b = pw.u[0].b;
         if (b != cur) {
           if (!mbar_wait_bounded(B_.q_full, rows & 1, sAbort, args.err)) break;
           ++rows;
           cur = b;
         }
-        const bool g1 = (unit & 1u) != 0;
-        Ring acc = g1 ? acc1 : acc0;  // register copy, written back after the unit
-        for (int l = 0; l < L; ++l) {
-          const int as = ast.stage;
-          const uint32_t ac = (g1 ? nacc_g : 0u) + acc.stage;
-          ok = mbar_wait_bounded(&B_.a_full[as], ast.phase, sAbort, args.err) &&
-               mbar_wait_bounded(&B_.acc_empty[ac], acc.phase ^ 1, sAbort, args.err);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t d = tmem_base + ac * (uint32_t)NQ;
-          const uint32_t a0 = smem_u32(sRaw + (size_t)as * kStageBytes);
-          const uint32_t b0 = smem_u32(sQ + (size_t)l * kQLayerBytes);
+        uint64_t bd = bdesc0;
+        for (int l = 0; l < L && ok; ++l, bd += kLayerStep) {
 #pragma unroll
-          for (int k = 0; k < kHeadDim / 32; ++k)
-            umma_f8f6f4(d, sdesc_kmajor_sw128(a0 + 32u * k), sdesc_kmajor_sw128(b0 + 32u * k), idesc,
-                        k > 0 ? 1u : 0u);
-          umma_commit(&B_.raw_empty[as]);  // the key stage may be refilled
-          umma_commit(&B_.acc_full[ac]);
-          ++item;
-          ast.advance();
-          acc.advance();
+          for (int j = 0; j < 2; ++j) {
+            if (j == 1 && !pw.has1) break;
+            const uint32_t ph = j == 0 ? ph0 : ph1;
+            ok = mbar_wait_bounded(&B_.a_full[ast.stage], ast.phase, sAbort, args.err) &&
+                 mbar_wait_bounded(&B_.acc_empty[j], ph ^ 1, sAbort, args.err);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t d = tmem_base + (uint32_t)j * ACCW;
+            const uint32_t a = tmem_base + ABASE + ast.stage * kACols;
+            umma_f8f6f4_ts(d, a, bd, idesc, 0u);
+            umma_f8f6f4_ts(d, a + 8u, bd + kKStep, idesc, 1u);
+            umma_f8f6f4_ts(d, a + 16u, bd + 2 * kKStep, idesc, 1u);
+            umma_f8f6f4_ts(d, a + 24u, bd + 3 * kKStep, idesc, 1u);
+            umma_commit(&B_.a_empty[ast.stage]);  // the TMEM key tile may be overwritten
+            umma_commit(&B_.acc_full[j]);
+            ++item;
+            ast.advance();
+            if (j == 0) ph0 ^= 1u; else ph1 ^= 1u;
+          }
         }
-        if (g1) acc1 = acc; else acc0 = acc;
-        ++unit;
         if (!ok) break;
-        walk.next();
-        if (!walk.valid() || walk.b != b) umma_commit(B_.q_empty);
+        pw.next();
+        if (!pw.valid() || pw.u[0].b != b) umma_commit(B_.q_empty);
       }
       if (item > 0) {  // every issued MMA and commit retired before TMEM and smem go away
         umma_commit(B_.done);
         mbar_drain(B_.done, 0, args.err);
       }
     }
-  } else if (warp >= kWarpXform0 && warp < kWarpXform0 + 4) {
-    // --------------------- transform: raw records -> MMA operand, in place
-    // One leader thread waits on the copy barrier and the four warps follow it
-    // through a named barrier, so the group always stops together.
-    const int tw = warp - kWarpXform0;
-    const bool leader = tw == 0 && lane == 0;
-    Ring raw(NR);
-    bool alive = true, stop = false;
-    for (walk.start(b_start, t_start, count); walk.valid() && !stop; walk.next()) {
-      for (int l = 0; l < L; ++l, raw.advance()) {
-        if (leader) {
-          alive = alive && mbar_wait_bounded(&B_.raw_full[raw.stage], raw.phase, sAbort, args.err);
-          *sXStatus = alive ? 1 : 0;
-        }
-        __syncwarp();
-        named_bar_sync(kBarXform, 128);
-        if (*sXStatus == 0) { stop = true; break; }
-        uint8_t* st = sRaw + (size_t)raw.stage * kStageBytes;
-        uint32_t v[32];
+  } else if (warp >= kWarpXform0 && warp < kWarpXform0 + 4 && (warp & 3) != 1) {
+    // ------------------------- transform: raw records -> TMEM key tile (A)
+    // Thread `lane` of this warp owns one chunk row of the tile: it reads the
+    // row's 128 key bytes (the 33-word row stride puts the 32 lanes of a load
+    // in 32 different banks) and stores them to its TMEM lane.  The three
+    // warps run independently; each arrives once per item on both barriers.
+    // Items arrive in the loader's order, so only their number matters here.
+    const uint32_t quarter = (uint32_t)warp & 3u;
+    const uint32_t row = (uint32_t)quarter_block((int)quarter) * 32u + (uint32_t)lane;
+    const uint32_t lane_base = tmem_base + ((quarter * 32u) << 16);
+    Ring raw(NR), ast(NA);
+    const int64_t items = count * L;
+    for (int64_t i = 0; i < items; ++i, raw.advance(), ast.advance()) {
+      int good = 1;
+      if (lane == 0)
+        good = mbar_wait_bounded(&B_.raw_full[raw.stage], raw.phase, sAbort, args.err) &&
+               mbar_wait_bounded(&B_.a_empty[ast.stage], ast.phase ^ 1, sAbort, args.err);
+      good = __shfl_sync(0xffffffffu, good, 0);
+      if (!good) break;
+      const uint32_t* src =
+          reinterpret_cast<const uint32_t*>(sRaw + (size_t)raw.stage * kRawBytes + row * kRecord);
+      uint32_t v[32];
 #pragma unroll
-        for (int rr = 0; rr < 32; ++rr)
-          v[rr] = *reinterpret_cast<const uint32_t*>(st + (tw * 32 + rr) * kRecord + lane * 4);
-        named_bar_sync(kBarXform, 128);  // every row read before any row is overwritten
-#pragma unroll
-        for (int rr = 0; rr < 32; ++rr)
-          *reinterpret_cast<uint32_t*>(st + sw128_offset(tw * 32 + rr, lane * 4)) = v[rr];
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B_.a_full[raw.stage]);
+      for (int w = 0; w < 32; ++w) v[w] = src[w];
+      tc_fence_after();  // the MMA that last read this TMEM stage has retired (a_empty)
+      tmem_st32_wait(lane_base + ABASE + ast.stage * kACols, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&B_.raw_empty[raw.stage]);
+        mbar_arrive(&B_.a_full[ast.stage]);
       }
     }
-    if (leader && !alive) *sAbort = 1;
-  } else if (warp >= kWarpEpi0) {
+  } else if (warp >= kWarpEpi0 && (warp & 3) != 1) {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - kWarpEpi0;  // 0..7
-    const uint32_t group = (uint32_t)ew >> 2;
+    const int group = (warp - kWarpEpi0) >> 2;
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
+    const int ew = group * kQuarters + quarter_block(quarter);  // 0..5
+    const int r = quarter_block(quarter) * 32 + lane;           // row of the tile
     float* sWpw = sWp + ew * L * kHeads;
-    const uint32_t lane_base = tmem_base + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t nacc_g = (uint32_t)lay.NACC / 2;
-    Ring acc(nacc_g);  // this group's own accumulator stages
+    const uint32_t col_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)group * ACCW;
+    uint32_t ph = 0;
     int cur = -1;
-    uint32_t unit = 0;
-    for (walk.start(b_start, t_start, count); walk.valid(); walk.next(), ++unit) {
-      if ((unit & 1u) != group) continue;  // the other group's unit
-      const int b = walk.b;
-      if (b != cur) {  // this warp's private copy of the row's head weights
+    for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); pw.valid(); pw.next()) {
+      if (group == 1 && !pw.has1) continue;
+      const Unit U = group == 0 ? pw.u[0] : pw.u[1];
+      if (U.b != cur) {  // this warp's private copy of the row's head weights
         __syncwarp();
         for (int i = lane; i < L * kHeads; i += 32)
-          sWpw[i] = __ldg(args.wprime + (size_t)b * L * kHeads + i);
+          sWpw[i] = __ldg(args.wprime + (size_t)U.b * L * kHeads + i);
         __syncwarp();
-        cur = b;
+        cur = U.b;
       }
-      const int n = walk.t * kTile + r;
-      const bool valid = n < walk.nv;
+      const int n = U.t * kTile + r;
+      const bool valid = n < U.nv;
       const bool in_row = n < args.N;
       // the chunk's scales, read from L2 while the accumulators are computed
       float sc[kMaxLayers];
@@ -415,59 +459,57 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       for (int l = 0; l < kMaxLayers; ++l) {
         sc[l] = 0.f;
         if (l < L && valid)
-          sc[l] = __ldg(reinterpret_cast<const float*>(args.comp_k[l] + (int64_t)b * args.row_stride +
+          sc[l] = __ldg(reinterpret_cast<const float*>(args.comp_k[l] + (int64_t)U.b * args.row_stride +
                                                        (int64_t)n * kRecord + kHeadDim));
       }
       float ens = 0.f;
       bool ok = true;
-      for (int l = 0; l < L; ++l, acc.advance()) {
+      for (int l = 0; l < L; ++l, ph ^= 1u) {
         const float s = l == 0 ? sc[0] : l == 1 ? sc[1] : l == 2 ? sc[2] : sc[3];
-        const uint32_t slot = group * nacc_g + acc.stage;
-        ok = mbar_wait_bounded(&B_.acc_full[slot], acc.phase, sAbort, args.err);
+        ok = mbar_wait_bounded(&B_.acc_full[group], ph, sAbort, args.err);
         if (!ok) break;
         tc_fence_after();
         const bool nonneg = __all_sync(0xffffffffu, !(s < 0.f));
-        const uint32_t col = lane_base + slot * (uint32_t)NQ;
         const float* w = sWpw + l * kHeads;
         HeadCols<P> c;
-        c.load(col);
+        c.load(col_base);
         if constexpr (DUMP) {
-          if (b == args.dbg_b && walk.t == args.dbg_t && l == args.dbg_layer)
+          if (U.b == args.dbg_b && U.t == args.dbg_t && l == args.dbg_layer)
             for (int p = 0; p < P; ++p)
-              for (int i = 0; i < 32; ++i) args.dbg_out[(size_t)r * NQ + p * kHeads + i] = c.at(p, i);
+              for (int i = 0; i < 32; ++i) args.dbg_out[(size_t)r * 192 + p * kHeads + i] = c.at(p, i);
         }
         float part = head_sum32<P>(c, w, s, nonneg);
-        c.load(col + 32);
+        c.load(col_base + 32);
         // the accumulator stage is free once this warp holds all its columns
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B_.acc_empty[slot]);
+        if (lane == 0) mbar_arrive(&B_.acc_empty[group]);
         if constexpr (DUMP) {
-          if (b == args.dbg_b && walk.t == args.dbg_t && l == args.dbg_layer)
+          if (U.b == args.dbg_b && U.t == args.dbg_t && l == args.dbg_layer)
             for (int p = 0; p < P; ++p)
               for (int i = 0; i < 32; ++i)
-                args.dbg_out[(size_t)r * NQ + p * kHeads + 32 + i] = c.at(p, i);
+                args.dbg_out[(size_t)r * 192 + p * kHeads + 32 + i] = c.at(p, i);
         }
         part += head_sum32<P>(c, w + 32, s, nonneg);
         const float logit = nonneg ? part * s : part;
         float score = 1.0f / (1.0f + __expf(-logit));
         if (!valid) score = 0.f;
-        if (args.scores && in_row) args.scores[((size_t)l * args.B + b) * args.N + n] = score;
+        if (args.scores && in_row) args.scores[((size_t)l * args.B + U.b) * args.N + n] = score;
         ens = (args.mode == FM_ENSEMBLE_MAX) ? (l == 0 ? score : fmaxf(ens, score)) : ens + score;
       }
       if (!ok) break;
       if (args.mode != FM_ENSEMBLE_MAX) ens = ens / (float)L;
       if (!valid) ens = 0.f;
       if (in_row) {
-        if (args.ens) args.ens[(size_t)b * args.N + n] = ens;
-        if (args.keep_thr) args.keep_thr[(size_t)b * args.N + n] = (valid && ens > args.thr) ? 1 : 0;
+        if (args.ens) args.ens[(size_t)U.b * args.N + n] = ens;
+        if (args.keep_thr) args.keep_thr[(size_t)U.b * args.N + n] = (valid && ens > args.thr) ? 1 : 0;
       }
     }
-    // zero the tail of every row that no tile covers: [128 * ceil(n_b / 128), N)
-    const int et = threadIdx.x - kWarpEpi0 * 32;
-    const int64_t gt = (int64_t)blockIdx.x * 256 + et, gs = (int64_t)gridDim.x * 256;
+    // zero the tail of every row that no tile covers: [96 * ceil(n_b / 96), N)
+    const int et = ew * 32 + lane;  // 0..191
+    const int64_t gt = (int64_t)blockIdx.x * 192 + et, gs = (int64_t)gridDim.x * 192;
     for (int b = 0; b < args.B; ++b) {
-      const int v = walk.nvalid_of(b);
+      const int v = pw.w.nvalid_of(b);
       const int from = min(args.N, ((v + kTile - 1) / kTile) * kTile);
       for (int64_t n = from + gt; n < args.N; n += gs) {
         if (args.scores)
@@ -497,10 +539,11 @@ fm_status launch_score_p(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t st) {
   // deepest key ring that fits: every stage is keys in flight
   int NR = 16;
   if (const char* e = getenv("FM_RAW_STAGES")) NR = atoi(e) < 2 ? 2 : atoi(e);
-  Layout lay = make_layout(a.L, P, NR);
+  constexpr int NA = (int)a_stages<P>();
+  Layout lay = make_layout(a.L, P, NR, NA);
   while (lay.total > (uint32_t)max_smem && NR > 2) {
     --NR;
-    lay = make_layout(a.L, P, NR);
+    lay = make_layout(a.L, P, NR, NA);
   }
   if (lay.total > (uint32_t)max_smem) return FM_ERR_UNSUPPORTED;
   if (configured_dev != ctx->device) {

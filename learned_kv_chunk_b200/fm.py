@@ -290,8 +290,7 @@ class Retriever:
     def fm_debug_tile_dots(self, comp_k, q, fused_w, layer: int, b: int, t: int, N=None):
         B, N, stride = _keys_shape(comp_k, N)
         arr = _comp_k_array(comp_k)
-        P = self.cfg.q_pieces
-        out = torch.full((128, P * 64), float("nan"), device=q.device, dtype=torch.float32)
+        out = torch.zeros((128, 192), device=q.device, dtype=torch.float32)
         e = torch.zeros(64, device=q.device, dtype=torch.int32)
         _check(_lib.fm_debug_tile_dots(self._h, arr, stride, B, N, _ptr(q), _ptr(fused_w), layer, b, t,
                                        _ptr(out), _ptr(e), _stream()), "fm_debug_tile_dots")
