@@ -1,0 +1,100 @@
+"""The C ABI without a GPU: libfm.so loads, exports every function that
+include/fm.h declares, and its host-side calls (defaults, status text,
+workspace sizing, argument checks that reject before any device work)
+behave as the header states."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fm.h")
+LIB = os.path.join(ROOT, "learned_kv_chunk_b200", "lib", "libfm.so")
+
+if not os.path.exists(LIB):
+    pytest.skip("libfm.so is not built (python -m learned_kv_chunk_b200.build)", allow_module_level=True)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w \*]*?\b(fm_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return ctypes.CDLL(LIB)
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for required in ["fm_create", "fm_destroy", "fm_query_prep", "fm_score", "fm_ensemble",
+                     "fm_score_fused", "fm_select_topk", "fm_select_threshold",
+                     "fm_topk_workspace_bytes", "fm_sync_status", "fm_strerror"]:
+        assert required in names, required
+
+
+def test_every_declared_function_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s+(fm_\w+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        getattr(lib, n)  # resolvable through the dynamic loader too
+
+
+def test_status_text(lib):
+    lib.fm_strerror.restype = ctypes.c_char_p
+    texts = [lib.fm_strerror(s).decode() for s in range(7)]
+    assert texts[0] == "ok"
+    assert len(set(texts)) == 7
+    assert lib.fm_strerror(99).decode() == "unknown status"
+
+
+def test_config_defaults(lib):
+    from learned_kv_chunk_b200.fm import fm_config
+    c = fm_config()
+    lib.fm_config_default(ctypes.byref(c))
+    assert (c.hidden, c.q_lora_rank, c.n_heads, c.head_dim, c.n_layers, c.rope_dim) == (4096, 1024, 64, 128, 3, 64)
+    assert (c.rope_base, c.rope_factor, c.rope_orig_max_pos) == (160000.0, 16.0, 65536.0)
+    assert (c.rope_beta_fast, c.rope_beta_slow) == (32.0, 1.0)
+    assert abs(c.rms_eps - 1e-6) < 1e-12
+    assert c.q_pieces in (2, 3) and c.max_batch >= 1
+
+
+def test_topk_workspace_sizing(lib):
+    f = lib.fm_topk_workspace_bytes
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_int, ctypes.c_int]
+    assert f(0, 100) == 0 and f(1, 0) == 0
+    a, b, c = f(1, 4096), f(2, 4096), f(1, 1 << 20)
+    assert 0 < a < b and a < c
+    assert a % 256 == 0 and c % 256 == 0
+    # the no-allocation variant's limit covers the 64-row, 262144-chunk workload
+    assert f(64, 262144) <= (4 << 20) < f(300, 262144)
+
+
+def test_host_side_argument_rejection(lib):
+    P, I = ctypes.c_void_p, ctypes.c_int
+    lib.fm_select_topk.argtypes = [P, P, I, I, I, P, P, ctypes.c_size_t, P]
+    lib.fm_select_topk_static.argtypes = [P, P, I, I, I, P, P]
+    lib.fm_select_threshold.argtypes = [P, P, I, I, ctypes.c_float, P, P]
+    lib.fm_ensemble.argtypes = [P, I, I, I, I, P, P]
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails its checks first
+    INVALID, ALIGN, UNSUP = 1, 2, 3
+    assert lib.fm_select_topk(None, None, 1, 10, 5, fake, fake, 1 << 20, None) == INVALID
+    assert lib.fm_select_topk(fake, None, 1, 10, 0, fake, fake, 1 << 20, None) == INVALID
+    assert lib.fm_select_topk(fake, None, 1, 10, 5, fake, fake, 0, None) == INVALID
+    assert lib.fm_select_topk(ctypes.c_void_p(0x1001), None, 1, 10, 5, fake, fake, 1 << 20, None) == ALIGN
+    assert lib.fm_select_topk_static(fake, None, 300, 262144, 5, fake, None) == UNSUP
+    assert lib.fm_select_topk_static(fake, None, 0, 10, 5, fake, None) == INVALID
+    assert lib.fm_select_threshold(None, None, 1, 10, 0.5, fake, None) == INVALID
+    assert lib.fm_ensemble(fake, 5, 1, 10, 0, fake, None) == INVALID  # more layers than supported
+    assert lib.fm_ensemble(fake, 3, 1, 10, 7, fake, None) == INVALID  # unknown mode
+    lib.fm_create.argtypes = [P, P, I, ctypes.POINTER(P)]
+    out = P(0x1234)
+    assert lib.fm_create(None, None, 0, ctypes.byref(out)) == INVALID
+    assert out.value is None
