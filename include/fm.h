@@ -77,7 +77,9 @@ typedef struct fm_config {
   float rms_eps;          /* 1e-6 */
   int max_batch;          /* largest B any call on this context will pass */
   int q_pieces;           /* e4m3 pieces per query element in the tensor-core
-                             product: 3 (default, ~2^-12 relative) or 2 (~2^-8) */
+                             product: 2 (default; query split error ~2^-8
+                             relative, scores within ~5e-4 on the shipped
+                             workloads) or 3 (~2^-12, ~1e-5; about 15% slower) */
 } fm_config;
 
 /* One layer's weights, fp32, row-major [out, in], no biases (README
@@ -95,7 +97,7 @@ typedef struct fm_ctx fm_ctx;
 
 /* Fills *cfg with the shipped constants (hidden 4096, rank 1024, 64 heads,
  * head_dim 128, 3 layers, YaRN 160000/16/65536/32/1, eps 1e-6, max_batch 64,
- * q_pieces 3). */
+ * q_pieces 2). */
 void fm_config_default(fm_config* cfg);
 
 /* Creates a context on `device`: uploads the weights (cfg->n_layers entries of
@@ -216,11 +218,10 @@ int fm_last_cuda_error(void);
 /* Number of kernel launches issued by this process since load (all calls). */
 uint64_t fm_launch_count(void);
 
-/* Diagnostic: the raw tensor-core dot products of one 96-chunk tile of layer
- * `layer`, row b, tile t (chunks t*96 .. t*96+95), before the per-chunk
- * scale, the per-head power-of-two scale and the epilogue, for r < 96 and
- * p < q_pieces:
- *   out[r, p*64 + h] = sum_d e4m3(comp_k[layer][b, t*96 + r, d]) * piece_p(q[b,layer,h])[d]
+/* Diagnostic: the raw tensor-core dot products of one 128-chunk tile of layer
+ * `layer`, row b, tile t (chunks t*128 .. t*128+127), before the per-chunk
+ * scale, the per-head power-of-two scale and the epilogue, for p < q_pieces:
+ *   out[r, p*64 + h] = sum_d e4m3(comp_k[layer][b, t*128 + r, d]) * piece_p(q[b,layer,h])[d]
  * where the query pieces satisfy
  *   q[b,layer,h,d] ~= 2^-pow2_exp[h] * sum_p 16^-p * piece_p[d].
  * out [128, 192] fp32 device (the entries above written, the rest untouched),

@@ -105,7 +105,7 @@ void fm_config_default(fm_config* c) {
   c->rope_beta_slow = 1.0;
   c->rms_eps = 1e-6f;
   c->max_batch = 64;
-  c->q_pieces = 3;
+  c->q_pieces = 2;
 }
 
 fm_status fm_create(const fm_config* cfg, const fm_layer_weights* w, int device, fm_ctx** out) {

@@ -17,9 +17,7 @@ constexpr int kHeads = 64;        // N_HEADS (the shipped value; checked at crea
 constexpr int kHeadDim = 128;     // HEAD_DIM (README "Architecture")
 constexpr int kRopeDim = 64;      // ROPE_DIM (README "Architecture")
 constexpr int kRecord = 132;      // bytes per compressed chunk (README "compressed_k format")
-constexpr int kTile = 96;         // chunks per scored tile: TMEM lanes 0-31 and 64-127 of an
-                                  // M = 128 MMA (lanes 32-63, the quarter that only warps on the
-                                  // MMA issuer's scheduler can reach, stay unused)
+constexpr int kTile = 128;        // chunks per tensor-core tile (MMA M, one TMEM lane each)
 constexpr int kMaxLayers = 4;
 constexpr int kMaxBatch = 4096;
 
@@ -75,7 +73,7 @@ struct ScoreArgs {
   int mode;                // FM_ENSEMBLE_*
   int* err;
   // diagnostic dump of one tile's raw accumulators
-  float* dbg_out;          // [128, 128] or null
+  float* dbg_out;          // [128, 192] or null
   int dbg_layer, dbg_b, dbg_t;
 };
 fm_status launch_score(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t stream);
@@ -270,6 +268,24 @@ __device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const uint32_t* v
       : "memory");
 }
 
+// As tmem_st32_wait, plus one more 32-bit column per lane at taddr1 (the same
+// wait covers both stores).
+__device__ __forceinline__ void tmem_st32_st1_wait(uint32_t taddr, const uint32_t* v, uint32_t taddr1,
+                                                   uint32_t v1) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x1.b32 [%33], {%34};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31]), "r"(taddr1), "r"(v1)
+      : "memory");
+}
+
 // Arrives on `bar` once every tcgen05.mma this thread issued before has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
@@ -319,6 +335,41 @@ __device__ __forceinline__ void tmem_ld32x2_wait(uint32_t t0, uint32_t t1, uint3
 }
 
 // Three 32-column loads and one wait.
+// Two 32-column loads plus one single column (ts, result in *s), one wait.
+__device__ __forceinline__ void tmem_ld32x2_x1_wait(uint32_t t0, uint32_t t1, uint32_t ts, uint32_t* a,
+                                                    uint32_t* b, uint32_t* s) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%64}, [%67];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%65];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%66];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : FM_TMEM_REGS32(a), FM_TMEM_REGS32(b), "=r"(*s)
+      : "r"(t0), "r"(t1), "r"(ts)
+      : "memory");
+}
+// Three 32-column loads plus one single column (ts, result in *s), one wait.
+__device__ __forceinline__ void tmem_ld32x3_x1_wait(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t ts,
+                                                    uint32_t* a, uint32_t* b, uint32_t* c, uint32_t* s) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%96}, [%100];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%97];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%98];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
+      "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95}, [%99];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : FM_TMEM_REGS32(a), FM_TMEM_REGS32(b), FM_TMEM_REGS32(c), "=r"(*s)
+      : "r"(t0), "r"(t1), "r"(t2), "r"(ts)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_ld32x3_wait(uint32_t t0, uint32_t t1, uint32_t t2,
                                                  uint32_t* a, uint32_t* b, uint32_t* c) {
   asm volatile(

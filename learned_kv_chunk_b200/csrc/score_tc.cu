@@ -7,43 +7,42 @@
 // threshold keep rule (toy decode loop, "sigmoid > thresh").
 //
 // Design (sm_100a):
-//  * one persistent CTA per SM walks a contiguous range of (row, 96-chunk
+//  * one persistent CTA per SM walks a contiguous range of (row, 128-chunk
 //    tile) units; each unit is scored for all L layers (one "item" per layer)
 //    so the ensemble stays in registers and one fp32 per chunk is written;
 //  * the keys go to the tensor cores as stored: kind::f8f6f4 MMA with A = the
 //    128 e4m3 bytes of each record (K = 128 dims) and B = the query split into
 //    P e4m3 pieces (N = P * 64: piece p of head h in column p*64 + h), fp32
-//    accumulators in TMEM -- four MMAs (the K steps) per item.  A tile holds
-//    96 chunks in TMEM lanes 0-31 and 64-127 of an M = 128 MMA; lanes 32-63
-//    stay unused (see the warp roles).  The per-chunk fp32 scale, the
+//    accumulators in TMEM -- four MMAs (the K steps) per item, M = 128 chunks
+//    in the 128 TMEM lanes.  The per-chunk fp32 scale, the
 //    per-head power-of-two scale of the pieces, relu, the head-weighted sum
 //    and the sigmoid run in the epilogue;
 //  * the 132-byte records are not 16-byte aligned, so a tile is fetched with
-//    one 1-D bulk copy (TMA engine) of 96 * 132 bytes into a shared-memory
-//    stage; three transform warps (one TMEM lane quarter each, one chunk row
+//    one 1-D bulk copy (TMA engine) of 128 * 132 bytes into a shared-memory
+//    stage; four transform warps (one TMEM lane quarter each, one chunk row
 //    per thread) read each row with conflict-free 4-byte loads (row stride 33
-//    words) and store it into TMEM, where the MMA takes A from.  A stage goes
-//    back to the key loader as soon as it has been read, so the ring holds
-//    little besides keys in flight from HBM;
-//  * one thread issues every MMA, and its issue rate bounds the pass: each
-//    tcgen05.mma, commit or mbarrier probe it executes costs tens of cycles.
-//    So an item is four MMAs with descriptors advanced by constant adds, and
-//    the thread's scheduler is left to it alone: warp w runs on scheduler
-//    w % 4 and may only touch TMEM lanes 32*(w % 4) .. +31, and a warp
-//    issuing back-to-back FP32 work on the issuer's scheduler (1) starves
-//    tcgen05.mma issue (measured: 8 MMAs went from ~400 to ~1700 cycles; on
-//    the other schedulers such warps cost nothing).  Hence no chunk lives in
-//    lane quarter 1;
+//    words) and store it into TMEM, where the MMA takes A from; each thread
+//    also moves its record's fp32 scale into a TMEM column that the epilogue
+//    reads with the accumulators, so no scale is read from global memory.  A
+//    stage goes back to the key loader as soon as it has been read, so the
+//    ring holds little besides keys in flight from HBM;
+//  * two single threads pace the pass: the key loader (its copies in flight
+//    set the HBM rate) and the MMA issuer (each tcgen05.mma, commit or
+//    mbarrier probe costs it tens of cycles, so an item is four MMAs with
+//    descriptors advanced by constant adds, and per-item work is kept off
+//    every role: scales travel through TMEM instead of as scattered global
+//    loads, which doubled the L2 request count).  Warp w runs on scheduler
+//    w % 4 and may only touch TMEM lanes 32*(w % 4) .. +31, so every
+//    scheduler hosts one transform warp and two epilogue warps;
 //  * warp roles (16 warps): 0 key loader, 1 MMA issuer, 2 TMEM owner + query
-//    loader, 4, 6, 7 transform, {8, 10, 11} and {12, 14, 15} two epilogue
-//    groups (one lane quarter per warp, all 64 heads of a chunk row), each
-//    with one accumulator stage.  Units are taken in pairs from the same row,
+//    loader, 4-7 transform, 8-11 and 12-15 two epilogue groups (one lane
+//    quarter per warp, all 64 heads of a chunk row), each with one
+//    accumulator stage.  Units are taken in pairs from the same row,
 //    the first for group 0 and the second for group 1, and their items are
 //    issued layer by layer alternately, (u0,l0) (u1,l0) (u0,l1) (u1,l1) ...,
 //    so each group has a whole MMA to drain its stage before it is needed
 //    again.  Every ring index is advanced incrementally (no runtime division
-//    in any loop), and the epilogue reads each chunk's scale from global
-//    memory (an L2 hit: the tile was fetched moments earlier).
+//    in any loop).
 #include <cstdlib>
 
 #include "fm_internal.cuh"
@@ -53,25 +52,33 @@ namespace {
 
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kRawBytes = kTile * kRecord;  // 12672, a multiple of 128
-constexpr int kMmaM = 128;                  // MMA rows (TMEM lanes); chunks use lanes 0-31, 64-127
-constexpr int kQuarters = 3;                // TMEM lane quarters holding chunks: 0, 2, 3
+constexpr int kRawBytes = kTile * kRecord;  // 16896, a multiple of 128
+constexpr int kMmaM = kTile;                // MMA rows = TMEM lanes = chunks of a tile
+constexpr int kQuarters = 4;                // TMEM lane quarters (32 lanes, one warp each)
 constexpr int kWarpLoader = 0, kWarpMma = 1, kWarpQ = 2;
-constexpr int kWarpXform0 = 4, kWarpEpi0 = 8;  // + 0, 2, 3 (scheduler 1 is left to the MMA issuer)
+constexpr int kWarpXform0 = 4, kWarpEpi0 = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACols = 32;  // 128 e4m3 bytes per row = 32 columns per key tile
 constexpr uint32_t kPieceBytes = kHeads * kHeadDim;  // one query piece of one layer
 
-// TMEM columns: accumulator of group g at [g * P*64, (g+1) * P*64), key tiles after them.
+// TMEM columns: accumulator of group g at [g * P*64, (g+1) * P*64), key tiles
+// after them, and the last 32 columns a ring of per-chunk scales (one column
+// per item, slot = item index mod 32).
+constexpr uint32_t kScaleSlots = 32;
+constexpr uint32_t kScaleCol = kTmemCols - kScaleSlots;
 template <int P>
 constexpr uint32_t acc_cols() { return (uint32_t)P * kHeads; }
 template <int P>
 constexpr uint32_t a_col_base() { return 2u * acc_cols<P>(); }
 template <int P>
-constexpr uint32_t a_stages() { return (kTmemCols - a_col_base<P>()) / kACols; }  // 8 (P=2), 4 (P=3)
+constexpr uint32_t a_stages() { return (kScaleCol - a_col_base<P>()) / kACols; }  // 7 (P=2), 3 (P=3)
+// A scale slot is rewritten 32 items after it was written.  The item that
+// rewrites it waits for its key stage, i.e. for the MMA of the item NA before
+// it, and that MMA was issued only after both epilogue groups had loaded
+// (scale included) every item up to two before it; so NA + 2 < 32 keeps every
+// scale alive until it has been read.
+static_assert(a_stages<2>() + 2 < kScaleSlots && a_stages<3>() + 2 < kScaleSlots, "scale ring too short");
 
-// TMEM lane quarter q in {0, 2, 3} -> block of 32 tile rows (0, 1, 2).
-__device__ __forceinline__ int quarter_block(int q) { return q == 0 ? 0 : q - 1; }
 
 struct Layout {
   uint32_t q_off, raw_off, wp_off, bar_off, misc_off, total;
@@ -163,7 +170,8 @@ struct PairWalk {
   __device__ void next() { fill(); }
 };
 
-// 32 lanes x 32 heads x P pieces of one accumulator stage, read in one load+wait.
+// 32 lanes x 32 heads x P pieces of one accumulator stage, read in one load+wait
+// (optionally with one more column, the chunk's scale).
 template <int P>
 struct HeadCols {
   uint32_t u[P][32];
@@ -172,6 +180,12 @@ struct HeadCols {
       tmem_ld32x3_wait(col0, col0 + kHeads, col0 + 2 * kHeads, u[0], u[1], u[2]);
     else
       tmem_ld32x2_wait(col0, col0 + kHeads, u[0], u[1]);
+  }
+  __device__ __forceinline__ void load_with(uint32_t col0, uint32_t scol, uint32_t* sv) {
+    if constexpr (P == 3)
+      tmem_ld32x3_x1_wait(col0, col0 + kHeads, col0 + 2 * kHeads, scol, u[0], u[1], u[2], sv);
+    else
+      tmem_ld32x2_x1_wait(col0, col0 + kHeads, scol, u[0], u[1], sv);
   }
   __device__ __forceinline__ float at(int p, int i) const { return __uint_as_float(u[p][i]); }
 };
@@ -261,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kWarpMma && lane == 0) {
-    // this CTA's share of the valid units: rows contribute ceil(n_b / 96) tiles
+    // this CTA's share of the valid units: rows contribute ceil(n_b / 128) tiles
     int64_t total = 0;
     for (int b = 0; b < args.B; ++b) {
       int v = args.n_valid ? __ldg(args.n_valid + b) : args.N;
@@ -397,15 +411,15 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
         mbar_drain(B_.done, 0, args.err);
       }
     }
-  } else if (warp >= kWarpXform0 && warp < kWarpXform0 + 4 && (warp & 3) != 1) {
+  } else if (warp >= kWarpXform0 && warp < kWarpXform0 + 4) {
     // ------------------------- transform: raw records -> TMEM key tile (A)
     // Thread `lane` of this warp owns one chunk row of the tile: it reads the
     // row's 128 key bytes (the 33-word row stride puts the 32 lanes of a load
-    // in 32 different banks) and stores them to its TMEM lane.  The three
+    // in 32 different banks) and stores them to its TMEM lane.  The four
     // warps run independently; each arrives once per item on both barriers.
     // Items arrive in the loader's order, so only their number matters here.
     const uint32_t quarter = (uint32_t)warp & 3u;
-    const uint32_t row = (uint32_t)quarter_block((int)quarter) * 32u + (uint32_t)lane;
+    const uint32_t row = quarter * 32u + (uint32_t)lane;
     const uint32_t lane_base = tmem_base + ((quarter * 32u) << 16);
     Ring raw(NR), ast(NA);
     const int64_t items = count * L;
@@ -421,8 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       uint32_t v[32];
 #pragma unroll
       for (int w = 0; w < 32; ++w) v[w] = src[w];
+      const uint32_t scale_bits = src[32];  // the record's little-endian fp32 scale
       tc_fence_after();  // the MMA that last read this TMEM stage has retired (a_empty)
-      tmem_st32_wait(lane_base + ABASE + ast.stage * kACols, v);
+      tmem_st32_st1_wait(lane_base + ABASE + ast.stage * kACols, v,
+                         lane_base + kScaleCol + ((uint32_t)i & (kScaleSlots - 1)), scale_bits);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -430,17 +446,20 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
         mbar_arrive(&B_.a_full[ast.stage]);
       }
     }
-  } else if (warp >= kWarpEpi0 && (warp & 3) != 1) {
+  } else if (warp >= kWarpEpi0) {
     // ------------------------------------------------------------ epilogue
     const int group = (warp - kWarpEpi0) >> 2;
     const int quarter = warp & 3;
-    const int ew = group * kQuarters + quarter_block(quarter);  // 0..5
-    const int r = quarter_block(quarter) * 32 + lane;           // row of the tile
+    const int ew = group * kQuarters + quarter;  // 0..7
+    const int r = quarter * 32 + lane;           // row of the tile
     float* sWpw = sWp + ew * L * kHeads;
     const uint32_t col_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)group * ACCW;
-    uint32_t ph = 0;
+    const uint32_t scale_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + kScaleCol;
+    uint32_t ph = 0, gbase = 0;  // gbase: index of the pair's first item in the CTA's item order
     int cur = -1;
     for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); pw.valid(); pw.next()) {
+      const uint32_t per = pw.has1 ? 2u : 1u, gb = gbase;  // items per layer in this pair
+      gbase += per * (uint32_t)L;
       if (group == 1 && !pw.has1) continue;
       const Unit U = group == 0 ? pw.u[0] : pw.u[1];
       if (U.b != cur) {  // this warp's private copy of the row's head weights
@@ -453,26 +472,19 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       const int n = U.t * kTile + r;
       const bool valid = n < U.nv;
       const bool in_row = n < args.N;
-      // the chunk's scales, read from L2 while the accumulators are computed
-      float sc[kMaxLayers];
-#pragma unroll
-      for (int l = 0; l < kMaxLayers; ++l) {
-        sc[l] = 0.f;
-        if (l < L && valid)
-          sc[l] = __ldg(reinterpret_cast<const float*>(args.comp_k[l] + (int64_t)U.b * args.row_stride +
-                                                       (int64_t)n * kRecord + kHeadDim));
-      }
       float ens = 0.f;
       bool ok = true;
       for (int l = 0; l < L; ++l, ph ^= 1u) {
-        const float s = l == 0 ? sc[0] : l == 1 ? sc[1] : l == 2 ? sc[2] : sc[3];
         ok = mbar_wait_bounded(&B_.acc_full[group], ph, sAbort, args.err);
         if (!ok) break;
         tc_fence_after();
-        const bool nonneg = __all_sync(0xffffffffu, !(s < 0.f));
+        const uint32_t item = gb + (uint32_t)l * per + (uint32_t)group;
         const float* w = sWpw + l * kHeads;
         HeadCols<P> c;
-        c.load(col_base);
+        uint32_t s_bits;
+        c.load_with(col_base, scale_base + (item & (kScaleSlots - 1)), &s_bits);
+        const float s = valid ? __uint_as_float(s_bits) : 0.f;  // rows past the tail hold stale bytes
+        const bool nonneg = __all_sync(0xffffffffu, !(s < 0.f));
         if constexpr (DUMP) {
           if (U.b == args.dbg_b && U.t == args.dbg_t && l == args.dbg_layer)
             for (int p = 0; p < P; ++p)
@@ -505,9 +517,9 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
         if (args.keep_thr) args.keep_thr[(size_t)U.b * args.N + n] = (valid && ens > args.thr) ? 1 : 0;
       }
     }
-    // zero the tail of every row that no tile covers: [96 * ceil(n_b / 96), N)
-    const int et = ew * 32 + lane;  // 0..191
-    const int64_t gt = (int64_t)blockIdx.x * 192 + et, gs = (int64_t)gridDim.x * 192;
+    // zero the tail of every row that no tile covers: [128 * ceil(n_b / 128), N)
+    const int et = ew * 32 + lane;  // 0..255
+    const int64_t gt = (int64_t)blockIdx.x * 256 + et, gs = (int64_t)gridDim.x * 256;
     for (int b = 0; b < args.B; ++b) {
       const int v = pw.w.nvalid_of(b);
       const int from = min(args.N, ((v + kTile - 1) / kTile) * kTile);

@@ -199,7 +199,7 @@ class Retriever:
     q_norm [R], wq_b [H*D, R], weights_proj [H, HID] (CPU or CUDA)."""
 
     def __init__(self, weights: List[dict], device: int = 0, max_batch: int = 64,
-                 q_pieces: int = 3, **overrides):
+                 q_pieces: int = 2, **overrides):
         cfg = fm_config_default()
         cfg.n_layers = len(weights)
         cfg.max_batch = max_batch

@@ -66,13 +66,11 @@ def test_tile_dot_products_layout(retr, weights):
         torch.cuda.synchronize()
         out = out.cpu().numpy().astype(np.float64)
         e = e.cpu().numpy()
-        codes = case.comp_k[l][b, t * 96:(t + 1) * 96, :128].numpy()
-        kv = O.e4m3_decode(codes).astype(np.float64)             # [96, 128]
-        exact = kv @ qh[b, l].T                                    # [96, 64]
-        assert np.all(out[96:] == 0.0)  # rows past the 96-chunk tile are untouched
-        assert np.all(out[:, P * 64:] == 0.0)  # columns past the pieces too
-        out = out[:96]
-        rec = np.zeros((96, 64))
+        codes = case.comp_k[l][b, t * 128:(t + 1) * 128, :128].numpy()
+        kv = O.e4m3_decode(codes).astype(np.float64)             # [128, 128]
+        exact = kv @ qh[b, l].T                                    # [128, 64]
+        assert np.all(out[:, P * 64:] == 0.0)  # columns past the pieces are untouched
+        rec = np.zeros((128, 64))
         for p in range(P):
             rec += out[:, p * 64:(p + 1) * 64] * 16.0 ** (-p)
         rec *= 2.0 ** (-e[None, :].astype(np.float64))
