@@ -146,6 +146,15 @@ fm_status fm_create(const fm_config* cfg, const fm_layer_weights* w, int device,
       {(void**)&c->wprime, (size_t)Bm * L * H * sizeof(float)},
       {(void**)&c->qexp, (size_t)Bm * L * H * sizeof(int32_t)},
       {(void**)&c->d_err, sizeof(int)},
+      {(void**)&c->w_down_hi, M * HID * sizeof(float)},
+      {(void**)&c->w_down_lo, M * HID * sizeof(float)},
+      {(void**)&c->w_up_hi, (size_t)L * H * D * R * sizeof(float)},
+      {(void**)&c->w_up_lo, (size_t)L * H * D * R * sizeof(float)},
+      {(void**)&c->x_hi, (size_t)Bm * HID * sizeof(float)},
+      {(void**)&c->x_lo, (size_t)Bm * HID * sizeof(float)},
+      {(void**)&c->r_hi, (size_t)Bm * L * R * sizeof(float)},
+      {(void**)&c->r_lo, (size_t)Bm * L * R * sizeof(float)},
+      {(void**)&c->up_part, (size_t)2 * Bm * L * H * D * sizeof(float)},
   };
   fm_status st = FM_OK;
   for (auto& a : allocs) {
@@ -175,6 +184,8 @@ fm_status fm_create(const fm_config* cfg, const fm_layer_weights* w, int device,
         (e = cudaMemset(c->d_err, 0, sizeof(int))) || (e = cudaDeviceSynchronize()))
       st = cuda_fail(e);
   }
+  if (st == FM_OK) st = prepare_tc_weights(c);
+  if (st == FM_OK && (e = cudaDeviceSynchronize())) st = cuda_fail(e);
   if (st != FM_OK) {
     fm_destroy(c);
     cudaSetDevice(prev);
@@ -191,8 +202,10 @@ fm_status fm_destroy(fm_ctx* c) {
   cudaGetDevice(&prev);
   cudaSetDevice(c->device);
   cudaDeviceSynchronize();
-  void* ptrs[] = {c->w_down, c->q_norm, c->w_up, c->rope_freq, c->a_part,
-                  c->r_norm, c->rope_cs, c->qpack, c->wprime, c->qexp, c->d_err};
+  void* ptrs[] = {c->w_down, c->q_norm,  c->w_up,    c->rope_freq, c->a_part,    c->r_norm,
+                  c->rope_cs, c->qpack,   c->wprime,  c->qexp,      c->d_err,     c->w_down_hi,
+                  c->w_down_lo, c->w_up_hi, c->w_up_lo, c->x_hi,    c->x_lo,      c->r_hi,
+                  c->r_lo,    c->up_part};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   cudaSetDevice(prev);

@@ -45,6 +45,15 @@ struct fm_ctx {
   float* wprime;    // [max_batch, L, 64] fused_w * 2^-e per head
   int32_t* qexp;    // [max_batch, L, 64] the exponent e of each head's scaling
   int* d_err;       // device error word
+  // tensor-core query path (three-pass TF32): each fp32 weight w is kept as
+  // hi = tf32(w) and lo = w - hi, and so are the activations
+  int tc_ok;        // the weight tensor maps could be encoded
+  float* w_down_hi; float* w_down_lo;  // [L*(R+H), HID]
+  float* w_up_hi; float* w_up_lo;      // [L*H*D, R]
+  float* x_hi; float* x_lo;            // [max_batch, HID] hidden, split
+  float* r_hi; float* r_lo;            // [max_batch, L, R] RMSNorm output, split
+  float* up_part;                      // [2, max_batch, L*H*D] K-split partial sums of wq_b . r
+  alignas(64) unsigned char wmaps[4][128];  // TMA tensor maps: w_down hi, lo; w_up hi, lo
 };
 
 namespace fm {
@@ -58,6 +67,9 @@ fm_status launch_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* pos
                             float* q, float* fused_w, cudaStream_t stream);
 fm_status launch_qpack(fm_ctx* ctx, const float* q, const float* fused_w, int B,
                        cudaStream_t stream);
+// Splits the weights for the tensor-core query path and encodes their tensor
+// maps (fm_create); leaves tc_ok = 0 when the maps cannot be encoded.
+fm_status prepare_tc_weights(fm_ctx* ctx);
 
 struct ScoreArgs {
   const uint8_t* comp_k[kMaxLayers];
@@ -283,6 +295,36 @@ __device__ __forceinline__ void tmem_st32_st1_wait(uint32_t taddr, const uint32_
       "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
       "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
       "r"(v[29]), "r"(v[30]), "r"(v[31]), "r"(taddr1), "r"(v1)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, tf32 inputs (fp32 containers,
+// the low 13 mantissa bits ignored), fp32 accumulate.
+__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Tiled TMA loads (no multicast) of a box at the given element coordinates,
+// completing on `bar`.  The innermost coordinate times the element size is a
+// multiple of 16 bytes at every call site.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
 

@@ -14,6 +14,8 @@
 //   qup_kernel    one CTA per (layer, head, row block): the 128 rows of one
 //                 head of wq_b, then RoPE and the 128-point Hadamard butterfly
 //                 in registers (warp shuffles), writing q in fp32.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_fp8.h>
 
 #include "fm_internal.cuh"
@@ -153,13 +155,180 @@ __global__ void __launch_bounds__(kThreads) qdown_kernel(const float* __restrict
   }
 }
 
+// fp32 -> tf32 (round to nearest, ties away; low 13 mantissa bits zero).
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+// x = hi + lo with hi = tf32(x): the operand split of three-pass TF32.
+__global__ void split_tf32_kernel(const float* __restrict__ x, float* __restrict__ hi,
+                                  float* __restrict__ lo, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float v = x[i];
+    const float h = tf32_round(v);
+    hi[i] = h;
+    lo[i] = v - h;
+  }
+}
+
+// ------------------------------------------------ tensor-core skinny GEMM
+// part[s][n][m] = sum over K split s of W[m][k] X[n][k], with both operands
+// given as hi + lo pairs and the product taken as hi*hi + hi*lo + lo*hi
+// (three TF32 MMAs, fp32 accumulation in TMEM): fp32-level accuracy at
+// tensor-core speed.  One CTA per (128 rows of W, K split, BN columns of X);
+// warp 0 lane 0 feeds a ring of shared-memory stages with tiled TMA loads of
+// the four 128B-swizzled tiles, warp 1 lane 0 issues the MMAs, and all four
+// warps read the accumulator (one TMEM lane quarter each) and store it.
+constexpr int kTcThreads = 128;
+constexpr int kTcBM = 128;                              // rows of W per CTA (MMA M)
+constexpr int kTcBK = 32;                               // K per stage: 32 fp32 = one 128-byte row
+constexpr uint32_t kTcWTile = kTcBM * kTcBK * 4;        // 16 KB
+
+struct TcGemmArgs {
+  int M, N, K;          // W [M, K]; X [N, K] (one layer of it); part [split][N][M]
+  int kb_per_split;     // K blocks of 32 per split (every split has exactly this many)
+  int rows_per_layer;   // W rows per X layer (the up projection); 0: X has one layer
+  float* part;
+  int64_t split_stride;
+  int* err;
+};
+
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
+  return (1u << 4)                                // D format F32
+         | (2u << 7) | (2u << 10)                 // A, B format TF32
+         | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
+}
+
+template <int BN>
+constexpr uint32_t tc_stage_bytes() { return 2u * kTcWTile + 2u * BN * kTcBK * 4; }
+
+template <int BN>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap w_hi, const __grid_constant__ CUtensorMap w_lo,
+                   const __grid_constant__ CUtensorMap x_hi, const __grid_constant__ CUtensorMap x_lo,
+                   TcGemmArgs a, int S) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  constexpr uint32_t kXTile = BN * kTcBK * 4;
+  constexpr uint32_t kStage = tc_stage_bytes<BN>();
+  constexpr uint32_t kCols = BN;  // BN in {32, 64, 128, 256}: a valid TMEM allocation
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * kStage);
+  uint64_t* empty = full + S;
+  uint64_t* done = empty + S;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kTcBM, n0 = blockIdx.z * BN;
+  const int kb0 = blockIdx.y * a.kb_per_split, nkb = a.kb_per_split;
+  const int layer = a.rows_per_layer ? m0 / a.rows_per_layer : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(done, 1);
+    *sAbort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    tmem_alloc(sTmem, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sTmem;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t stage = 0, phase = 0, issued = 0;
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!mbar_wait_bounded(&empty[stage], phase ^ 1, sAbort, a.err)) break;
+      uint8_t* st = smem + (size_t)stage * kStage;
+      const int k = (kb0 + kb) * kTcBK;
+      mbar_arrive_expect_tx(&full[stage], kStage);
+      tma_load_2d(st, &w_hi, k, m0, &full[stage]);
+      tma_load_2d(st + kTcWTile, &w_lo, k, m0, &full[stage]);
+      tma_load_3d(st + 2 * kTcWTile, &x_hi, k, layer, n0, &full[stage]);
+      tma_load_3d(st + 2 * kTcWTile + kXTile, &x_lo, k, layer, n0, &full[stage]);
+      ++issued;
+      if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
+    }
+    // every copy issued lands before the CTA can exit
+    const uint32_t inflight = issued < (uint32_t)S ? issued : (uint32_t)S;
+    for (uint32_t j = 0; j < inflight; ++j) {
+      const uint32_t it = issued - 1 - j;
+      mbar_drain(&full[it % S], (it / S) & 1, a.err);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = idesc_tf32_f32(kTcBM, BN);
+    uint32_t stage = 0, phase = 0;
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!mbar_wait_bounded(&full[stage], phase, sAbort, a.err)) break;
+      tc_fence_after();
+      const uint32_t base = smem_u32(smem + (size_t)stage * kStage);
+      const uint64_t dwh = sdesc_kmajor_sw128(base), dwl = sdesc_kmajor_sw128(base + kTcWTile);
+      const uint64_t dxh = sdesc_kmajor_sw128(base + 2 * kTcWTile);
+      const uint64_t dxl = sdesc_kmajor_sw128(base + 2 * kTcWTile + kXTile);
+#pragma unroll
+      for (int k = 0; k < kTcBK / 8; ++k) {  // K = 8 tf32 (32 bytes) per MMA
+        const uint64_t o = 2u * (uint32_t)k;  // +32 bytes in the 16-byte address field
+        umma_tf32(tmem, dwh + o, dxh + o, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+        umma_tf32(tmem, dwh + o, dxl + o, idesc, 1u);
+        umma_tf32(tmem, dwl + o, dxh + o, idesc, 1u);
+      }
+      umma_commit(&empty[stage]);  // the stage may be refilled once these MMAs retire
+      if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
+    }
+    umma_commit(done);
+  }
+  // ------------------------------------------------------------ epilogue
+  int good = 1;
+  if (lane == 0) good = mbar_wait_bounded(done, 0, sAbort, a.err) && !*sAbort;
+  good = __shfl_sync(0xffffffffu, good, 0);
+  tc_fence_after();
+  if (good) {
+    const int m = m0 + warp * 32 + lane;
+    float* out = a.part + (int64_t)blockIdx.y * a.split_stride;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      uint32_t v[32];
+      tmem_ld32_wait(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+      if (m < a.M) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int n = n0 + c0 + j;
+          if (n < a.N) out[(int64_t)n * a.M + m] = __uint_as_float(v[j]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
+// The up projection's K-split partials summed, then RoPE and the Hadamard:
+// one warp per (row, layer, head).
+__global__ void __launch_bounds__(kThreads) qup_finish_kernel(const float* __restrict__ part, int ksplit,
+                                                              int64_t split_stride, int B, int L,
+                                                              const float* __restrict__ rope_cs,
+                                                              float* __restrict__ q);
+
 // One CTA per (row b, layer l): reduce the K splits, RMSNorm the wq_a part,
 // scale the weights_proj part into fused_w, and (layer 0) the RoPE table.
 __global__ void __launch_bounds__(kThreads) qnorm_kernel(
     const float* __restrict__ a_part, int ksplit, int B, int L, int R, int H,
     const float* __restrict__ q_norm, float eps, float w_scale, const int64_t* __restrict__ positions,
     const double* __restrict__ rope_freq, int rope_half, float* __restrict__ r_norm,
-    float* __restrict__ fused_w, float* __restrict__ rope_cs) {
+    float* __restrict__ fused_w, float* __restrict__ rope_cs, float* __restrict__ r_hi,
+    float* __restrict__ r_lo) {
   const int b = blockIdx.x, l = blockIdx.y;
   const int M = L * (R + H);
   const float* base = a_part + (size_t)b * M + (size_t)l * (R + H);
@@ -181,7 +350,13 @@ __global__ void __launch_bounds__(kThreads) qnorm_kernel(
   for (int i = threadIdx.x; i < R; i += kThreads) {
     float a = 0.f;
     for (int s = 0; s < ksplit; ++s) a += base[(size_t)s * B * M + i];
-    r_norm[((size_t)b * L + l) * R + i] = a * inv_rms * q_norm[(size_t)l * R + i];
+    const float r = a * inv_rms * q_norm[(size_t)l * R + i];
+    r_norm[((size_t)b * L + l) * R + i] = r;
+    if (r_hi) {  // the split operand of the tensor-core up projection
+      const float hi = tf32_round(r);
+      r_hi[((size_t)b * L + l) * R + i] = hi;
+      r_lo[((size_t)b * L + l) * R + i] = r - hi;
+    }
   }
   for (int h = threadIdx.x; h < H; h += kThreads) {
     float a = 0.f;
@@ -195,6 +370,75 @@ __global__ void __launch_bounds__(kThreads) qnorm_kernel(
     sincos(theta, &sn, &cs);
     rope_cs[((size_t)b * rope_half + j) * 2 + 0] = (float)cs;
     rope_cs[((size_t)b * rope_half + j) * 2 + 1] = (float)sn;
+  }
+}
+
+// RoPE on dims 64..127 (pairs (64+j, 96+j)) and the normalised Hadamard of
+// one head vector held by a warp, four dims per lane (lane holds dims
+// 4*lane .. 4*lane+3), written to q[b, l, h, :].
+__device__ __forceinline__ void rope_wht_store(float x[4], int b, int l, int h, int L, int lane,
+                                               const float* __restrict__ rope_cs,
+                                               float* __restrict__ q) {
+  // RoPE: lanes 16..23 hold dims 64..95 (x1), lanes 24..31 dims 96..127 (x2)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float other = __shfl_xor_sync(0xffffffffu, x[i], 8);
+    if (lane >= 16) {
+      const int j = (lane * 4 + i - 64) & 31;
+      const float c = rope_cs[((size_t)b * 32 + j) * 2 + 0];
+      const float s = rope_cs[((size_t)b * 32 + j) * 2 + 1];
+      x[i] = (lane < 24) ? (x[i] * c - other * s) : (x[i] * c + other * s);
+    }
+  }
+  // Walsh-Hadamard butterflies, Sylvester order: bits 0,1 inside the thread,
+  // bits 2..6 across lanes.
+  {
+    float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
+    x[0] = a0 + a2; x[2] = a0 - a2; x[1] = a1 + a3; x[3] = a1 - a3;
+  }
+#pragma unroll
+  for (int sbit = 0; sbit < 5; ++sbit) {
+    const int mask = 1 << sbit;
+    const bool upper = (lane & mask) != 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[i], mask);
+      x[i] = upper ? (o - x[i]) : (x[i] + o);
+    }
+  }
+  const float inv_sqrt_d = 0.088388347648318440f;  // 128^-1/2
+  float* dst = q + (((size_t)b * L + l) * kHeads + h) * kHeadDim + lane * 4;
+  *reinterpret_cast<float4*>(dst) =
+      make_float4(x[0] * inv_sqrt_d, x[1] * inv_sqrt_d, x[2] * inv_sqrt_d, x[3] * inv_sqrt_d);
+}
+
+__global__ void __launch_bounds__(kThreads) qup_finish_kernel(const float* __restrict__ part, int ksplit,
+                                                              int64_t split_stride, int B, int L,
+                                                              const float* __restrict__ rope_cs,
+                                                              float* __restrict__ q) {
+  const int idx = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);  // (b*L + l)*64 + h
+  if (idx >= B * L * kHeads) return;
+  const int lane = threadIdx.x & 31;
+  const int h = idx % kHeads, bl = idx / kHeads, l = bl % L, b = bl / L;
+  const float* src = part + (size_t)b * L * kHeads * kHeadDim + ((size_t)l * kHeads + h) * kHeadDim + lane * 4;
+  float4 acc = __ldg(reinterpret_cast<const float4*>(src));
+  for (int s = 1; s < ksplit; ++s) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(src + (int64_t)s * split_stride));
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  float x[4] = {acc.x, acc.y, acc.z, acc.w};
+  rope_wht_store(x, b, l, h, L, lane, rope_cs, q);
+}
+
+// The same for rows [b0, b0 + nb) of one head staged in Cs ([rows, 128]
+// floats); one warp per row.
+__device__ __forceinline__ void qup_epilogue(const float* Cs, int rows, int b0, int nb, int L, int l,
+                                             int h, int lane, int warp, const float* __restrict__ rope_cs,
+                                             float* __restrict__ q) {
+  for (int bl = warp; bl < nb && bl < rows; bl += kThreads / 32) {
+    const float4 v4 = *reinterpret_cast<const float4*>(&Cs[bl * kHeadDim + lane * 4]);
+    float x[4] = {v4.x, v4.y, v4.z, v4.w};
+    rope_wht_store(x, b0 + bl, l, h, L, lane, rope_cs, q);
   }
 }
 
@@ -216,54 +460,25 @@ __global__ void __launch_bounds__(kThreads) qup_kernel(const float* __restrict__
   Tile t;
   t.run(W, R, kHeadDim, r_norm + ((size_t)b0 * L + l) * R, L * R, nb, 0, 0, R, Ws, Xs);
 
-  // stage the [BN, 128] head block through shared memory (reuse Ws)
-  __syncthreads();
-  float* Cs = &Ws[0][0];  // BN * 128 floats <= BK * BM_PAD for BN <= 32
+  // stage the [BN, 128] head block through shared memory (reuse Ws), at most
+  // 32 rows at a time (32 * 128 floats <= BK * BM_PAD)
+  constexpr int kStageRows = Tile::BN < 32 ? Tile::BN : 32;
+  float* Cs = &Ws[0][0];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-#pragma unroll
-  for (int j = 0; j < TN; ++j) {
-    const int bl = ty * TN + j;
-    *reinterpret_cast<float4*>(&Cs[bl * kHeadDim + tx * 4]) =
-        make_float4(t.acc[0][j], t.acc[1][j], t.acc[2][j], t.acc[3][j]);
-  }
-  __syncthreads();
-
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int bl = warp; bl < nb; bl += kThreads / 32) {
-    const int b = b0 + bl;
-    float4 v4 = *reinterpret_cast<const float4*>(&Cs[bl * kHeadDim + lane * 4]);
-    float x[4] = {v4.x, v4.y, v4.z, v4.w};
-    // RoPE: lanes 16..23 hold dims 64..95 (x1), lanes 24..31 dims 96..127 (x2)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float other = __shfl_xor_sync(0xffffffffu, x[i], 8);
-      if (lane >= 16) {
-        const int j = (lane * 4 + i - 64) & 31;
-        const float c = rope_cs[((size_t)b * 32 + j) * 2 + 0];
-        const float s = rope_cs[((size_t)b * 32 + j) * 2 + 1];
-        x[i] = (lane < 24) ? (x[i] * c - other * s) : (x[i] * c + other * s);
-      }
-    }
-    // Walsh-Hadamard butterflies, Sylvester order: bits 0,1 inside the thread,
-    // bits 2..6 across lanes.
-    {
-      float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
-      x[0] = a0 + a2; x[2] = a0 - a2; x[1] = a1 + a3; x[3] = a1 - a3;
-    }
+  for (int half = 0; half < Tile::BN / kStageRows; ++half) {
+    __syncthreads();
 #pragma unroll
-    for (int sbit = 0; sbit < 5; ++sbit) {
-      const int mask = 1 << sbit;
-      const bool upper = (lane & mask) != 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, x[i], mask);
-        x[i] = upper ? (o - x[i]) : (x[i] + o);
-      }
+    for (int j = 0; j < TN; ++j) {
+      const int bl = ty * TN + j - half * kStageRows;
+      if (bl >= 0 && bl < kStageRows)
+        *reinterpret_cast<float4*>(&Cs[bl * kHeadDim + tx * 4]) =
+            make_float4(t.acc[0][j], t.acc[1][j], t.acc[2][j], t.acc[3][j]);
     }
-    const float inv_sqrt_d = 0.088388347648318440f;  // 128^-1/2
-    float* dst = q + (((size_t)b * L + l) * kHeads + h) * kHeadDim + lane * 4;
-    *reinterpret_cast<float4*>(dst) =
-        make_float4(x[0] * inv_sqrt_d, x[1] * inv_sqrt_d, x[2] * inv_sqrt_d, x[3] * inv_sqrt_d);
+    __syncthreads();
+    qup_epilogue(Cs, kStageRows, b0 + half * kStageRows, min(kStageRows, nb - half * kStageRows), L, l,
+                 h, lane, warp, rope_cs, q);
   }
 }
 
@@ -341,10 +556,160 @@ void launch_qup(fm_ctx* ctx, int B, float* q, cudaStream_t st) {
   note_launch();
 }
 
+// ------------------------------------------------ tensor maps (host)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+// fp32 tensor of `rank` dims (innermost first), 128-byte swizzled boxes of
+// 32 elements along dim 0; out-of-range elements of a box read as zero.
+bool encode_f32_map(void* map, const float* base, int rank, const cuuint64_t* dims,
+                    const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint32_t elem[3] = {1, 1, 1};
+  return enc(reinterpret_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (cuuint32_t)rank,
+             const_cast<float*>(base), dims, strides_bytes, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// W [rows, K] row-major, boxes of 32 x 128 rows.
+bool encode_weight_map(void* map, const float* w, int rows, int K) {
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 4};
+  const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcBM};
+  return encode_f32_map(map, w, 2, dims, strides, box);
+}
+
+// X [n, layers, K] row-major (K innermost), boxes of 32 x 1 x bn.
+bool encode_act_map(void* map, const float* x, int n, int layers, int K, int bn) {
+  const cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)layers, (cuuint64_t)n};
+  const cuuint64_t strides[2] = {(cuuint64_t)K * 4, (cuuint64_t)K * layers * 4};
+  const cuuint32_t box[3] = {(cuuint32_t)kTcBK, 1u, (cuuint32_t)bn};
+  return encode_f32_map(map, x, 3, dims, strides, box);
+}
+
+void launch_split(const float* x, float* hi, float* lo, int64_t n, cudaStream_t st) {
+  const int64_t g = (n + 255) / 256;
+  split_tf32_kernel<<<(unsigned)(g < 4096 ? g : 4096), 256, 0, st>>>(x, hi, lo, n);
+  note_launch();
+}
+
+template <int BN>
+fm_status launch_tc_gemm_bn(fm_ctx* ctx, const void* wh, const void* wl, const void* xh, const void* xl,
+                            const TcGemmArgs& a, int mtiles, int ksplit, int ntiles, cudaStream_t st) {
+  static int configured_dev = -1;
+  constexpr uint32_t stage = tc_stage_bytes<BN>();
+  int S = (int)((200u * 1024u) / stage);
+  S = S < 2 ? 2 : (S > 6 ? 6 : S);
+  const uint32_t smem = (uint32_t)S * stage + (uint32_t)(2 * S + 1) * 8 + 16 + 1024;
+  if (configured_dev != ctx->device) {
+    if (cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return check_launch();
+    configured_dev = ctx->device;
+  }
+  tc_gemm_kernel<BN><<<dim3(mtiles, ksplit, ntiles), kTcThreads, smem, st>>>(
+      *reinterpret_cast<const CUtensorMap*>(wh), *reinterpret_cast<const CUtensorMap*>(wl),
+      *reinterpret_cast<const CUtensorMap*>(xh), *reinterpret_cast<const CUtensorMap*>(xl), a, S);
+  note_launch();
+  return check_launch();
+}
+
+// part[s][n][m] for W (maps wh, wl: [M, K]) against X (maps xh, xl) in K splits.
+fm_status launch_tc_gemm(fm_ctx* ctx, const void* wh, const void* wl, const float* x_hi, const float* x_lo,
+                         int x_layers, int M, int N, int K, int ksplit, int rows_per_layer, float* part,
+                         cudaStream_t st) {
+  const int bn = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+  alignas(64) unsigned char xh[128], xl[128];
+  if (!encode_act_map(xh, x_hi, N, x_layers, K, bn) || !encode_act_map(xl, x_lo, N, x_layers, K, bn))
+    return FM_ERR_CUDA;
+  TcGemmArgs a;
+  a.M = M; a.N = N; a.K = K;
+  a.kb_per_split = K / kTcBK / ksplit;
+  a.rows_per_layer = rows_per_layer;
+  a.part = part;
+  a.split_stride = (int64_t)N * M;
+  a.err = ctx->d_err;
+  const int mtiles = (M + kTcBM - 1) / kTcBM, ntiles = (N + bn - 1) / bn;
+  switch (bn) {
+    case 32: return launch_tc_gemm_bn<32>(ctx, wh, wl, xh, xl, a, mtiles, ksplit, ntiles, st);
+    case 64: return launch_tc_gemm_bn<64>(ctx, wh, wl, xh, xl, a, mtiles, ksplit, ntiles, st);
+    case 128: return launch_tc_gemm_bn<128>(ctx, wh, wl, xh, xl, a, mtiles, ksplit, ntiles, st);
+    default: return launch_tc_gemm_bn<256>(ctx, wh, wl, xh, xl, a, mtiles, ksplit, ntiles, st);
+  }
+}
+
+// The query chain with both projections on the tensor cores (three-pass TF32).
+fm_status launch_query_prep_tc(fm_ctx* ctx, const float* hidden, const int64_t* positions, int B,
+                               float* q, float* fused_w, cudaStream_t st) {
+  const fm_config& c = ctx->cfg;
+  const int L = c.n_layers, R = c.q_lora_rank, HID = c.hidden;
+  const int Md = L * (R + kHeads), Mu = L * kHeads * kHeadDim;
+  const int bn_tiles = (B + 255) / 256;
+  // down projection: K splits until every SM has a CTA (splits divide K/32)
+  const int mtiles_d = (Md + kTcBM - 1) / kTcBM;
+  int ks_d = 1;
+  while (ks_d * 2 <= ctx->splitk_max && (HID / kTcBK) % (ks_d * 2) == 0 && mtiles_d * bn_tiles * ks_d < ctx->num_sms)
+    ks_d *= 2;
+  launch_split(hidden, ctx->x_hi, ctx->x_lo, (int64_t)B * HID, st);
+  fm_status s = launch_tc_gemm(ctx, ctx->wmaps[0], ctx->wmaps[1], ctx->x_hi, ctx->x_lo, 1, Md, B, HID, ks_d, 0,
+                               ctx->a_part, st);
+  if (s != FM_OK) return s;
+  const float w_scale = (float)(1.0 / sqrt((double)c.head_dim * (double)c.n_heads));
+  qnorm_kernel<<<dim3(B, L), kThreads, 0, st>>>(ctx->a_part, ks_d, B, L, R, c.n_heads, ctx->q_norm, c.rms_eps,
+                                                 w_scale, positions, ctx->rope_freq, c.rope_dim / 2,
+                                                 ctx->r_norm, fused_w, ctx->rope_cs, ctx->r_hi, ctx->r_lo);
+  note_launch();
+  // up projection: two K splits (its partials buffer holds two)
+  const int ks_u = (R / kTcBK) % 2 == 0 ? 2 : 1;
+  s = launch_tc_gemm(ctx, ctx->wmaps[2], ctx->wmaps[3], ctx->r_hi, ctx->r_lo, L, Mu, B, R, ks_u,
+                     kHeads * kHeadDim, ctx->up_part, st);
+  if (s != FM_OK) return s;
+  const int warps = B * L * kHeads;
+  qup_finish_kernel<<<(warps + kThreads / 32 - 1) / (kThreads / 32), kThreads, 0, st>>>(
+      ctx->up_part, ks_u, (int64_t)B * Mu, B, L, ctx->rope_cs, q);
+  note_launch();
+  return check_launch();
+}
+
 }  // namespace
+
+fm_status prepare_tc_weights(fm_ctx* ctx) {
+  const fm_config& c = ctx->cfg;
+  const int L = c.n_layers, R = c.q_lora_rank, HID = c.hidden;
+  const int Md = L * (R + kHeads), Mu = L * kHeads * kHeadDim;
+  ctx->tc_ok = 0;
+  launch_split(ctx->w_down, ctx->w_down_hi, ctx->w_down_lo, (int64_t)Md * HID, 0);
+  launch_split(ctx->w_up, ctx->w_up_hi, ctx->w_up_lo, (int64_t)Mu * R, 0);
+  const fm_status s = check_launch();
+  if (s != FM_OK) return s;
+  ctx->tc_ok = encode_weight_map(ctx->wmaps[0], ctx->w_down_hi, Md, HID) &&
+               encode_weight_map(ctx->wmaps[1], ctx->w_down_lo, Md, HID) &&
+               encode_weight_map(ctx->wmaps[2], ctx->w_up_hi, Mu, R) &&
+               encode_weight_map(ctx->wmaps[3], ctx->w_up_lo, Mu, R);
+  return FM_OK;
+}
 
 fm_status launch_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* positions, int B,
                             float* q, float* fused_w, cudaStream_t st) {
+  // Past 8 rows the projections are bound by fp32 FMA on the CUDA cores; the
+  // tensor-core path then reads twice the weight bytes (hi and lo) at a far
+  // higher math rate.  Up to 8 rows the CUDA-core GEMVs read the weights once.
+  if (ctx->tc_ok && B > 8) return launch_query_prep_tc(ctx, hidden, positions, B, q, fused_w, st);
   const fm_config& c = ctx->cfg;
   const int M = c.n_layers * (c.q_lora_rank + c.n_heads);
   const int mtiles = (M + BM - 1) / BM;
@@ -366,13 +731,20 @@ fm_status launch_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* pos
   const float w_scale = (float)(1.0 / sqrt((double)c.head_dim * (double)c.n_heads));
   qnorm_kernel<<<dim3(B, c.n_layers), kThreads, 0, st>>>(
       ctx->a_part, ksplit, B, c.n_layers, c.q_lora_rank, c.n_heads, ctx->q_norm, c.rms_eps,
-      w_scale, positions, ctx->rope_freq, c.rope_dim / 2, ctx->r_norm, fused_w, ctx->rope_cs);
+      w_scale, positions, ctx->rope_freq, c.rope_dim / 2, ctx->r_norm, fused_w, ctx->rope_cs, nullptr,
+      nullptr);
   note_launch();
 
+  // one row block covers the batch up to 64 rows, so each head's wq_b rows
+  // are read once per 64 rows
   if (B <= 8)
     launch_qup<1>(ctx, B, q, st);
-  else
+  else if (B <= 16)
     launch_qup<2>(ctx, B, q, st);
+  else if (B <= 32)
+    launch_qup<4>(ctx, B, q, st);
+  else
+    launch_qup<8>(ctx, B, q, st);
   return check_launch();
 }
 

@@ -136,13 +136,26 @@ __global__ void __launch_bounds__(kThreads) topk_hist_kernel(Workspace w, const 
   __syncthreads();
   const int64_t base = (int64_t)blockIdx.x * kChunk;
   const float* row = ens + (int64_t)b * N;
-#pragma unroll 4
+  // all loads first (16 in flight per thread), then the counting
+  float v[kPerThread];
+#pragma unroll
   for (int i = 0; i < kPerThread; ++i) {
     const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
-    if (n < nv) {
-      const uint32_t key = order_key(row[n]);
-      const bool match = (hi_shift >= 32) || ((key >> (hi_shift & 31)) == (prefix >> (hi_shift & 31)));
-      if (match) atomicAdd(&sh[(key >> shift) & (bins - 1)], 1u);
+    v[i] = n < nv ? __ldg(row + n) : 0.f;
+  }
+  // Scores crowd into a few digits (sigmoid outputs share their exponent), so
+  // lanes holding the same digit are counted with one shared-memory atomic.
+  const unsigned lane_lt = (1u << (threadIdx.x & 31)) - 1u;
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
+    const uint32_t key = order_key(v[i]);
+    const bool act = n < nv && ((hi_shift >= 32) || ((key >> (hi_shift & 31)) == (prefix >> (hi_shift & 31))));
+    const unsigned active = __ballot_sync(0xffffffffu, act);
+    if (act) {
+      const uint32_t bin = (key >> shift) & (bins - 1);
+      const unsigned peers = __match_any_sync(active, bin);
+      if ((peers & lane_lt) == 0) atomicAdd(&sh[bin], (uint32_t)__popc(peers));
     }
   }
   __syncthreads();
@@ -235,6 +248,25 @@ __global__ void __launch_bounds__(kThreads) topk_mask_kernel(Workspace w, const 
   const float* row = ens + (int64_t)b * N;
   uint8_t* out = keep + (int64_t)b * N;
   if (!split_tie) {
+    if ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(ens) & 15u) == 0 &&
+        (reinterpret_cast<uintptr_t>(keep) & 3u) == 0) {
+      // four consecutive chunks per thread: 16-byte loads, one 4-byte mask store
+#pragma unroll
+      for (int i = 0; i < kPerThread / 4; ++i) {
+        const int64_t n = base + ((int64_t)i * kThreads + threadIdx.x) * 4;
+        if (n >= N) break;
+        const float4 e = __ldg(reinterpret_cast<const float4*>(row + n));
+        const float ev[4] = {e.x, e.y, e.z, e.w};
+        uint32_t word = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const bool k = n + c < nv && (mode == kModeAll || order_key(ev[c]) >= T);
+          word |= (k ? 1u : 0u) << (8 * c);
+        }
+        *reinterpret_cast<uint32_t*>(out + n) = word;
+      }
+      return;
+    }
     for (int i = 0; i < kPerThread; ++i) {
       const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
       if (n >= N) break;

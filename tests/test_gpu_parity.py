@@ -82,6 +82,32 @@ def test_tile_dot_products_layout(retr, weights):
         assert np.all(np.abs(rec - exact) <= bound), np.abs(rec - exact).max()
 
 
+@pytest.mark.parametrize("B", [24, 40, 64, 300])
+def test_query_prep_tensor_core_path_matches_oracle(weights, B):
+    """Past 8 rows both projections run on the tensor cores (three-pass TF32:
+    hi*hi + hi*lo + lo*hi with hi = tf32(x)); the result must keep fp32-level
+    accuracy.  300 rows take two 256-column tiles."""
+    g = np.random.default_rng(100 + B)
+    hidden = g.standard_normal((B, G.HIDDEN)).astype(np.float32)
+    pos = g.integers(0, 1 << 20, size=B).astype(np.int64)
+    r = fm.Retriever(weights, device=0, max_batch=max(64, B))
+    try:
+        q, w = r.fm_query_prep(torch.from_numpy(hidden).to(DEV), torch.from_numpy(pos).to(DEV))
+        torch.cuda.synchronize()
+        r.fm_sync_status()
+        layers = H.np_layers(weights)
+        for b in range(0, B, max(1, B // 7)):  # a spread of rows, through the oracle
+            qo, wo = zip(*[O.query_prep(lw, hidden[b:b + 1].astype(np.float64), pos[b:b + 1]) for lw in layers])
+            qo = np.stack([x[0] for x in qo])  # [L, H, D]
+            wo = np.stack([x[0] for x in wo])  # [L, H]
+            qg = q[b].cpu().numpy().astype(np.float64)
+            err = np.linalg.norm(qg - qo, axis=-1) / np.linalg.norm(qo, axis=-1)
+            assert err.max() < 2e-5, (b, err.max())
+            np.testing.assert_allclose(w[b].cpu().numpy(), wo, rtol=1e-4, atol=1e-6)
+    finally:
+        r.close()
+
+
 @pytest.mark.parametrize("shape", [
     dict(B=1, N=4096, nv=[4096]),
     dict(B=3, N=1001, nv=[1001, 517, 0]),
