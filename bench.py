@@ -50,6 +50,24 @@ def parse():
     return ap.parse_args()
 
 
+def recorded_traffic(decisions: int):
+    """DRAM bytes per scoring launch from the committed ncu summary, scaled to
+    this launch's decisions; None once the kernel source differs from the one
+    the counters were taken on."""
+    import hashlib
+    import re
+    try:
+        text = open(os.path.join(ROOT, "profiles", "score_kernel_B8xN65536.md")).read()
+        sha = re.search(r"kernel_source_sha1: ([0-9a-f]{40})", text).group(1)
+        per = float(re.search(r"traffic_bytes_per_decision: ([0-9.]+)", text).group(1))
+        m = hashlib.sha1()
+        for f in ("score_tc.cu", "fm_internal.cuh"):
+            m.update(open(os.path.join(ROOT, "learned_kv_chunk_b200", "csrc", f), "rb").read())
+        return int(per * decisions) if m.hexdigest() == sha else None
+    except Exception:
+        return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -235,10 +253,11 @@ def run_ours(args, rank, world, local_rank):
     value = job_throughput(decisions, world, args.steps, elapsed_max)
 
     hbm_peak, peak_kind = peaks()
+    traffic = recorded_traffic(decisions)
     alg_bytes = decisions * (L * G.RECORD_BYTES + 4)  # keys + ensembled score per decision
     achieved = alg_bytes / (score_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                 "kernel": "score_kernel (fused scoring pass, via fm_score_fused)",
                 "kernel_ms": round(score_ms, 4), "peak_kind": peak_kind,
                 "alg_bytes_per_launch": alg_bytes}
