@@ -201,7 +201,7 @@ __device__ __forceinline__ float head_sum32(const HeadCols<P>& c, const float* _
   constexpr float kInv16 = 0.0625f, kInv256 = 0.00390625f;
   if (nonneg) {
     const uint64_t c16 = f2_pack(kInv16, kInv16), c256 = f2_pack(kInv256, kInv256);
-    uint64_t acc_a = f2_pack(0.f, 0.f), acc_b = f2_pack(0.f, 0.f);
+    uint64_t acc = f2_pack(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const uint64_t p0 = f2_pack(c.at(0, 2 * j), c.at(0, 2 * j + 1));
@@ -212,15 +212,11 @@ __device__ __forceinline__ float head_sum32(const HeadCols<P>& c, const float* _
       f2_unpack(d, dx, dy);
       const float2 ww = *reinterpret_cast<const float2*>(w + 2 * j);
       const uint64_t rr = f2_pack(fmaxf(dx, 0.f), fmaxf(dy, 0.f));
-      if (j & 1)
-        acc_b = f2_fma(rr, f2_pack(ww.x, ww.y), acc_b);
-      else
-        acc_a = f2_fma(rr, f2_pack(ww.x, ww.y), acc_a);
+      acc = f2_fma(rr, f2_pack(ww.x, ww.y), acc);  // one chain: fewer registers, same issue count
     }
-    float a0, a1, b0, b1;
-    f2_unpack(acc_a, a0, a1);
-    f2_unpack(acc_b, b0, b1);
-    return (a0 + a1) + (b0 + b1);
+    float a0, a1;
+    f2_unpack(acc, a0, a1);
+    return a0 + a1;
   }
   float acc = 0.f;
   for (int i = 0; i < 32; ++i) {

@@ -17,7 +17,7 @@
 namespace fm {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;  // top-K blocks: 8192 chunks each, so few per-block merges per row
 constexpr int kPerThread = 16;
 constexpr int kChunk = kThreads * kPerThread;  // elements per block slice
 constexpr int kBins0 = 2048, kBins1 = 2048, kBins2 = 1024;
