@@ -60,9 +60,11 @@ def recorded_traffic(decisions: int):
         text = open(os.path.join(ROOT, "profiles", "score_kernel_B8xN65536.md")).read()
         sha = re.search(r"kernel_source_sha1: ([0-9a-f]{40})", text).group(1)
         per = float(re.search(r"traffic_bytes_per_decision: ([0-9.]+)", text).group(1))
+        src = os.path.join(ROOT, "learned_kv_chunk_b200", "csrc")
         m = hashlib.sha1()
-        for f in ("score_tc.cu", "fm_internal.cuh"):
-            m.update(open(os.path.join(ROOT, "learned_kv_chunk_b200", "csrc", f), "rb").read())
+        m.update(open(os.path.join(src, "score_tc.cu"), "rb").read())
+        header = open(os.path.join(src, "fm_internal.cuh"), "rb").read()
+        m.update(header[header.index(b"#if defined(__CUDACC__)"):])  # the header's device code
         return int(per * decisions) if m.hexdigest() == sha else None
     except Exception:
         return None

@@ -204,6 +204,48 @@ fm_status fm_select_topk_static(const float* ens, const int32_t* n_valid, int B,
 fm_status fm_select_threshold(const float* ens, const int32_t* n_valid, int B, int N, float thr,
                               uint8_t* keep, cudaStream_t stream);
 
+/* Sharded top-K: the keep mask of fm_select_topk (README "Usage"
+ * select_topk(top_k=K)) for rows whose chunks are split over G shards (GPUs),
+ * shard g holding a consecutive slice of each row, slices in shard order.  The
+ * pages describe no multi-GPU form of the retriever; this is the same mask,
+ * computed without moving scores between shards: the caller runs the phases
+ * below on every shard in the same order and does the two exchanges between
+ * them (with NCCL or any other collective library):
+ *
+ *   fm_topk_shard_begin(n_valid_local, B, N, k, hist, ws, ...)
+ *   for pass in 0, 1, 2:
+ *     fm_topk_shard_hist(ens_local, B, N, pass, hist, ws, ...)
+ *     all-reduce (sum) `hist` over the shards            -- exchange 1
+ *     fm_topk_shard_pick(B, N, pass, hist, ws, ...)
+ *   fm_topk_shard_ties(ens_local, B, N, eq_local, ws, ...)
+ *   all-gather `eq_local` into eq_all [G, B], shard order -- exchange 2
+ *   fm_topk_shard_mask(ens_local, B, N, eq_all, g, keep_local, ws, ...)
+ *
+ * After it, the union of the shards' masks keeps, per row, the min(k, total
+ * valid) largest scores of the whole row, equal scores in increasing global
+ * chunk index, exactly as fm_select_topk on the concatenated row would.
+ * Every shard passes the same B and k; N (its slice length) may differ.
+ * ens_local [B, N] fp32 device: this shard's slice; n_valid_local [B] int32
+ * device or NULL (= N): valid chunks in this slice (a row's valid prefix
+ * split over the slices: clamp(n_b - slice_start, 0, N));
+ * hist [B, FM_TOPK_SHARD_BINS] int32 device, 16-byte aligned, owned by the
+ * caller, written by begin and pick, summed in place by the caller;
+ * eq_local [B] int32 device; eq_all [G, B] int32 device; keep_local [B, N]
+ * uint8 device; ws: this shard's workspace of fm_topk_workspace_bytes(B, N)
+ * bytes, 16-byte aligned, kept between the phases.  Exchange sizes: 8 KiB
+ * per row per pass, 4 bytes per row for the ties. */
+#define FM_TOPK_SHARD_BINS 2048
+fm_status fm_topk_shard_begin(const int32_t* n_valid_local, int B, int N, int k, int32_t* hist,
+                              void* ws, size_t ws_bytes, cudaStream_t stream);
+fm_status fm_topk_shard_hist(const float* ens_local, int B, int N, int pass, int32_t* hist, void* ws,
+                             size_t ws_bytes, cudaStream_t stream);
+fm_status fm_topk_shard_pick(int B, int N, int pass, int32_t* hist, void* ws, size_t ws_bytes,
+                             cudaStream_t stream);
+fm_status fm_topk_shard_ties(const float* ens_local, int B, int N, int32_t* eq_local, void* ws,
+                             size_t ws_bytes, cudaStream_t stream);
+fm_status fm_topk_shard_mask(const float* ens_local, int B, int N, const int32_t* eq_all, int shard,
+                             uint8_t* keep_local, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* Synchronises `stream` and returns FM_ERR_DEVICE if a kernel launched on this
  * context recorded an error since the last call (the record is cleared),
  * FM_ERR_CUDA if the stream reports a CUDA error, FM_OK otherwise. */

@@ -300,6 +300,52 @@ fm_status fm_select_threshold(const float* ens, const int32_t* n_valid, int B, i
   return launch_threshold(ens, n_valid, B, N, thr, keep, stream);
 }
 
+// Checks shared by the sharded top-K phases.
+static fm_status shard_args(int B, int N, const void* hist, const void* ws, size_t ws_bytes) {
+  if (!ws || B < 1 || N < 1 || B > 65535) return FM_ERR_INVALID_ARG;
+  if (!aligned(ws, 16) || (hist && !aligned(hist, 16))) return FM_ERR_ALIGNMENT;
+  if (ws_bytes < topk_workspace_bytes(B, N)) return FM_ERR_INVALID_ARG;
+  return FM_OK;
+}
+
+fm_status fm_topk_shard_begin(const int32_t* n_valid_local, int B, int N, int k, int32_t* hist,
+                              void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!hist || k < 1) return FM_ERR_INVALID_ARG;
+  if (fm_status s = shard_args(B, N, hist, ws, ws_bytes)) return s;
+  return launch_topk_shard_begin(n_valid_local, B, N, k, hist, ws, ws_bytes, stream);
+}
+
+fm_status fm_topk_shard_hist(const float* ens_local, int B, int N, int pass, int32_t* hist, void* ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+  if (!ens_local || !hist || pass < 0 || pass > 2) return FM_ERR_INVALID_ARG;
+  if (fm_status s = shard_args(B, N, hist, ws, ws_bytes)) return s;
+  if (!aligned(ens_local, 4)) return FM_ERR_ALIGNMENT;
+  return launch_topk_shard_hist(ens_local, B, N, pass, hist, ws, ws_bytes, stream);
+}
+
+fm_status fm_topk_shard_pick(int B, int N, int pass, int32_t* hist, void* ws, size_t ws_bytes,
+                             cudaStream_t stream) {
+  if (!hist || pass < 0 || pass > 2) return FM_ERR_INVALID_ARG;
+  if (fm_status s = shard_args(B, N, hist, ws, ws_bytes)) return s;
+  return launch_topk_shard_pick(B, N, pass, hist, ws, ws_bytes, stream);
+}
+
+fm_status fm_topk_shard_ties(const float* ens_local, int B, int N, int32_t* eq_local, void* ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+  if (!ens_local || !eq_local) return FM_ERR_INVALID_ARG;
+  if (fm_status s = shard_args(B, N, nullptr, ws, ws_bytes)) return s;
+  if (!aligned(ens_local, 4) || !aligned(eq_local, 4)) return FM_ERR_ALIGNMENT;
+  return launch_topk_shard_ties(ens_local, B, N, eq_local, ws, ws_bytes, stream);
+}
+
+fm_status fm_topk_shard_mask(const float* ens_local, int B, int N, const int32_t* eq_all, int shard,
+                             uint8_t* keep_local, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!ens_local || !eq_all || !keep_local || shard < 0) return FM_ERR_INVALID_ARG;
+  if (fm_status s = shard_args(B, N, nullptr, ws, ws_bytes)) return s;
+  if (!aligned(ens_local, 4) || !aligned(eq_all, 4)) return FM_ERR_ALIGNMENT;
+  return launch_topk_shard_mask(ens_local, B, N, eq_all, shard, keep_local, ws, ws_bytes, stream);
+}
+
 fm_status fm_sync_status(fm_ctx* c, cudaStream_t stream) {
   if (!c) return FM_ERR_INVALID_ARG;
   cudaError_t e = cudaStreamSynchronize(stream);

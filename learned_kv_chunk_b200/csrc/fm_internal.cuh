@@ -97,6 +97,16 @@ fm_status launch_threshold(const float* ens, const int32_t* n_valid, int B, int 
 size_t topk_workspace_bytes(int B, int N);
 fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, int k, uint8_t* keep,
                       void* ws, size_t ws_bytes, cudaStream_t stream);
+fm_status launch_topk_shard_begin(const int32_t* n_valid, int B, int N, int k, int32_t* hist, void* ws,
+                                  size_t ws_bytes, cudaStream_t stream);
+fm_status launch_topk_shard_hist(const float* ens, int B, int N, int pass, int32_t* hist, void* ws,
+                                 size_t ws_bytes, cudaStream_t stream);
+fm_status launch_topk_shard_pick(int B, int N, int pass, int32_t* hist, void* ws, size_t ws_bytes,
+                                 cudaStream_t stream);
+fm_status launch_topk_shard_ties(const float* ens, int B, int N, int32_t* eq_local, void* ws,
+                                 size_t ws_bytes, cudaStream_t stream);
+fm_status launch_topk_shard_mask(const float* ens, int B, int N, const int32_t* eq_all, int shard,
+                                 uint8_t* keep, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 // ------------------------------------------------------------ PTX wrappers
 #if defined(__CUDACC__)

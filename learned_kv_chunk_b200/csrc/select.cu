@@ -12,6 +12,14 @@
 // with a per-block count pass and an in-block ordered scan).  Each histogram
 // pass ends in its last-arriving block (atomic ticket, no waiting), which
 // chooses the digit for the row; no kernel waits on another block.
+//
+// The sharded form splits one row's chunks over several GPUs (each holds a
+// consecutive slice, in shard order).  The same passes run with the digit
+// choice taken out of the histogram kernel: each shard histograms its slice
+// into a caller buffer, the caller sums the buffers over the shards (one
+// all-reduce per pass), and every shard then picks the same digit from the
+// same global histogram.  Ties at T are ranked across shards by an exclusive
+// sum of the per-shard tie counts in shard order (one all-gather).
 #include "fm_internal.cuh"
 
 namespace fm {
@@ -22,6 +30,8 @@ constexpr int kPerThread = 16;
 constexpr int kChunk = kThreads * kPerThread;  // elements per block slice
 constexpr int kBins0 = 2048, kBins1 = 2048, kBins2 = 1024;
 constexpr int kHistWords = kBins0 + kBins1 + kBins2;
+constexpr int kShardBins = FM_TOPK_SHARD_BINS;  // row stride of the sharded form's histograms
+static_assert(kShardBins >= kBins0 && kShardBins >= kBins1 && kShardBins >= kBins2, "histogram row");
 constexpr int kShift[3] = {21, 10, 0};
 constexpr int kBits[3] = {11, 11, 10};
 
@@ -118,9 +128,92 @@ __global__ void topk_init_kernel(Workspace w, const int32_t* __restrict__ n_vali
   }
 }
 
-template <int PASS>
+// Chooses the digit of pass PASS holding the remaining-th largest key of the
+// row from its complete histogram `gh` (bins in digit order), one block of
+// kThreads; records the digit in the row state.  Thread t owns bins
+// [t*per, (t+1)*per) in descending order of value.  With CLEAR the thread
+// also zeroes the bins it read, ready for the next pass; with TOTAL (the first
+// pass of the sharded form) the row's mode is settled from the histogram's
+// total, which only the summed histogram knows.
+// Sharded form: this shard's row states (its own valid count; the mode is
+// settled by the first pick, from the summed histogram) and a zeroed histogram.
+__global__ void topk_shard_init_kernel(Workspace w, const int32_t* __restrict__ n_valid, int N, int k,
+                                       uint32_t* __restrict__ xh) {
+  const int b = blockIdx.x;
+  uint32_t* h = xh + (size_t)b * kShardBins;
+  for (int i = threadIdx.x; i < kShardBins; i += blockDim.x) h[i] = 0u;
+  if (threadIdx.x == 0) {
+    RowState s = {};
+    s.nv = row_nvalid(n_valid, b, N);
+    s.mode = kModeSelect;
+    s.prefix = 0u;
+    s.remaining = k;
+    w.state[b] = s;
+  }
+}
+
+template <int PASS, bool CLEAR, bool TOTAL>
+__device__ __forceinline__ void pick_digit(RowState* st, uint32_t* gh, uint32_t* s_suffix) {
+  constexpr int bins = PASS == 0 ? kBins0 : (PASS == 1 ? kBins1 : kBins2);
+  constexpr int shift = kShift[PASS];
+  constexpr int per = bins / kThreads;
+  // every thread reads the row state before the first barrier below: the one
+  // thread that finds the digit rewrites it after the last barrier
+  const uint32_t prefix = st->prefix;
+  const uint32_t want0 = (uint32_t)st->remaining;
+  uint32_t cnt[per];
+  uint32_t mine = 0;
+#pragma unroll
+  for (int j = 0; j < per; ++j) {
+    const int d = bins - 1 - (threadIdx.x * per + j);  // descending digit
+    cnt[j] = __ldcg(&gh[d]);
+    if (CLEAR) gh[d] = 0u;
+    mine += cnt[j];
+  }
+  s_suffix[threadIdx.x] = mine;
+  __syncthreads();
+  // inclusive scan over threads (descending digit order)
+  for (int off = 1; off < kThreads; off <<= 1) {
+    const uint32_t v = threadIdx.x >= off ? s_suffix[threadIdx.x - off] : 0u;
+    __syncthreads();
+    s_suffix[threadIdx.x] += v;
+    __syncthreads();
+  }
+  uint32_t want = want0;
+  if (TOTAL) {
+    const uint32_t total = s_suffix[kThreads - 1];
+    if (total == 0u || want >= total) {
+      if (threadIdx.x == 0) st->mode = total == 0u ? kModeEmpty : kModeAll;
+      return;
+    }
+  }
+  const uint32_t before = s_suffix[threadIdx.x] - mine;  // keys with a larger digit
+  if (before < want && before + mine >= want) {
+    uint32_t acc = before;
+#pragma unroll
+    for (int j = 0; j < per; ++j) {
+      if (acc + cnt[j] >= want) {
+        const int d = bins - 1 - (threadIdx.x * per + j);
+        st->prefix = prefix | ((uint32_t)d << shift);
+        st->remaining = (int)(want - acc);
+        if (PASS == 2) {
+          st->need_eq = (int)(want - acc);
+          st->cnt_eq = (int)cnt[j];
+        }
+        break;
+      }
+      acc += cnt[j];
+    }
+  }
+}
+
+// Histogram of digit PASS over the keys of the row that match the digits
+// chosen so far.  FUSED: into the workspace, and the last-arriving block of the
+// row picks the digit.  Otherwise (sharded form): into the caller's buffer
+// `xh` [B, kShardBins], for the caller to sum over the shards.
+template <int PASS, bool FUSED>
 __global__ void __launch_bounds__(kThreads) topk_hist_kernel(Workspace w, const float* __restrict__ ens,
-                                                             int N) {
+                                                             int N, uint32_t* __restrict__ xh) {
   constexpr int bins = PASS == 0 ? kBins0 : (PASS == 1 ? kBins1 : kBins2);
   constexpr int shift = kShift[PASS];
   constexpr int hi_shift = shift + kBits[PASS];  // digits above this pass
@@ -159,59 +252,34 @@ __global__ void __launch_bounds__(kThreads) topk_hist_kernel(Workspace w, const 
     }
   }
   __syncthreads();
-  uint32_t* gh = w.hist + (size_t)b * kHistWords + (PASS == 0 ? 0 : (PASS == 1 ? kBins0 : kBins0 + kBins1));
+  uint32_t* gh = FUSED ? w.hist + (size_t)b * kHistWords + (PASS == 0 ? 0 : (PASS == 1 ? kBins0 : kBins0 + kBins1))
+                       : xh + (size_t)b * kShardBins;
   for (int i = threadIdx.x; i < bins; i += kThreads)
     if (sh[i]) atomicAdd(&gh[i], sh[i]);
+  if (!FUSED) return;
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) s_last = (atomicAdd(&st->tickets[PASS], 1) == (int)gridDim.x - 1);
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // Last block of the row: pick the digit holding the remaining-th largest key.
-  // Thread t owns bins [t*per, (t+1)*per) in descending order of value.
-  constexpr int per = bins / kThreads;
-  uint32_t cnt[per];
-  uint32_t mine = 0;
-#pragma unroll
-  for (int j = 0; j < per; ++j) {
-    const int d = bins - 1 - (threadIdx.x * per + j);  // descending digit
-    cnt[j] = __ldcg(&gh[d]);
-    mine += cnt[j];
-  }
-  s_suffix[threadIdx.x] = mine;
-  __syncthreads();
-  // inclusive scan over threads (descending digit order)
-  for (int off = 1; off < kThreads; off <<= 1) {
-    const uint32_t v = threadIdx.x >= off ? s_suffix[threadIdx.x - off] : 0u;
-    __syncthreads();
-    s_suffix[threadIdx.x] += v;
-    __syncthreads();
-  }
-  const uint32_t before = s_suffix[threadIdx.x] - mine;  // keys with a larger digit
-  const uint32_t want = (uint32_t)st->remaining;
-  if (before < want && before + mine >= want) {
-    uint32_t acc = before;
-#pragma unroll
-    for (int j = 0; j < per; ++j) {
-      if (acc + cnt[j] >= want) {
-        const int d = bins - 1 - (threadIdx.x * per + j);
-        st->prefix = prefix | ((uint32_t)d << shift);
-        st->remaining = (int)(want - acc);
-        if (PASS == 2) {
-          st->need_eq = (int)(want - acc);
-          st->cnt_eq = (int)cnt[j];
-        }
-        break;
-      }
-      acc += cnt[j];
-    }
-  }
+  pick_digit<PASS, false, false>(st, gh, s_suffix);
 }
 
-// Per-block count of keys equal to T, only for rows whose tie at T is split.
+// Sharded form: the digit choice of pass PASS from the histogram summed over
+// the shards (one block per row); clears the histogram for the next pass.
+template <int PASS>
+__global__ void __launch_bounds__(kThreads) topk_shard_pick_kernel(Workspace w, uint32_t* __restrict__ xh) {
+  __shared__ uint32_t s_suffix[kThreads];
+  RowState* st = w.state + blockIdx.x;
+  if (st->mode != kModeSelect) return;
+  pick_digit<PASS, true, PASS == 0>(st, xh + (size_t)blockIdx.x * kShardBins, s_suffix);
+}
+
+// Per-block count of keys equal to T, only for rows whose tie at T is split;
+// with eq_row (zeroed by the caller) also the row's total over the blocks.
 __global__ void __launch_bounds__(kThreads) topk_eqcount_kernel(Workspace w, const float* __restrict__ ens,
-                                                                int N, int nblk) {
+                                                                int N, int nblk, int32_t* __restrict__ eq_row) {
   const int b = blockIdx.y;
   const RowState* st = w.state + b;
   if (st->mode != kModeSelect || st->need_eq == st->cnt_eq) return;
@@ -233,11 +301,16 @@ __global__ void __launch_bounds__(kThreads) topk_eqcount_kernel(Workspace w, con
     int t = 0;
     for (int i = 0; i < kThreads / 32; ++i) t += red[i];
     w.eqcnt[(size_t)b * nblk + blockIdx.x] = t;
+    if (eq_row && t) atomicAdd(eq_row + b, t);  // sharded form: the slice's total
   }
 }
 
+// eq_all [shards, B] (sharded form, else NULL): each shard's count of keys == T
+// per row; the ones of the shards before `shard` rank ahead of this slice's.
 __global__ void __launch_bounds__(kThreads) topk_mask_kernel(Workspace w, const float* __restrict__ ens,
-                                                             int N, int nblk, uint8_t* __restrict__ keep) {
+                                                             int N, int nblk, uint8_t* __restrict__ keep,
+                                                             const int32_t* __restrict__ eq_all, int shard,
+                                                             int B) {
   const int b = blockIdx.y;
   const RowState* st = w.state + b;
   const int mode = st->mode, nv = st->nv;
@@ -281,6 +354,8 @@ __global__ void __launch_bounds__(kThreads) topk_mask_kernel(Workspace w, const 
   __shared__ int s_warp[kThreads / 32];
   if (threadIdx.x == 0) {
     int p = 0;
+    if (eq_all)
+      for (int r = 0; r < shard; ++r) p += eq_all[(size_t)r * B + b];
     for (int j = 0; j < (int)blockIdx.x; ++j) p += w.eqcnt[(size_t)b * nblk + j];
     s_prefix = p;
   }
@@ -346,12 +421,80 @@ fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, in
   Workspace w = carve(ws, B, nblk);
   topk_init_kernel<<<B, 256, 0, st>>>(w, n_valid, N, k);
   dim3 grid(nblk, B);
-  topk_hist_kernel<0><<<grid, kThreads, 0, st>>>(w, ens, N);
-  topk_hist_kernel<1><<<grid, kThreads, 0, st>>>(w, ens, N);
-  topk_hist_kernel<2><<<grid, kThreads, 0, st>>>(w, ens, N);
-  topk_eqcount_kernel<<<grid, kThreads, 0, st>>>(w, ens, N, nblk);
-  topk_mask_kernel<<<grid, kThreads, 0, st>>>(w, ens, N, nblk, keep);
+  topk_hist_kernel<0, true><<<grid, kThreads, 0, st>>>(w, ens, N, nullptr);
+  topk_hist_kernel<1, true><<<grid, kThreads, 0, st>>>(w, ens, N, nullptr);
+  topk_hist_kernel<2, true><<<grid, kThreads, 0, st>>>(w, ens, N, nullptr);
+  topk_eqcount_kernel<<<grid, kThreads, 0, st>>>(w, ens, N, nblk, nullptr);
+  topk_mask_kernel<<<grid, kThreads, 0, st>>>(w, ens, N, nblk, keep, nullptr, 0, B);
   for (int i = 0; i < 6; ++i) note_launch();
+  return check_launch();
+}
+
+// ---------------------------------------------------- sharded top-K phases
+static fm_status shard_ws(void* ws, size_t ws_size, int B, int N, Workspace* w, int* nblk) {
+  *nblk = (int)(((int64_t)N + kChunk - 1) / kChunk);
+  if (ws_size < ws_bytes(B, *nblk)) return FM_ERR_INVALID_ARG;
+  *w = carve(ws, B, *nblk);
+  return FM_OK;
+}
+
+fm_status launch_topk_shard_begin(const int32_t* n_valid, int B, int N, int k, int32_t* hist, void* ws,
+                                  size_t ws_size, cudaStream_t st) {
+  Workspace w;
+  int nblk;
+  if (fm_status e = shard_ws(ws, ws_size, B, N, &w, &nblk)) return e;
+  topk_shard_init_kernel<<<B, 256, 0, st>>>(w, n_valid, N, k, reinterpret_cast<uint32_t*>(hist));
+  note_launch();
+  return check_launch();
+}
+
+fm_status launch_topk_shard_hist(const float* ens, int B, int N, int pass, int32_t* hist, void* ws,
+                                 size_t ws_size, cudaStream_t st) {
+  Workspace w;
+  int nblk;
+  if (fm_status e = shard_ws(ws, ws_size, B, N, &w, &nblk)) return e;
+  uint32_t* xh = reinterpret_cast<uint32_t*>(hist);
+  dim3 grid(nblk, B);
+  if (pass == 0) topk_hist_kernel<0, false><<<grid, kThreads, 0, st>>>(w, ens, N, xh);
+  else if (pass == 1) topk_hist_kernel<1, false><<<grid, kThreads, 0, st>>>(w, ens, N, xh);
+  else topk_hist_kernel<2, false><<<grid, kThreads, 0, st>>>(w, ens, N, xh);
+  note_launch();
+  return check_launch();
+}
+
+fm_status launch_topk_shard_pick(int B, int N, int pass, int32_t* hist, void* ws, size_t ws_size,
+                                 cudaStream_t st) {
+  Workspace w;
+  int nblk;
+  if (fm_status e = shard_ws(ws, ws_size, B, N, &w, &nblk)) return e;
+  uint32_t* xh = reinterpret_cast<uint32_t*>(hist);
+  if (pass == 0) topk_shard_pick_kernel<0><<<B, kThreads, 0, st>>>(w, xh);
+  else if (pass == 1) topk_shard_pick_kernel<1><<<B, kThreads, 0, st>>>(w, xh);
+  else topk_shard_pick_kernel<2><<<B, kThreads, 0, st>>>(w, xh);
+  note_launch();
+  return check_launch();
+}
+
+fm_status launch_topk_shard_ties(const float* ens, int B, int N, int32_t* eq_local, void* ws,
+                                 size_t ws_size, cudaStream_t st) {
+  Workspace w;
+  int nblk;
+  if (fm_status e = shard_ws(ws, ws_size, B, N, &w, &nblk)) return e;
+  if (cudaMemsetAsync(eq_local, 0, sizeof(int32_t) * (size_t)B, st) != cudaSuccess) return check_launch();
+  dim3 grid(nblk, B);
+  topk_eqcount_kernel<<<grid, kThreads, 0, st>>>(w, ens, N, nblk, eq_local);
+  note_launch();
+  return check_launch();
+}
+
+fm_status launch_topk_shard_mask(const float* ens, int B, int N, const int32_t* eq_all, int shard,
+                                 uint8_t* keep, void* ws, size_t ws_size, cudaStream_t st) {
+  Workspace w;
+  int nblk;
+  if (fm_status e = shard_ws(ws, ws_size, B, N, &w, &nblk)) return e;
+  dim3 grid(nblk, B);
+  topk_mask_kernel<<<grid, kThreads, 0, st>>>(w, ens, N, nblk, keep, eq_all, shard, B);
+  note_launch();
   return check_launch();
 }
 

@@ -21,6 +21,7 @@ FM_OK, FM_ERR_INVALID_ARG, FM_ERR_ALIGNMENT, FM_ERR_UNSUPPORTED = 0, 1, 2, 3
 FM_ERR_CUDA, FM_ERR_OOM, FM_ERR_DEVICE = 4, 5, 6
 FM_ENSEMBLE_MAX, FM_ENSEMBLE_MEAN = 0, 1
 MODES = {"max": FM_ENSEMBLE_MAX, "mean": FM_ENSEMBLE_MEAN}
+FM_TOPK_SHARD_BINS = 2048
 
 
 class fm_config(ctypes.Structure):
@@ -66,6 +67,11 @@ def _load():
         "fm_select_topk": (I, [P, P, I, I, I, P, P, S, P]),
         "fm_select_threshold": (I, [P, P, I, I, F, P, P]),
         "fm_select_topk_static": (I, [P, P, I, I, I, P, P]),
+        "fm_topk_shard_begin": (I, [P, I, I, I, P, P, S, P]),
+        "fm_topk_shard_hist": (I, [P, I, I, I, P, P, S, P]),
+        "fm_topk_shard_pick": (I, [I, I, I, P, P, S, P]),
+        "fm_topk_shard_ties": (I, [P, I, I, P, P, S, P]),
+        "fm_topk_shard_mask": (I, [P, I, I, P, I, P, P, S, P]),
         "fm_sync_status": (I, [P, P]),
         "fm_strerror": (ctypes.c_char_p, [I]),
         "fm_last_cuda_error": (I, []),
@@ -190,6 +196,96 @@ def fm_select_threshold(ens: torch.Tensor, thr: float, n_valid: Optional[torch.T
     _check(_lib.fm_select_threshold(_ptr(ens), _ptr(n_valid), B, N, float(thr), _ptr(keep),
                                     _stream(stream)), "fm_select_threshold")
     return keep
+
+
+class TopKShard:
+    """One shard's side of the sharded top-K (fm_topk_shard_*): this shard's
+    slice `ens_local` [B, N] of rows whose chunks are split over the shards in
+    shard order, with its buffers (workspace, the histogram the shards sum, the
+    tie count they gather, the keep mask).  The phases are called in the order
+    fm_select_topk_sharded uses; the exchanges between them are the caller's."""
+
+    def __init__(self, ens_local: torch.Tensor, k: int, n_valid_local: Optional[torch.Tensor] = None,
+                 stream=None):
+        _need(ens_local, torch.float32, "ens_local")
+        if n_valid_local is not None:
+            _need(n_valid_local, torch.int32, "n_valid_local")
+        self.ens, self.k, self.n_valid, self.stream = ens_local, int(k), n_valid_local, stream
+        self.B, self.N = ens_local.shape
+        dev = ens_local.device
+        self.ws = torch.empty(fm_topk_workspace_bytes(self.B, self.N), device=dev, dtype=torch.uint8)
+        self.hist = torch.empty(self.B, FM_TOPK_SHARD_BINS, device=dev, dtype=torch.int32)
+        self.eq_local = torch.empty(self.B, device=dev, dtype=torch.int32)
+        self.keep = torch.empty(self.B, self.N, device=dev, dtype=torch.bool)
+
+    def _tail(self):
+        return _ptr(self.ws), self.ws.numel(), _stream(self.stream)
+
+    def begin(self):
+        _check(_lib.fm_topk_shard_begin(_ptr(self.n_valid), self.B, self.N, self.k, _ptr(self.hist),
+                                        *self._tail()), "fm_topk_shard_begin")
+
+    def hist_pass(self, p: int) -> torch.Tensor:
+        """This slice's histogram of pass p, to be summed over the shards in place."""
+        _check(_lib.fm_topk_shard_hist(_ptr(self.ens), self.B, self.N, p, _ptr(self.hist), *self._tail()),
+               "fm_topk_shard_hist")
+        return self.hist
+
+    def pick(self, p: int):
+        _check(_lib.fm_topk_shard_pick(self.B, self.N, p, _ptr(self.hist), *self._tail()),
+               "fm_topk_shard_pick")
+
+    def ties(self) -> torch.Tensor:
+        """This slice's count of keys equal to the K-th, per row, to be gathered."""
+        _check(_lib.fm_topk_shard_ties(_ptr(self.ens), self.B, self.N, _ptr(self.eq_local), *self._tail()),
+               "fm_topk_shard_ties")
+        return self.eq_local
+
+    def mask(self, eq_all: torch.Tensor, shard: int) -> torch.Tensor:
+        _need(eq_all, torch.int32, "eq_all")
+        _check(_lib.fm_topk_shard_mask(_ptr(self.ens), self.B, self.N, _ptr(eq_all), int(shard),
+                                       _ptr(self.keep), *self._tail()), "fm_topk_shard_mask")
+        return self.keep
+
+
+class TorchDistExchange:
+    """The two exchanges of the sharded top-K over a torch.distributed group
+    (NCCL between GPUs): a sum of the histograms and a gather of the tie counts.
+    The shard index is the rank in the group."""
+
+    def __init__(self, group=None):
+        import torch.distributed as dist
+        self.dist, self.group = dist, group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+
+    def all_reduce_sum_(self, t: torch.Tensor):
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.SUM, group=self.group)
+
+    def all_gather(self, t: torch.Tensor) -> torch.Tensor:
+        t = t.contiguous()
+        out = torch.empty(self.world * t.numel(), device=t.device, dtype=t.dtype)
+        self.dist.all_gather_into_tensor(out, t.reshape(-1), group=self.group)
+        return out.view((self.world,) + tuple(t.shape))
+
+
+def fm_select_topk_sharded(ens_local: torch.Tensor, k: int, n_valid_local: Optional[torch.Tensor] = None,
+                           exchange=None, shard=None) -> torch.Tensor:
+    """Top-K keep mask of rows split over the ranks of a group: rank g holds the
+    g-th consecutive slice of every row (`ens_local` [B, N_g]).  Returns this
+    rank's slice of the mask that fm_select_topk gives on the whole rows.  Per
+    pass one all-reduce of B*2048 int32, then one all-gather of B int32;
+    scores never leave their GPU.  `exchange` defaults to the default
+    torch.distributed group; `shard` (an object with TopKShard's phases)
+    defaults to this library's kernels."""
+    ex = exchange if exchange is not None else TorchDistExchange()
+    sh = shard if shard is not None else TopKShard(ens_local, k, n_valid_local)
+    sh.begin()
+    for p in range(3):
+        ex.all_reduce_sum_(sh.hist_pass(p))
+        sh.pick(p)
+    eq_all = ex.all_gather(sh.ties())
+    return sh.mask(eq_all, ex.rank)
 
 
 class Retriever:

@@ -94,6 +94,16 @@ def test_host_side_argument_rejection(lib):
     assert lib.fm_select_threshold(None, None, 1, 10, 0.5, fake, None) == INVALID
     assert lib.fm_ensemble(fake, 5, 1, 10, 0, fake, None) == INVALID  # more layers than supported
     assert lib.fm_ensemble(fake, 3, 1, 10, 7, fake, None) == INVALID  # unknown mode
+    S = ctypes.c_size_t
+    lib.fm_topk_shard_begin.argtypes = [P, I, I, I, P, P, S, P]
+    lib.fm_topk_shard_hist.argtypes = [P, I, I, I, P, P, S, P]
+    lib.fm_topk_shard_pick.argtypes = [I, I, I, P, P, S, P]
+    lib.fm_topk_shard_mask.argtypes = [P, I, I, P, I, P, P, S, P]
+    assert lib.fm_topk_shard_begin(None, 1, 10, 0, fake, fake, 1 << 20, None) == INVALID  # k < 1
+    assert lib.fm_topk_shard_begin(None, 1, 10, 5, ctypes.c_void_p(0x1004), fake, 1 << 20, None) == ALIGN
+    assert lib.fm_topk_shard_hist(fake, 1, 10, 3, fake, fake, 1 << 20, None) == INVALID  # pass 3
+    assert lib.fm_topk_shard_pick(1, 10, 0, fake, fake, 16, None) == INVALID  # workspace too small
+    assert lib.fm_topk_shard_mask(fake, 1, 10, fake, -1, fake, fake, 1 << 20, None) == INVALID
     lib.fm_create.argtypes = [P, P, I, ctypes.POINTER(P)]
     out = P(0x1234)
     assert lib.fm_create(None, None, 0, ctypes.byref(out)) == INVALID
