@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--path", default="retrieve", choices=["retrieve", "recall"],
+                    help="retrieve: the scoring path (default); recall: keep mask -> index lists -> "
+                         "gather of the kept chunks' records into a resident buffer")
     return ap.parse_args()
 
 
@@ -296,6 +299,138 @@ def run_ours(args, rank, world, local_rank):
                 key_bytes=key_bytes)
 
 
+# ------------------------------------------------------------ recall path
+def _timed_flushed(fn, steps, flush_buf, stream):
+    """Mean CUDA-event time (ms) of fn() over `steps` calls, L2 flushed before each."""
+    total = 0.0
+    for _ in range(steps):
+        flush_buf.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        total += a.elapsed_time(b)
+    return total / steps
+
+
+def run_recall(args):
+    """Keep mask -> index lists -> the kept chunks' records gathered into a
+    resident buffer, on the top-4096 masks of 64 rows x 262144 chunks.  The
+    records are 132 bytes (the compressed_k record, the one chunk record size
+    the pages define); the source is device memory or pinned host memory."""
+    from learned_kv_chunk_b200 import fm
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B, N, K, rec = 64, 262144, 4096, 132
+    g = torch.Generator(device=dev).manual_seed(2024)
+    ens = torch.rand(B, N, device=dev, generator=g)
+    keep = fm.fm_select_topk(ens, K)
+    src_dev = torch.randint(0, 256, (B, N, rec), device=dev, dtype=torch.uint8, generator=g)
+    src_host = src_dev.cpu().pin_memory()
+    idx = torch.empty(B, K, device=dev, dtype=torch.int32)
+    count = torch.empty(B, device=dev, dtype=torch.int32)
+    ws = torch.empty(int(fm.lib().fm_compact_workspace_bytes(B, N)), device=dev, dtype=torch.uint8)
+    dst = torch.empty(B, K, rec, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(max(2 * l2, 1 << 28) // 4, device=dev, dtype=torch.float32)
+
+    def compact():
+        fm.fm_compact_mask(keep, K, idx=idx, count=count, workspace=ws)
+
+    def step_dev():
+        compact()
+        fm.fm_gather_records(src_dev, idx, count, dst)
+
+    def gather_host():
+        fm.fm_gather_records(src_host, idx, count, dst)
+
+    for _ in range(max(3, args.warmup)):
+        step_dev()
+        gather_host()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(0)
+    launches0 = fm.fm_launch_count()
+    with sampler:
+        t_step = _timed_flushed(step_dev, args.steps, flush_buf, stream)
+        t_compact = _timed_flushed(compact, args.steps, flush_buf, stream)
+        t_host = _timed_flushed(gather_host, max(3, args.steps // 10), flush_buf, stream)
+    launches = fm.fm_launch_count() - launches0
+    # the bus: one pinned host -> device copy of 256 MB with the copy engine, same run
+    hbuf = torch.empty(1 << 28, dtype=torch.uint8).pin_memory()
+    dbuf = torch.empty(1 << 28, dtype=torch.uint8, device=dev)
+    dbuf.copy_(hbuf, non_blocking=True)
+    t_h2d = _timed_flushed(lambda: dbuf.copy_(hbuf, non_blocking=True), 5, flush_buf, stream)
+    h2d_gbs = (1 << 28) / (t_h2d / 1e3) / 1e9
+
+    torch.cuda.synchronize()
+    assert int(count.min()) == K
+    sel = B * K
+    alg_dev = B * N + sel * 4 + B * 4 + 2 * sel * rec  # mask once, index list, count, records in + out
+    hbm_peak, peak_kind = peaks()
+    ach = alg_dev / (t_step / 1e3) / 1e9
+    host_gbs = sel * rec / (t_host / 1e3) / 1e9
+    out = {"metric": "resident-set records recalled/sec (mask -> index list -> gather)",
+           "value": sel / (t_step / 1e3), "unit": "records/s", "n_gpus": 1, "steps": args.steps,
+           "warmup": max(3, args.warmup), "ms_per_step": t_step, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic (seeded)",
+           "config": {"workload": "recall_B64_N262144_top4096_rec132", "rows": B, "chunks_per_row": N,
+                      "kept_per_row": K, "record_bytes": rec, "source": "device memory",
+                      "l2": "flushed between steps (256 MB write)"},
+           "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                        "frac": round(ach / hbm_peak, 4), "traffic": None, "peak_kind": peak_kind,
+                        "kernel": "compaction (2 kernels) + gather, one step",
+                        "alg_bytes_per_step": alg_dev},
+           "compact_ms": round(t_compact, 4),
+           "host_source": {"value": sel / (t_host / 1e3), "unit": "records/s", "gather_ms": round(t_host, 4),
+                           "achieved_gbs": round(host_gbs, 2),
+                           "h2d_copy_gbs": round(h2d_gbs, 2),
+                           "frac_of_h2d_copy": round(host_gbs / h2d_gbs, 4),
+                           "note": "records read from pinned host memory by the kernel over the bus; "
+                                   "denominator: a 256 MB pinned host-to-device copy in the same run"},
+           "gpu_launches": launches, "clocks": sampler.summary(),
+           "cpu_baseline": recall_oracle_sample(keep, src_dev, K)}
+    return out
+
+
+def run_recall_reference(args):
+    """--path recall --impl reference: the recall oracle on host cores, one
+    row of the workload per step."""
+    g = torch.Generator().manual_seed(2024)
+    B, N, K, rec = 64, 262144, 4096, 132
+    keep = torch.zeros(1, N, dtype=torch.bool)
+    keep[0, torch.randperm(N, generator=g)[:K]] = True
+    src = torch.randint(0, 256, (1, N, rec), generator=g, dtype=torch.uint8)
+    for _ in range(args.warmup):
+        recall_oracle_sample(keep, src, K)
+    vals = [recall_oracle_sample(keep, src, K) for _ in range(args.steps)]
+    v = statistics.median(x["value"] for x in vals)
+    return {"impl": "reference", "metric": "resident-set records recalled/sec (mask -> index list -> gather)",
+            "value": v, "unit": "records/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": K / v * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "u8", "data": "synthetic (seeded)",
+            "config": {"workload": "recall_B64_N262144_top4096_rec132", "rows": B, "chunks_per_row": N,
+                       "kept_per_row": K, "record_bytes": rec},
+            "cpu_baseline": dict(vals[0], value=v),
+            "e2e": {"value": v, "unit": "records/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def recall_oracle_sample(keep, src, K, rows=1):
+    """The recall oracle (compaction + gather, plain loops) on the first rows."""
+    import oracle.recall as OR
+    km = keep[:rows].cpu().numpy()
+    sm = src[:rows].cpu().numpy()
+    t0 = time.perf_counter()
+    idx, cnt = OR.compact_mask(km, K)
+    OR.gather_records(sm, idx, cnt, np.zeros((rows, K, sm.shape[2]), np.uint8))
+    dt = time.perf_counter() - t0
+    return {"value": rows * K / dt, "unit": "records/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} row(s) of the workload: compaction of {km.shape[1]} mask bytes and "
+                      f"gather of {K} records ({dt:.2f} s)"}
+
+
 def _oracle_threads():
     try:
         import threadpoolctl
@@ -382,6 +517,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.path == "recall":
+        if rank == 0:
+            print(json.dumps(run_recall_reference(args) if args.impl == "reference" else run_recall(args)),
+                  flush=True)
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)

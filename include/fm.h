@@ -246,6 +246,39 @@ fm_status fm_topk_shard_ties(const float* ens_local, int B, int N, int32_t* eq_l
 fm_status fm_topk_shard_mask(const float* ens_local, int B, int N, const int32_t* eq_all, int shard,
                              uint8_t* keep_local, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* ----------------------------------------------------------------- recall
+ * The model card's "How it works" (Level 1): the chunks the Memory Indexer
+ * selects form a resident set recalled from the CPU-side bulk KV cache to the
+ * GPU.  These two calls turn a keep mask into that set. */
+
+/* Bytes of device workspace fm_compact_mask needs for B rows of N chunks. */
+size_t fm_compact_workspace_bytes(int B, int N);
+
+/* Keep mask -> index list.  keep [B, N] uint8 device (nonzero = kept);
+ * idx [B, max_sel] int32 device (written): the kept chunk indices of row b in
+ * increasing order in idx[b, 0:min(count[b], max_sel)], -1 after them;
+ * count [B] int32 device (written): the number of kept chunks of row b (it
+ * may exceed max_sel; then only the first max_sel indices are listed);
+ * ws: fm_compact_workspace_bytes(B, N) bytes, 16-byte aligned, caller-owned,
+ * contents on entry irrelevant.  idx and count 4-byte aligned. */
+fm_status fm_compact_mask(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx, int32_t* count,
+                          void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Gathers the selected chunks' records into a resident buffer:
+ * for every row b and j < min(count[b], max_sel) with 0 <= idx[b, j] < n_src,
+ *   dst[b*dst_row_stride + j*rec_bytes, +rec_bytes) =
+ *   src[b*src_row_stride + idx[b, j]*rec_bytes, +rec_bytes).
+ * Other slots of dst are not written.  src: the bulk store of fixed-size
+ * records (n_src per row), in device memory or in pinned host memory
+ * (cudaHostAlloc / torch pin_memory; read over the bus by the kernel);
+ * pageable host memory is rejected with FM_ERR_INVALID_ARG.  dst: device
+ * memory.  idx, count as written by fm_compact_mask (device).  Any record
+ * size; 16-byte copies when both pointers, the strides and rec_bytes are
+ * multiples of 16, 4-byte ones when of 4, else byte copies. */
+fm_status fm_gather_records(const void* src, int64_t src_row_stride_bytes, int n_src, int64_t rec_bytes,
+                            const int32_t* idx, const int32_t* count, int B, int max_sel, void* dst,
+                            int64_t dst_row_stride_bytes, cudaStream_t stream);
+
 /* Synchronises `stream` and returns FM_ERR_DEVICE if a kernel launched on this
  * context recorded an error since the last call (the record is cleared),
  * FM_ERR_CUDA if the stream reports a CUDA error, FM_OK otherwise. */

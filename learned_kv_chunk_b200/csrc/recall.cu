@@ -1,0 +1,289 @@
+// recall.cu -- from a keep mask to a resident set on the GPU.
+//
+// The model card's "How it works": every 64 decode steps the Memory Indexer
+// selects the query-critical chunks, and that resident set is recalled from
+// the CPU-side bulk KV cache to the GPU; only recalled chunks and the
+// compressed indexer keys live on the GPU.  Two steps follow the keep mask:
+//
+//   compaction  keep [B, N] -> idx [B, max_sel] (kept chunk indices in
+//               increasing order, -1 past the end) and count [B];
+//   gather      for j < min(count[b], max_sel): copy the fixed-size record of
+//               chunk idx[b, j] from a bulk store (pinned host memory, read
+//               over the bus by the SMs, or device memory) into slot j of a
+//               resident buffer on the GPU.
+//
+// Compaction is two passes over the mask (1 byte per chunk): per-block counts,
+// then an ordered write in which each block starts at the sum of the counts
+// of the blocks before it.  No block waits on another.  The gather is a copy
+// with one warp per record and several records in flight per warp: the
+// selected records are scattered, so the copy engines (one call per
+// contiguous run) are not used.
+#include "fm_internal.cuh"
+
+namespace fm {
+namespace {
+
+constexpr int kCThreads = 512;
+constexpr int kCBytes = 32;                      // mask bytes per thread
+constexpr int kCChunk = kCThreads * kCBytes;     // mask bytes per block
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int compact_blocks(int N) { return (int)(((int64_t)N + kCChunk - 1) / kCChunk); }
+
+// The 32 mask bytes of this thread as eight words (bytes past N read as 0),
+// and how many of them are nonzero.
+__device__ __forceinline__ int load_mask(const uint8_t* __restrict__ row, int64_t n0, int N, bool vec,
+                                         uint32_t w[8]) {
+  if (vec && n0 + kCBytes <= N) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(row + n0));
+    const uint4 c = __ldg(reinterpret_cast<const uint4*>(row + n0 + 16));
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = c.x; w[5] = c.y; w[6] = c.z; w[7] = c.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int64_t n = n0 + 4 * i + k;
+        if (n < N) x |= (uint32_t)row[n] << (8 * k);
+      }
+      w[i] = x;
+    }
+  }
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) c += __popc(__vcmpne4(w[i], 0u)) >> 3;
+  return c;
+}
+
+__device__ __forceinline__ bool row_vec_ok(const uint8_t* keep, int N) {
+  return (N & 15) == 0 && (reinterpret_cast<uintptr_t>(keep) & 15u) == 0;
+}
+
+__device__ __forceinline__ int block_sum(int v, int* s_warp) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) s_warp[threadIdx.x >> 5] = v;
+  __syncthreads();
+  int t = 0;
+#pragma unroll
+  for (int i = 0; i < kCThreads / 32; ++i) t += s_warp[i];
+  return t;
+}
+
+__global__ void __launch_bounds__(kCThreads) compact_count_kernel(const uint8_t* __restrict__ keep, int N,
+                                                                  int nblk, int* __restrict__ blkcnt) {
+  __shared__ int s_warp[kCThreads / 32];
+  const int b = blockIdx.y;
+  const uint8_t* row = keep + (int64_t)b * N;
+  uint32_t w[8];
+  const int c = load_mask(row, (int64_t)blockIdx.x * kCChunk + (int64_t)threadIdx.x * kCBytes, N,
+                          row_vec_ok(keep, N), w);
+  const int t = block_sum(c, s_warp);
+  if (threadIdx.x == 0) blkcnt[(size_t)b * nblk + blockIdx.x] = t;
+}
+
+__global__ void __launch_bounds__(kCThreads) compact_write_kernel(const uint8_t* __restrict__ keep, int N,
+                                                                  int nblk, const int* __restrict__ blkcnt,
+                                                                  int max_sel, int32_t* __restrict__ idx,
+                                                                  int32_t* __restrict__ count) {
+  __shared__ int s_warp[kCThreads / 32];
+  __shared__ int s_scan[kCThreads / 32];
+  __shared__ int s_prefix;
+  const int b = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // kept entries of the blocks before this one (warp 0, strided)
+  if (warp == 0) {
+    int p = 0;
+    for (int j = lane; j < (int)blockIdx.x; j += 32) p += blkcnt[(size_t)b * nblk + j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+    if (lane == 0) s_prefix = p;
+  }
+  const uint8_t* row = keep + (int64_t)b * N;
+  const int64_t n0 = (int64_t)blockIdx.x * kCChunk + (int64_t)threadIdx.x * kCBytes;
+  uint32_t w[8];
+  const int c = load_mask(row, n0, N, row_vec_ok(keep, N), w);
+  // exclusive scan of the per-thread counts in thread (= chunk) order
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = lane < kCThreads / 32 ? s_warp[lane] : 0;
+    int s = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += u;
+    }
+    if (lane < kCThreads / 32) s_scan[lane] = s - v;  // exclusive over warps
+  }
+  __syncthreads();
+  int pos = s_prefix + s_scan[warp] + (incl - c);
+  int32_t* out = idx + (size_t)b * max_sel;
+  if (c) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if ((w[i] >> (8 * k)) & 0xffu) {
+          if (pos < max_sel) out[pos] = (int32_t)(n0 + 4 * i + k);
+          ++pos;
+        }
+      }
+    }
+  }
+  if (blockIdx.x == gridDim.x - 1) {
+    // the last block knows the row's total: the count, and -1 past it
+    const int total = s_prefix + s_scan[kCThreads / 32 - 1] + s_warp[kCThreads / 32 - 1];
+    if (threadIdx.x == 0) count[b] = total;
+    for (int j = total + threadIdx.x; j < max_sel; j += kCThreads) out[j] = -1;
+  }
+}
+
+// One warp per record, RU records in flight per warp, each lane moving UPL
+// units of VEC bytes per record per round.
+template <int VEC>
+struct Unit;
+template <>
+struct Unit<16> { using T = uint4; };
+template <>
+struct Unit<4> { using T = uint32_t; };
+template <>
+struct Unit<1> { using T = uint8_t; };
+
+template <int VEC>
+__global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__ src, int64_t src_stride,
+                                                     int n_src, int64_t rec, const int32_t* __restrict__ idx,
+                                                     const int32_t* __restrict__ count, int max_sel,
+                                                     int64_t total, uint8_t* __restrict__ dst,
+                                                     int64_t dst_stride) {
+  using U = typename Unit<VEC>::T;
+  constexpr int RU = 4, UPL = 2;
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t units = rec / VEC;
+  for (int64_t r0 = gw * RU; r0 < total; r0 += nw * RU) {
+    const U* s[RU];
+    U* d[RU];
+#pragma unroll
+    for (int q = 0; q < RU; ++q) {
+      s[q] = nullptr;
+      d[q] = nullptr;
+      const int64_t r = r0 + q;
+      if (r < total) {
+        const int b = (int)(r / max_sel), j = (int)(r - (int64_t)b * max_sel);
+        const int cnt = min(count[b], max_sel);
+        const int n = j < cnt ? idx[r] : -1;
+        if (n >= 0 && n < n_src) {
+          s[q] = reinterpret_cast<const U*>(src + b * src_stride + (int64_t)n * rec);
+          d[q] = reinterpret_cast<U*>(dst + b * dst_stride + (int64_t)j * rec);
+        }
+      }
+    }
+    for (int64_t u0 = 0; u0 < units; u0 += 32 * UPL) {
+      U v[RU][UPL];
+#pragma unroll
+      for (int q = 0; q < RU; ++q)
+#pragma unroll
+        for (int i = 0; i < UPL; ++i) {
+          const int64_t u = u0 + i * 32 + lane;
+          if (s[q] && u < units) v[q][i] = s[q][u];
+        }
+#pragma unroll
+      for (int q = 0; q < RU; ++q)
+#pragma unroll
+        for (int i = 0; i < UPL; ++i) {
+          const int64_t u = u0 + i * 32 + lane;
+          if (d[q] && u < units) d[q][u] = v[q][i];
+        }
+    }
+  }
+}
+
+// Device address of `p` for kernels (pinned host memory maps into the GPU's
+// address space); null for pageable host memory.
+const void* device_address(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return p;
+  if (a.type == cudaMemoryTypeHost) return a.devicePointer;
+  return nullptr;
+}
+
+}  // namespace
+}  // namespace fm
+
+using namespace fm;
+
+extern "C" size_t fm_compact_workspace_bytes(int B, int N) {
+  if (B < 1 || N < 1) return 0;
+  return align256(sizeof(int) * (size_t)B * compact_blocks(N));
+}
+
+extern "C" fm_status fm_compact_mask(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx,
+                                     int32_t* count, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!keep || !idx || !count || !ws || B < 1 || N < 1 || max_sel < 1 || B > 65535)
+    return FM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(count) & 3u) ||
+      (reinterpret_cast<uintptr_t>(ws) & 15u))
+    return FM_ERR_ALIGNMENT;
+  if (ws_bytes < fm_compact_workspace_bytes(B, N)) return FM_ERR_INVALID_ARG;
+  const int nblk = compact_blocks(N);
+  int* blkcnt = static_cast<int*>(ws);
+  dim3 grid(nblk, B);
+  compact_count_kernel<<<grid, kCThreads, 0, stream>>>(keep, N, nblk, blkcnt);
+  compact_write_kernel<<<grid, kCThreads, 0, stream>>>(keep, N, nblk, blkcnt, max_sel, idx, count);
+  note_launch();
+  note_launch();
+  return check_launch();
+}
+
+extern "C" fm_status fm_gather_records(const void* src, int64_t src_row_stride_bytes, int n_src,
+                                       int64_t rec_bytes, const int32_t* idx, const int32_t* count, int B,
+                                       int max_sel, void* dst, int64_t dst_row_stride_bytes,
+                                       cudaStream_t stream) {
+  if (!src || !idx || !count || !dst || B < 1 || max_sel < 1 || n_src < 1 || rec_bytes < 1)
+    return FM_ERR_INVALID_ARG;
+  if (src_row_stride_bytes < (int64_t)n_src * rec_bytes ||
+      dst_row_stride_bytes < (int64_t)max_sel * rec_bytes)
+    return FM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(count) & 3u))
+    return FM_ERR_ALIGNMENT;
+  const uint8_t* s = static_cast<const uint8_t*>(device_address(src));
+  if (!s || !device_address(dst)) return FM_ERR_INVALID_ARG;  // pageable host memory
+  uint8_t* d = static_cast<uint8_t*>(dst);
+  auto all_aligned = [&](uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(s) % a) == 0 && (reinterpret_cast<uintptr_t>(d) % a) == 0 &&
+           rec_bytes % (int64_t)a == 0 && src_row_stride_bytes % (int64_t)a == 0 &&
+           dst_row_stride_bytes % (int64_t)a == 0;
+  };
+  const int64_t total = (int64_t)B * max_sel;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = (total + 4 * 8 - 1) / (4 * 8);  // 8 warps of 256 threads, 4 records each
+  const int grid = (int)(want < (int64_t)sms * 8 ? (want > 0 ? want : 1) : (int64_t)sms * 8);
+  if (all_aligned(16))
+    gather_kernel<16><<<grid, 256, 0, stream>>>(s, src_row_stride_bytes, n_src, rec_bytes, idx, count,
+                                                max_sel, total, d, dst_row_stride_bytes);
+  else if (all_aligned(4))
+    gather_kernel<4><<<grid, 256, 0, stream>>>(s, src_row_stride_bytes, n_src, rec_bytes, idx, count,
+                                               max_sel, total, d, dst_row_stride_bytes);
+  else
+    gather_kernel<1><<<grid, 256, 0, stream>>>(s, src_row_stride_bytes, n_src, rec_bytes, idx, count,
+                                               max_sel, total, d, dst_row_stride_bytes);
+  note_launch();
+  return check_launch();
+}

@@ -67,6 +67,9 @@ def _load():
         "fm_select_topk": (I, [P, P, I, I, I, P, P, S, P]),
         "fm_select_threshold": (I, [P, P, I, I, F, P, P]),
         "fm_select_topk_static": (I, [P, P, I, I, I, P, P]),
+        "fm_compact_workspace_bytes": (S, [I, I]),
+        "fm_compact_mask": (I, [P, I, I, I, P, P, P, S, P]),
+        "fm_gather_records": (I, [P, I64, I, I64, P, P, I, I, P, I64, P]),
         "fm_topk_shard_begin": (I, [P, I, I, I, P, P, S, P]),
         "fm_topk_shard_hist": (I, [P, I, I, I, P, P, S, P]),
         "fm_topk_shard_pick": (I, [I, I, I, P, P, S, P]),
@@ -196,6 +199,50 @@ def fm_select_threshold(ens: torch.Tensor, thr: float, n_valid: Optional[torch.T
     _check(_lib.fm_select_threshold(_ptr(ens), _ptr(n_valid), B, N, float(thr), _ptr(keep),
                                     _stream(stream)), "fm_select_threshold")
     return keep
+
+
+def fm_compact_mask(keep: torch.Tensor, max_sel: int, idx: Optional[torch.Tensor] = None,
+                    count: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    stream=None):
+    """Keep mask [B, N] (bool or uint8, device) -> (idx [B, max_sel] int32, kept
+    chunk indices in increasing order then -1; count [B] int32)."""
+    if keep.dtype not in (torch.bool, torch.uint8):
+        raise ValueError("keep must be bool or uint8")
+    if not keep.is_cuda or not keep.is_contiguous():
+        raise ValueError("keep must be a contiguous CUDA tensor")
+    B, N = keep.shape
+    dev = keep.device
+    idx = idx if idx is not None else torch.empty(B, max_sel, device=dev, dtype=torch.int32)
+    count = count if count is not None else torch.empty(B, device=dev, dtype=torch.int32)
+    _need(idx, torch.int32, "idx")
+    _need(count, torch.int32, "count")
+    nbytes = int(_lib.fm_compact_workspace_bytes(B, N))
+    ws = workspace if workspace is not None else torch.empty(nbytes, device=dev, dtype=torch.uint8)
+    _check(_lib.fm_compact_mask(_ptr(keep), B, N, int(max_sel), _ptr(idx), _ptr(count), _ptr(ws), ws.numel(),
+                                _stream(stream)), "fm_compact_mask")
+    return idx, count
+
+
+def fm_gather_records(src: torch.Tensor, idx: torch.Tensor, count: torch.Tensor,
+                      dst: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Resident buffer [B, max_sel, rec] (uint8, device): slot j of row b holds
+    record idx[b, j] of src[b] for j < min(count[b], max_sel); other slots are
+    left as they were (zeros in a new buffer).  src [B, n_src, rec] uint8 on
+    the device or in pinned host memory."""
+    if src.dtype != torch.uint8 or src.dim() != 3 or not src.is_contiguous():
+        raise ValueError("src must be a contiguous uint8 tensor [B, n_src, rec]")
+    if not src.is_cuda and not src.is_pinned():
+        raise ValueError("src must be on the device or in pinned host memory")
+    _need(idx, torch.int32, "idx")
+    _need(count, torch.int32, "count")
+    B, n_src, rec = src.shape
+    max_sel = idx.shape[1]
+    if dst is None:
+        dst = torch.zeros(B, max_sel, rec, device=idx.device, dtype=torch.uint8)
+    _need(dst, torch.uint8, "dst")
+    _check(_lib.fm_gather_records(_ptr(src), n_src * rec, n_src, rec, _ptr(idx), _ptr(count), B, max_sel,
+                                  _ptr(dst), dst.stride(0), _stream(stream)), "fm_gather_records")
+    return dst
 
 
 class TopKShard:

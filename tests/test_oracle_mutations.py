@@ -148,3 +148,62 @@ def test_pins_catch_planted_mistake(monkeypatch, name, fn):
         except Exception:  # noqa: BLE001 - any failure counts as detection
             caught.append(pin.__name__)
     assert caught, f"no pin caught the mutation {name}:{fn.__name__}"
+
+
+# ------------------------------------------------------------------ recall
+import oracle.recall as OR  # noqa: E402
+
+
+def _compact_count_capped(keep, max_sel):
+    idx, count = OR.__dict__["_orig_compact_mask"](keep, max_sel)
+    return idx, np.minimum(count, max_sel).astype(np.int32)
+
+
+def _compact_fill_zero(keep, max_sel):
+    idx, count = OR.__dict__["_orig_compact_mask"](keep, max_sel)
+    return np.where(idx < 0, 0, idx).astype(np.int32), count
+
+
+def _compact_descending(keep, max_sel):
+    keep = np.asarray(keep)
+    return OR.__dict__["_orig_compact_mask"](keep[:, ::-1], max_sel)
+
+
+def _compact_one_based(keep, max_sel):
+    idx, count = OR.__dict__["_orig_compact_mask"](keep, max_sel)
+    return np.where(idx >= 0, idx + 1, -1).astype(np.int32), count
+
+
+def _gather_ignores_idx(src, idx, count, dst):
+    out = np.array(dst, copy=True)
+    for b in range(src.shape[0]):
+        m = min(int(count[b]), idx.shape[1], src.shape[1])
+        out[b, :m] = src[b, :m]
+    return out
+
+
+def _gather_row_zero(src, idx, count, dst):
+    return OR.__dict__["_orig_gather_records"](np.broadcast_to(src[:1], src.shape), idx, count, dst)
+
+
+RECALL_MUTATIONS = [
+    ("compact_mask", _compact_count_capped),
+    ("compact_mask", _compact_fill_zero),
+    ("compact_mask", _compact_descending),
+    ("compact_mask", _compact_one_based),
+    ("gather_records", _gather_ignores_idx),
+    ("gather_records", _gather_row_zero),
+]
+
+
+@pytest.mark.parametrize("name,fn", RECALL_MUTATIONS, ids=[f"{n}:{f.__name__}" for n, f in RECALL_MUTATIONS])
+def test_recall_pins_catch_planted_mistake(monkeypatch, name, fn):
+    monkeypatch.setitem(OR.__dict__, "_orig_" + name, getattr(OR, name))
+    monkeypatch.setattr(OR, name, fn)
+    caught = []
+    for pin in PINS:
+        try:
+            pin()
+        except Exception:  # noqa: BLE001 - any failure counts as detection
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the mutation {name}:{fn.__name__}"

@@ -404,3 +404,52 @@ def test_threshold_is_strict_and_respects_length():
     ens = np.array([[0.5, 0.50000006, 0.4, 0.9, 0.9]], np.float32)
     keep = O.select_threshold(ens, np.array([4]), 0.5)
     np.testing.assert_array_equal(keep[0], [False, True, False, True, False])
+
+
+# ------------------------------------------------------------------ recall
+import oracle.recall as OR  # noqa: E402
+
+
+def test_compact_hand_example():
+    keep = np.array([[0, 1, 1, 0, 1, 0], [0, 0, 0, 0, 0, 0], [1, 1, 1, 1, 1, 1]], np.uint8)
+    idx, count = OR.compact_mask(keep, 4)
+    assert idx.tolist() == [[1, 2, 4, -1], [-1, -1, -1, -1], [0, 1, 2, 3]]
+    assert count.tolist() == [3, 0, 6]  # row 2 keeps more than it can list
+
+
+def test_compact_matches_flatnonzero_and_invariants():
+    rng = np.random.default_rng(3)
+    keep = rng.random((5, 300)) < np.array([0.0, 0.02, 0.5, 0.97, 1.0])[:, None]
+    idx, count = OR.compact_mask(keep, 64)
+    for b in range(5):
+        nz = np.flatnonzero(keep[b])  # library routine
+        assert count[b] == keep[b].sum() == len(nz)
+        m = min(len(nz), 64)
+        assert np.array_equal(idx[b, :m], nz[:m])
+        assert (idx[b, m:] == -1).all()
+        assert (np.diff(idx[b, :m]) > 0).all() and keep[b, idx[b, :m]].all()
+
+
+def test_gather_hand_example_and_untouched_slots():
+    src = np.arange(2 * 5 * 3, dtype=np.uint8).reshape(2, 5, 3)
+    idx = np.array([[4, 0, -1], [2, 9, 1]], np.int32)  # 9 is out of range: skipped
+    count = np.array([2, 3], np.int32)
+    dst = np.full((2, 3, 3), 255, np.uint8)
+    out = OR.gather_records(src, idx, count, dst)
+    assert out[0, 0].tolist() == [12, 13, 14] and out[0, 1].tolist() == [0, 1, 2]
+    assert (out[0, 2] == 255).all()  # past count
+    assert out[1, 0].tolist() == [21, 22, 23] and (out[1, 1] == 255).all()
+    assert out[1, 2].tolist() == [18, 19, 20]
+    assert (dst == 255).all()  # the input is not modified
+
+
+def test_gather_matches_fancy_indexing():
+    rng = np.random.default_rng(4)
+    src = rng.integers(0, 256, (3, 50, 132), dtype=np.uint8)
+    keep = rng.random((3, 50)) < 0.3
+    idx, count = OR.compact_mask(keep, 20)
+    out = OR.gather_records(src, idx, count, np.zeros((3, 20, 132), np.uint8))
+    for b in range(3):
+        m = min(int(count[b]), 20)
+        assert np.array_equal(out[b, :m], src[b][np.flatnonzero(keep[b])[:m]])  # library routine
+        assert not out[b, m:].any()
