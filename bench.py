@@ -47,9 +47,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--path", default="retrieve", choices=["retrieve", "recall"],
+    ap.add_argument("--path", default="retrieve", choices=["retrieve", "recall", "level2"],
                     help="retrieve: the scoring path (default); recall: keep mask -> index lists -> "
-                         "gather of the kept chunks' records into a resident buffer")
+                         "gather of the kept chunks' records into a resident buffer; level2: the "
+                         "per-step top-512 over a resident set of 4096 chunks per row, one CUDA graph")
     return ap.parse_args()
 
 
@@ -417,6 +418,63 @@ def run_recall_reference(args):
             "e2e": {"value": v, "unit": "records/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------ level-2 path
+def run_level2(args):
+    """The per-step selection over the resident set (one CUDA graph launch per
+    decode step): 64 rows, 4096 resident chunks per row (the recalled top-4096
+    of 262144), top-512.  Resident records come from the seeded key generator;
+    each step reads the 154 MB of query weights and the 104 MB of resident
+    keys, and L2 is flushed before each step (the rest of a decode step would
+    evict it)."""
+    from learned_kv_chunk_b200 import fm
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B, R, k, N1 = 64, 4096, 512, 262144
+    weights = G.make_weights(5000, G.N_LAYERS)
+    r = fm.Retriever(weights, device=0, max_batch=B, q_pieces=args.q_pieces)
+    g = torch.Generator().manual_seed(5001)
+    ids = torch.stack([torch.randperm(N1, generator=g)[:R].sort().values for _ in range(B)]).to(torch.int32)
+    res_keys = G.make_keys(5002, [R] * B, R, G.N_LAYERS, None, device=dev)
+    res_ids = ids.to(dev)
+    count = torch.full((B,), R, dtype=torch.int32, device=dev)
+    step = fm.Level2Step(r, res_keys, res_ids, count, k=k, mode="max")
+    step.hidden.copy_(G.make_hidden(5003, B).to(dev))
+    step.positions.copy_(torch.full((B,), 4 * N1, dtype=torch.int64).to(dev))
+    stream = torch.cuda.current_stream()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(max(2 * l2, 1 << 28) // 4, device=dev, dtype=torch.float32)
+    for _ in range(max(3, args.warmup)):
+        step.launch()
+    torch.cuda.synchronize()
+    r.fm_sync_status()
+    sampler = ClockSampler(0)
+    with sampler:
+        t_step = _timed_flushed(step.launch, args.steps, flush_buf, stream)
+    r.fm_sync_status()
+    assert int(step.out_count.min()) == k
+    cfg = r.cfg
+    L, HID, RK, H, D = G.N_LAYERS, cfg.hidden, cfg.q_lora_rank, cfg.n_heads, cfg.head_dim
+    w_bytes = 4 * L * ((RK + H) * HID + H * D * RK)
+    alg = w_bytes + B * HID * 4 + B * R * (L * G.RECORD_BYTES + 4) + B * R * 4 * 3 + B * R + B * k * 8
+    hbm_peak, peak_kind = peaks()
+    ach = alg / (t_step / 1e3) / 1e9
+    step.close()
+    r.close()
+    return {"metric": "level-2 resident chunks scored/sec (per-step top-512, CUDA graph)",
+            "value": B * R / (t_step / 1e3), "unit": "chunks/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3", "data": "synthetic (seeded generator, random-init weights)",
+            "config": {"workload": "level2_B64_R4096_top512", "rows": B, "resident_per_row": R, "top_k": k,
+                       "layers": L, "ensemble": "max", "query_prep_in_step": True,
+                       "l2": "flushed between steps (256 MB write)"},
+            "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(ach / hbm_peak, 4), "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "the whole step (one graph: query prep, scoring, top-k, compaction, id map)",
+                         "alg_bytes_per_step": int(alg)},
+            "gpu_launches_per_step": "one graph launch", "clocks": sampler.summary()}
+
+
 def recall_oracle_sample(keep, src, K, rows=1):
     """The recall oracle (compaction + gather, plain loops) on the first rows."""
     import oracle.recall as OR
@@ -517,6 +575,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.path == "level2":
+        if rank == 0:
+            print(json.dumps(run_level2(args)), flush=True)
+        return
     if args.path == "recall":
         if rank == 0:
             print(json.dumps(run_recall_reference(args) if args.impl == "reference" else run_recall(args)),

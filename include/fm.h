@@ -22,7 +22,8 @@
  *     written in that case.  Errors raised inside a kernel (a bounded wait
  *     that ran out) are recorded in the context and reported by
  *     fm_sync_status.
- *   - No call allocates device memory except fm_create (and fm_destroy frees).
+ *   - No call allocates device memory except fm_create and fm_level2_create
+ *     (and their destroy calls free).
  *     Calls on one context must not run concurrently on different streams:
  *     they share the context's packed-query workspace.
  *   - Shapes: L = n_layers (1..4), H = n_heads = 64, D = head_dim = 128,
@@ -278,6 +279,52 @@ fm_status fm_compact_mask(const uint8_t* keep, int B, int N, int max_sel, int32_
 fm_status fm_gather_records(const void* src, int64_t src_row_stride_bytes, int n_src, int64_t rec_bytes,
                             const int32_t* idx, const int32_t* count, int B, int max_sel, void* dst,
                             int64_t dst_row_stride_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------- Level 2
+ * The model card's "How it works", Level 2: at every decode step a top-512
+ * confined to the resident set, run inside a CUDA graph.  DS-V4's own Level-2
+ * indexer is not described by the pages; this step runs this library's stages
+ * on the resident chunks: query prep for the step's hidden states, fused
+ * scoring of the R resident records of every layer with the ensemble, top-k
+ * of the ensembled scores (ties to the lower resident slot, which is the
+ * lower chunk id), and the mapping of the kept slots to chunk ids. */
+typedef struct fm_level2 fm_level2;
+
+typedef struct fm_level2_desc {
+  const float* hidden;             /* [B, HID] fp32 device, 16-byte aligned: read at every launch */
+  const int64_t* positions;        /* [B] int64 device: read at every launch */
+  const uint8_t* resident_keys[4]; /* per layer (n_layers used): [B, R, 132] device, 16-byte aligned;
+                                      the resident chunks' compressed_k records (fm_gather_records) */
+  const int32_t* resident_ids;     /* [B, R] int32 device: chunk id of each resident slot, ascending
+                                      (fm_compact_mask's idx) */
+  const int32_t* resident_count;   /* [B] int32 device: resident chunks per row (clamped to R) */
+  int B;                           /* rows, 1..max_batch of the context */
+  int R;                           /* resident slots per row, a multiple of 4 */
+  int k;                           /* chunks selected per row, 1..R (512 in the model card) */
+  int mode;                        /* FM_ENSEMBLE_MAX or FM_ENSEMBLE_MEAN */
+  int32_t* out_ids;                /* [B, k] int32 device, written at every launch: the selected chunk
+                                      ids, ascending, -1 past the row's count */
+  int32_t* out_count;              /* [B] int32 device or NULL: min(k, resident_count[b]) */
+} fm_level2_desc;
+
+/* Builds the step for the buffers of `d` (the pointers are kept; the contents
+ * are read at every launch): allocates its intermediates (q, fused_w, scores,
+ * mask, index lists and workspaces; one of the two calls besides fm_create
+ * that allocate device memory), runs the step once on `stream` (synchronous),
+ * then captures the same launches into a CUDA graph.  The step uses the
+ * context's packed-query workspace: no other call on `ctx` may run while a
+ * launch is in flight.  *out is NULL on failure. */
+fm_status fm_level2_create(fm_ctx* ctx, const fm_level2_desc* d, cudaStream_t stream, fm_level2** out);
+
+/* Runs one step (one graph launch) on `stream`. */
+fm_status fm_level2_launch(fm_level2* step, cudaStream_t stream);
+
+/* Copies the ensembled scores [B, R] of the last step (fp32) into dst (device),
+ * on `stream`. */
+fm_status fm_level2_copy_scores(const fm_level2* step, float* dst, cudaStream_t stream);
+
+/* Waits for the device and frees the step. */
+fm_status fm_level2_destroy(fm_level2* step);
 
 /* Synchronises `stream` and returns FM_ERR_DEVICE if a kernel launched on this
  * context recorded an error since the last call (the record is cleared),

@@ -83,6 +83,11 @@ fm_status check_launch() {
   return e == cudaSuccess ? FM_OK : cuda_fail(e);
 }
 
+fm_status record_cuda_error(cudaError_t e) {
+  cudaGetLastError();  // clear the sticky copy of a non-fatal error
+  return cuda_fail(e);
+}
+
 }  // namespace fm
 
 using namespace fm;

@@ -61,6 +61,8 @@ namespace fm {
 // launch helpers (fm_api.cu)
 void note_launch();
 fm_status check_launch();
+// Records `e` for fm_last_cuda_error and returns FM_ERR_CUDA.
+fm_status record_cuda_error(cudaError_t e);
 
 // kernels' host entry points
 fm_status launch_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* positions, int B,
@@ -97,6 +99,14 @@ fm_status launch_threshold(const float* ens, const int32_t* n_valid, int B, int 
 size_t topk_workspace_bytes(int B, int N);
 fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, int k, uint8_t* keep,
                       void* ws, size_t ws_bytes, cudaStream_t stream);
+size_t compact_workspace_bytes(int B, int N);
+fm_status launch_compact(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx, int32_t* count,
+                         void* ws, cudaStream_t stream);
+// src and dst: addresses a kernel can dereference (device memory, or the
+// device address of pinned host memory).
+fm_status launch_gather(const void* src, int64_t src_row_stride_bytes, int n_src, int64_t rec_bytes,
+                        const int32_t* idx, const int32_t* count, int B, int max_sel, void* dst,
+                        int64_t dst_row_stride_bytes, cudaStream_t stream);
 fm_status launch_topk_shard_begin(const int32_t* n_valid, int B, int N, int k, int32_t* hist, void* ws,
                                   size_t ws_bytes, cudaStream_t stream);
 fm_status launch_topk_shard_hist(const float* ens, int B, int N, int pass, int32_t* hist, void* ws,

@@ -225,21 +225,12 @@ const void* device_address(const void* p) {
 }  // namespace
 }  // namespace fm
 
-using namespace fm;
+namespace fm {
 
-extern "C" size_t fm_compact_workspace_bytes(int B, int N) {
-  if (B < 1 || N < 1) return 0;
-  return align256(sizeof(int) * (size_t)B * compact_blocks(N));
-}
+size_t compact_workspace_bytes(int B, int N) { return align256(sizeof(int) * (size_t)B * compact_blocks(N)); }
 
-extern "C" fm_status fm_compact_mask(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx,
-                                     int32_t* count, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  if (!keep || !idx || !count || !ws || B < 1 || N < 1 || max_sel < 1 || B > 65535)
-    return FM_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(count) & 3u) ||
-      (reinterpret_cast<uintptr_t>(ws) & 15u))
-    return FM_ERR_ALIGNMENT;
-  if (ws_bytes < fm_compact_workspace_bytes(B, N)) return FM_ERR_INVALID_ARG;
+fm_status launch_compact(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx, int32_t* count,
+                         void* ws, cudaStream_t stream) {
   const int nblk = compact_blocks(N);
   int* blkcnt = static_cast<int*>(ws);
   dim3 grid(nblk, B);
@@ -250,19 +241,10 @@ extern "C" fm_status fm_compact_mask(const uint8_t* keep, int B, int N, int max_
   return check_launch();
 }
 
-extern "C" fm_status fm_gather_records(const void* src, int64_t src_row_stride_bytes, int n_src,
-                                       int64_t rec_bytes, const int32_t* idx, const int32_t* count, int B,
-                                       int max_sel, void* dst, int64_t dst_row_stride_bytes,
-                                       cudaStream_t stream) {
-  if (!src || !idx || !count || !dst || B < 1 || max_sel < 1 || n_src < 1 || rec_bytes < 1)
-    return FM_ERR_INVALID_ARG;
-  if (src_row_stride_bytes < (int64_t)n_src * rec_bytes ||
-      dst_row_stride_bytes < (int64_t)max_sel * rec_bytes)
-    return FM_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(count) & 3u))
-    return FM_ERR_ALIGNMENT;
-  const uint8_t* s = static_cast<const uint8_t*>(device_address(src));
-  if (!s || !device_address(dst)) return FM_ERR_INVALID_ARG;  // pageable host memory
+fm_status launch_gather(const void* src, int64_t src_row_stride_bytes, int n_src, int64_t rec_bytes,
+                        const int32_t* idx, const int32_t* count, int B, int max_sel, void* dst,
+                        int64_t dst_row_stride_bytes, cudaStream_t stream) {
+  const uint8_t* s = static_cast<const uint8_t*>(src);
   uint8_t* d = static_cast<uint8_t*>(dst);
   auto all_aligned = [&](uintptr_t a) {
     return (reinterpret_cast<uintptr_t>(s) % a) == 0 && (reinterpret_cast<uintptr_t>(d) % a) == 0 &&
@@ -286,4 +268,41 @@ extern "C" fm_status fm_gather_records(const void* src, int64_t src_row_stride_b
                                                max_sel, total, d, dst_row_stride_bytes);
   note_launch();
   return check_launch();
+}
+
+}  // namespace fm
+
+using namespace fm;
+
+extern "C" size_t fm_compact_workspace_bytes(int B, int N) {
+  if (B < 1 || N < 1) return 0;
+  return compact_workspace_bytes(B, N);
+}
+
+extern "C" fm_status fm_compact_mask(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx,
+                                     int32_t* count, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!keep || !idx || !count || !ws || B < 1 || N < 1 || max_sel < 1 || B > 65535)
+    return FM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(count) & 3u) ||
+      (reinterpret_cast<uintptr_t>(ws) & 15u))
+    return FM_ERR_ALIGNMENT;
+  if (ws_bytes < compact_workspace_bytes(B, N)) return FM_ERR_INVALID_ARG;
+  return launch_compact(keep, B, N, max_sel, idx, count, ws, stream);
+}
+
+extern "C" fm_status fm_gather_records(const void* src, int64_t src_row_stride_bytes, int n_src,
+                                       int64_t rec_bytes, const int32_t* idx, const int32_t* count, int B,
+                                       int max_sel, void* dst, int64_t dst_row_stride_bytes,
+                                       cudaStream_t stream) {
+  if (!src || !idx || !count || !dst || B < 1 || max_sel < 1 || n_src < 1 || rec_bytes < 1)
+    return FM_ERR_INVALID_ARG;
+  if (src_row_stride_bytes < (int64_t)n_src * rec_bytes ||
+      dst_row_stride_bytes < (int64_t)max_sel * rec_bytes)
+    return FM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(count) & 3u))
+    return FM_ERR_ALIGNMENT;
+  const void* s = device_address(src);
+  if (!s || !device_address(dst)) return FM_ERR_INVALID_ARG;  // pageable host memory
+  return launch_gather(s, src_row_stride_bytes, n_src, rec_bytes, idx, count, B, max_sel, dst,
+                       dst_row_stride_bytes, stream);
 }

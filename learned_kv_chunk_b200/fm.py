@@ -39,6 +39,14 @@ class fm_layer_weights(ctypes.Structure):
                 ("wq_b", ctypes.c_void_p), ("weights_proj", ctypes.c_void_p)]
 
 
+class fm_level2_desc(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_void_p), ("positions", ctypes.c_void_p),
+                ("resident_keys", ctypes.c_void_p * 4), ("resident_ids", ctypes.c_void_p),
+                ("resident_count", ctypes.c_void_p), ("B", ctypes.c_int), ("R", ctypes.c_int),
+                ("k", ctypes.c_int), ("mode", ctypes.c_int), ("out_ids", ctypes.c_void_p),
+                ("out_count", ctypes.c_void_p)]
+
+
 class FMError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -70,6 +78,10 @@ def _load():
         "fm_compact_workspace_bytes": (S, [I, I]),
         "fm_compact_mask": (I, [P, I, I, I, P, P, P, S, P]),
         "fm_gather_records": (I, [P, I64, I, I64, P, P, I, I, P, I64, P]),
+        "fm_level2_create": (I, [P, ctypes.POINTER(fm_level2_desc), P, ctypes.POINTER(P)]),
+        "fm_level2_launch": (I, [P, P]),
+        "fm_level2_copy_scores": (I, [P, P, P]),
+        "fm_level2_destroy": (I, [P]),
         "fm_topk_shard_begin": (I, [P, I, I, I, P, P, S, P]),
         "fm_topk_shard_hist": (I, [P, I, I, I, P, P, S, P]),
         "fm_topk_shard_pick": (I, [I, I, I, P, P, S, P]),
@@ -243,6 +255,67 @@ def fm_gather_records(src: torch.Tensor, idx: torch.Tensor, count: torch.Tensor,
     _check(_lib.fm_gather_records(_ptr(src), n_src * rec, n_src, rec, _ptr(idx), _ptr(count), B, max_sel,
                                   _ptr(dst), dst.stride(0), _stream(stream)), "fm_gather_records")
     return dst
+
+
+class Level2Step:
+    """The per-step selection over a resident set, as one CUDA graph
+    (fm_level2_*): query prep for the step's hidden states, scoring of the
+    resident records of every layer with the ensemble, top-k, and the kept
+    slots mapped to chunk ids.  The graph reads `hidden` and `positions` at
+    every launch: write the next step's values into them in place
+    (Level2Step.hidden.copy_(...)) and call launch().
+
+    resident_keys: per layer [B, R, 132] uint8 (fm_gather_records' output);
+    resident_ids [B, R] int32 and resident_count [B] int32 (fm_compact_mask's
+    output for the resident set)."""
+
+    def __init__(self, retriever: "Retriever", resident_keys: Sequence[torch.Tensor],
+                 resident_ids: torch.Tensor, resident_count: torch.Tensor, k: int = 512, mode: str = "max",
+                 stream=None):
+        for i, t in enumerate(resident_keys):
+            _need(t, torch.uint8, f"resident_keys[{i}]")
+        _need(resident_ids, torch.int32, "resident_ids")
+        _need(resident_count, torch.int32, "resident_count")
+        B, R = resident_ids.shape
+        dev = resident_ids.device
+        cfg = retriever.cfg
+        self.hidden = torch.zeros(B, cfg.hidden, device=dev, dtype=torch.float32)
+        self.positions = torch.zeros(B, device=dev, dtype=torch.int64)
+        self.out_ids = torch.empty(B, k, device=dev, dtype=torch.int32)
+        self.out_count = torch.empty(B, device=dev, dtype=torch.int32)
+        self._keep_alive = (retriever, list(resident_keys), resident_ids, resident_count)
+        self.B, self.R, self.k = B, R, int(k)
+        d = fm_level2_desc()
+        d.hidden, d.positions = self.hidden.data_ptr(), self.positions.data_ptr()
+        for l, t in enumerate(resident_keys):
+            d.resident_keys[l] = t.data_ptr()
+        d.resident_ids, d.resident_count = resident_ids.data_ptr(), resident_count.data_ptr()
+        d.B, d.R, d.k, d.mode = B, R, int(k), MODES[mode]
+        d.out_ids, d.out_count = self.out_ids.data_ptr(), self.out_count.data_ptr()
+        h = ctypes.c_void_p()
+        _check(_lib.fm_level2_create(retriever.handle, ctypes.byref(d), _stream(stream), ctypes.byref(h)),
+               "fm_level2_create")
+        self._h = h
+
+    def launch(self, stream=None):
+        _check(_lib.fm_level2_launch(self._h, _stream(stream)), "fm_level2_launch")
+
+    def scores(self, stream=None) -> torch.Tensor:
+        """The ensembled scores [B, R] of the last step (a copy)."""
+        out = torch.empty(self.B, self.R, device=self.out_ids.device, dtype=torch.float32)
+        _check(_lib.fm_level2_copy_scores(self._h, _ptr(out), _stream(stream)), "fm_level2_copy_scores")
+        return out
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.fm_level2_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class TopKShard:
