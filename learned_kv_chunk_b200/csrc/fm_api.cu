@@ -151,10 +151,6 @@ fm_status fm_create(const fm_config* cfg, const fm_layer_weights* w, int device,
       {(void**)&c->wprime, (size_t)Bm * L * H * sizeof(float)},
       {(void**)&c->qexp, (size_t)Bm * L * H * sizeof(int32_t)},
       {(void**)&c->d_err, sizeof(int)},
-      {(void**)&c->w_down_hi, M * HID * sizeof(float)},
-      {(void**)&c->w_down_lo, M * HID * sizeof(float)},
-      {(void**)&c->w_up_hi, (size_t)L * H * D * R * sizeof(float)},
-      {(void**)&c->w_up_lo, (size_t)L * H * D * R * sizeof(float)},
       {(void**)&c->x_hi, (size_t)Bm * HID * sizeof(float)},
       {(void**)&c->x_lo, (size_t)Bm * HID * sizeof(float)},
       {(void**)&c->r_hi, (size_t)Bm * L * R * sizeof(float)},
@@ -207,10 +203,9 @@ fm_status fm_destroy(fm_ctx* c) {
   cudaGetDevice(&prev);
   cudaSetDevice(c->device);
   cudaDeviceSynchronize();
-  void* ptrs[] = {c->w_down, c->q_norm,  c->w_up,    c->rope_freq, c->a_part,    c->r_norm,
-                  c->rope_cs, c->qpack,   c->wprime,  c->qexp,      c->d_err,     c->w_down_hi,
-                  c->w_down_lo, c->w_up_hi, c->w_up_lo, c->x_hi,    c->x_lo,      c->r_hi,
-                  c->r_lo,    c->up_part};
+  void* ptrs[] = {c->w_down, c->q_norm, c->w_up,   c->rope_freq, c->a_part, c->r_norm, c->rope_cs,
+                  c->qpack,  c->wprime, c->qexp,   c->d_err,     c->x_hi,   c->x_lo,   c->r_hi,
+                  c->r_lo,   c->up_part};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   cudaSetDevice(prev);

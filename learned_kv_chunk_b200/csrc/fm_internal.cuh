@@ -45,15 +45,13 @@ struct fm_ctx {
   float* wprime;    // [max_batch, L, 64] fused_w * 2^-e per head
   int32_t* qexp;    // [max_batch, L, 64] the exponent e of each head's scaling
   int* d_err;       // device error word
-  // tensor-core query path (three-pass TF32): each fp32 weight w is kept as
-  // hi = tf32(w) and lo = w - hi, and so are the activations
+  // tensor-core query path (three-pass TF32): the activations are stored
+  // split as hi = tf32(x), lo = x - hi; the weights are split in the GEMM
   int tc_ok;        // the weight tensor maps could be encoded
-  float* w_down_hi; float* w_down_lo;  // [L*(R+H), HID]
-  float* w_up_hi; float* w_up_lo;      // [L*H*D, R]
   float* x_hi; float* x_lo;            // [max_batch, HID] hidden, split
   float* r_hi; float* r_lo;            // [max_batch, L, R] RMSNorm output, split
   float* up_part;                      // [2, max_batch, L*H*D] K-split partial sums of wq_b . r
-  alignas(64) unsigned char wmaps[4][128];  // TMA tensor maps: w_down hi, lo; w_up hi, lo
+  alignas(64) unsigned char wmaps[2][128];  // TMA tensor maps (fp32): w_down, w_up
 };
 
 namespace fm {
@@ -69,8 +67,8 @@ fm_status launch_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* pos
                             float* q, float* fused_w, cudaStream_t stream);
 fm_status launch_qpack(fm_ctx* ctx, const float* q, const float* fused_w, int B,
                        cudaStream_t stream);
-// Splits the weights for the tensor-core query path and encodes their tensor
-// maps (fm_create); leaves tc_ok = 0 when the maps cannot be encoded.
+// Encodes the weights' tensor maps for the tensor-core query path (fm_create);
+// leaves tc_ok = 0 when they cannot be encoded.
 fm_status prepare_tc_weights(fm_ctx* ctx);
 
 struct ScoreArgs {

@@ -175,17 +175,27 @@ __global__ void split_tf32_kernel(const float* __restrict__ x, float* __restrict
 }
 
 // ------------------------------------------------ tensor-core skinny GEMM
-// part[s][n][m] = sum over K split s of W[m][k] X[n][k], with both operands
-// given as hi + lo pairs and the product taken as hi*hi + hi*lo + lo*hi
-// (three TF32 MMAs, fp32 accumulation in TMEM): fp32-level accuracy at
-// tensor-core speed.  One CTA per (128 rows of W, K split, BN columns of X);
-// warp 0 lane 0 feeds a ring of shared-memory stages with tiled TMA loads of
-// the four 128B-swizzled tiles, warp 1 lane 0 issues the MMAs, and all four
-// warps read the accumulator (one TMEM lane quarter each) and store it.
-constexpr int kTcThreads = 128;
+// part[s][n][m] = sum over K split s of W[m][k] X[n][k] at fp32-level accuracy
+// on the tensor cores: each operand is split as hi = tf32(v), lo = v - hi and
+// the product is taken as hi*hi + hi*lo + lo*hi (three TF32 MMAs, fp32
+// accumulation in TMEM).  X (a few hundred KB) arrives already split; W, the
+// bulk of the bytes, streams in as fp32 once and is split inside the CTA:
+//
+//   warp 0 lane 0   TMA producer: per stage the fp32 W tile (128 rows x 32)
+//                   and the X hi / lo tiles (BN rows x 32), 128B-swizzled
+//   warps 4..7      split: thread t reads row t of the W tile, writes its hi
+//                   and lo parts into the stage's TMEM columns (the MMA's A
+//                   operand), then reads out the accumulator at the end
+//   warp 1 lane 0   MMA issuer: A from TMEM, B (X hi / lo) from shared memory
+//
+// A stage's TMEM columns are reused only after its shared-memory stage was
+// refilled, which waits for the MMAs of the previous use to retire.  One CTA
+// per (128 rows of W, K split, BN columns of X).
+constexpr int kTcThreads = 256;
 constexpr int kTcBM = 128;                              // rows of W per CTA (MMA M)
 constexpr int kTcBK = 32;                               // K per stage: 32 fp32 = one 128-byte row
 constexpr uint32_t kTcWTile = kTcBM * kTcBK * 4;        // 16 KB
+constexpr int kTcSplitWarp0 = 4;                        // warps 4..7: TMEM lane quarters 0..3
 
 struct TcGemmArgs {
   int M, N, K;          // W [M, K]; X [N, K] (one layer of it); part [split][N][M]
@@ -203,21 +213,36 @@ __host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, TF32 inputs, fp32 accumulate.  A's
+// rows are the TMEM lanes, one TF32 value per 32-bit column.
+__device__ __forceinline__ void umma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 template <int BN>
-constexpr uint32_t tc_stage_bytes() { return 2u * kTcWTile + 2u * BN * kTcBK * 4; }
+constexpr uint32_t tc_stage_bytes() { return kTcWTile + 2u * BN * kTcBK * 4; }
+
+// TMEM: the accumulator in columns [0, BN), then 64 columns (hi, lo) per stage.
+template <int BN>
+constexpr int tc_tmem_stages() { return (512 - BN) / 64; }
 
 template <int BN>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap w_hi, const __grid_constant__ CUtensorMap w_lo,
-                   const __grid_constant__ CUtensorMap x_hi, const __grid_constant__ CUtensorMap x_lo,
-                   TcGemmArgs a, int S) {
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap w_map, const __grid_constant__ CUtensorMap x_hi,
+                   const __grid_constant__ CUtensorMap x_lo, TcGemmArgs a, int S) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   constexpr uint32_t kXTile = BN * kTcBK * 4;
   constexpr uint32_t kStage = tc_stage_bytes<BN>();
-  constexpr uint32_t kCols = BN;  // BN in {32, 64, 128, 256}: a valid TMEM allocation
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * kStage);
-  uint64_t* empty = full + S;
+  uint64_t* split = full + S;
+  uint64_t* empty = split + S;
   uint64_t* done = empty + S;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
@@ -227,13 +252,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int layer = a.rows_per_layer ? m0 / a.rows_per_layer : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&split[i], 4);  // one arrival per split warp
+      mbar_init(&empty[i], 1);
+    }
     mbar_init(done, 1);
     *sAbort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 2) {
-    tmem_alloc(sTmem, kCols);
+    tmem_alloc(sTmem, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -249,10 +278,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint8_t* st = smem + (size_t)stage * kStage;
       const int k = (kb0 + kb) * kTcBK;
       mbar_arrive_expect_tx(&full[stage], kStage);
-      tma_load_2d(st, &w_hi, k, m0, &full[stage]);
-      tma_load_2d(st + kTcWTile, &w_lo, k, m0, &full[stage]);
-      tma_load_3d(st + 2 * kTcWTile, &x_hi, k, layer, n0, &full[stage]);
-      tma_load_3d(st + 2 * kTcWTile + kXTile, &x_lo, k, layer, n0, &full[stage]);
+      tma_load_2d(st, &w_map, k, m0, &full[stage]);
+      tma_load_3d(st + kTcWTile, &x_hi, k, layer, n0, &full[stage]);
+      tma_load_3d(st + kTcWTile + kXTile, &x_lo, k, layer, n0, &full[stage]);
       ++issued;
       if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
     }
@@ -267,41 +295,76 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr uint32_t idesc = idesc_tf32_f32(kTcBM, BN);
     uint32_t stage = 0, phase = 0;
     for (int kb = 0; kb < nkb; ++kb) {
-      if (!mbar_wait_bounded(&full[stage], phase, sAbort, a.err)) break;
+      if (!mbar_wait_bounded(&split[stage], phase, sAbort, a.err)) break;
       tc_fence_after();
       const uint32_t base = smem_u32(smem + (size_t)stage * kStage);
-      const uint64_t dwh = sdesc_kmajor_sw128(base), dwl = sdesc_kmajor_sw128(base + kTcWTile);
-      const uint64_t dxh = sdesc_kmajor_sw128(base + 2 * kTcWTile);
-      const uint64_t dxl = sdesc_kmajor_sw128(base + 2 * kTcWTile + kXTile);
+      const uint64_t dxh = sdesc_kmajor_sw128(base + kTcWTile);
+      const uint64_t dxl = sdesc_kmajor_sw128(base + kTcWTile + kXTile);
+      const uint32_t a_hi = tmem + (uint32_t)BN + stage * 64u, a_lo = a_hi + 32u;
 #pragma unroll
-      for (int k = 0; k < kTcBK / 8; ++k) {  // K = 8 tf32 (32 bytes) per MMA
+      for (int k = 0; k < kTcBK / 8; ++k) {  // K = 8 tf32 per MMA: 8 TMEM columns, 32 smem bytes
         const uint64_t o = 2u * (uint32_t)k;  // +32 bytes in the 16-byte address field
-        umma_tf32(tmem, dwh + o, dxh + o, idesc, (kb > 0 || k > 0) ? 1u : 0u);
-        umma_tf32(tmem, dwh + o, dxl + o, idesc, 1u);
-        umma_tf32(tmem, dwl + o, dxh + o, idesc, 1u);
+        const uint32_t c = 8u * (uint32_t)k;
+        umma_tf32_ts(tmem, a_hi + c, dxh + o, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+        umma_tf32_ts(tmem, a_hi + c, dxl + o, idesc, 1u);
+        umma_tf32_ts(tmem, a_lo + c, dxh + o, idesc, 1u);
       }
       umma_commit(&empty[stage]);  // the stage may be refilled once these MMAs retire
       if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
     }
     umma_commit(done);
-  }
-  // ------------------------------------------------------------ epilogue
-  int good = 1;
-  if (lane == 0) good = mbar_wait_bounded(done, 0, sAbort, a.err) && !*sAbort;
-  good = __shfl_sync(0xffffffffu, good, 0);
-  tc_fence_after();
-  if (good) {
-    const int m = m0 + warp * 32 + lane;
-    float* out = a.part + (int64_t)blockIdx.y * a.split_stride;
-#pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 32) {
-      uint32_t v[32];
-      tmem_ld32_wait(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
-      if (m < a.M) {
+  } else if (warp >= kTcSplitWarp0) {
+    // --------------------------------------------------------------- split
+    const int q = warp - kTcSplitWarp0;  // TMEM lane quarter
+    const int r = q * 32 + lane;         // row of the W tile
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    uint32_t stage = 0, phase = 0;
+    for (int kb = 0; kb < nkb; ++kb) {
+      // every lane waits (each needs the TMA data visible); the warp leaves
+      // together if any lane's wait ran out, before the .aligned TMEM stores
+      const bool ok = mbar_wait_bounded(&full[stage], phase, sAbort, a.err);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      // row r: 128 bytes, its 16-byte chunk c stored at chunk c ^ (r % 8)
+      const uint8_t* row = smem + (size_t)stage * kStage + (size_t)r * 128;
+      uint32_t hi[32], lo[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int n = n0 + c0 + j;
-          if (n < a.N) out[(int64_t)n * a.M + m] = __uint_as_float(v[j]);
+      for (int c = 0; c < 8; ++c) {
+        const float4 v = *reinterpret_cast<const float4*>(row + ((c ^ (r & 7)) << 4));
+        const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float h = tf32_round(e[i]);
+          hi[4 * c + i] = __float_as_uint(h);
+          lo[4 * c + i] = __float_as_uint(e[i] - h);
+        }
+      }
+      const uint32_t col = (uint32_t)BN + stage * 64u;
+      tmem_st32_wait(lane_base + col, hi);
+      tmem_st32_wait(lane_base + col + 32u, lo);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&split[stage]);
+      if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
+    }
+    // ---------------------------------------------------------- epilogue
+    int good = 1;
+    if (lane == 0) good = mbar_wait_bounded(done, 0, sAbort, a.err) && !*sAbort;
+    good = __shfl_sync(0xffffffffu, good, 0);
+    tc_fence_after();
+    if (good) {
+      const int m = m0 + r;
+      float* out = a.part + (int64_t)blockIdx.y * a.split_stride;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32_wait(lane_base + (uint32_t)c0, v);
+        if (m < a.M) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = n0 + c0 + j;
+            if (n < a.N) out[(int64_t)n * a.M + m] = __uint_as_float(v[j]);
+          }
         }
       }
     }
@@ -310,7 +373,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem, kCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -609,30 +672,30 @@ void launch_split(const float* x, float* hi, float* lo, int64_t n, cudaStream_t 
 }
 
 template <int BN>
-fm_status launch_tc_gemm_bn(fm_ctx* ctx, const void* wh, const void* wl, const void* xh, const void* xl,
-                            const TcGemmArgs& a, int mtiles, int ksplit, int ntiles, cudaStream_t st) {
+fm_status launch_tc_gemm_bn(fm_ctx* ctx, const void* wmap, const void* xh, const void* xl, const TcGemmArgs& a,
+                            int mtiles, int ksplit, int ntiles, cudaStream_t st) {
   static int configured_dev = -1;
   constexpr uint32_t stage = tc_stage_bytes<BN>();
   int S = (int)((200u * 1024u) / stage);
-  S = S < 2 ? 2 : (S > 6 ? 6 : S);
-  const uint32_t smem = (uint32_t)S * stage + (uint32_t)(2 * S + 1) * 8 + 16 + 1024;
+  S = S < 2 ? 2 : S;
+  if (S > tc_tmem_stages<BN>()) S = tc_tmem_stages<BN>();
+  const uint32_t smem = (uint32_t)S * stage + (uint32_t)(3 * S + 1) * 8 + 16 + 1024;
   if (configured_dev != ctx->device) {
-    if (cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+    if (cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
         cudaSuccess)
       return check_launch();
     configured_dev = ctx->device;
   }
   tc_gemm_kernel<BN><<<dim3(mtiles, ksplit, ntiles), kTcThreads, smem, st>>>(
-      *reinterpret_cast<const CUtensorMap*>(wh), *reinterpret_cast<const CUtensorMap*>(wl),
-      *reinterpret_cast<const CUtensorMap*>(xh), *reinterpret_cast<const CUtensorMap*>(xl), a, S);
+      *reinterpret_cast<const CUtensorMap*>(wmap), *reinterpret_cast<const CUtensorMap*>(xh),
+      *reinterpret_cast<const CUtensorMap*>(xl), a, S);
   note_launch();
   return check_launch();
 }
 
-// part[s][n][m] for W (maps wh, wl: [M, K]) against X (maps xh, xl) in K splits.
-fm_status launch_tc_gemm(fm_ctx* ctx, const void* wh, const void* wl, const float* x_hi, const float* x_lo,
-                         int x_layers, int M, int N, int K, int ksplit, int rows_per_layer, float* part,
-                         cudaStream_t st) {
+// part[s][n][m] for W (fp32 map: [M, K]) against X (split maps) in K splits.
+fm_status launch_tc_gemm(fm_ctx* ctx, const void* wmap, const float* x_hi, const float* x_lo, int x_layers,
+                         int M, int N, int K, int ksplit, int rows_per_layer, float* part, cudaStream_t st) {
   const int bn = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
   alignas(64) unsigned char xh[128], xl[128];
   if (!encode_act_map(xh, x_hi, N, x_layers, K, bn) || !encode_act_map(xl, x_lo, N, x_layers, K, bn))
@@ -646,10 +709,10 @@ fm_status launch_tc_gemm(fm_ctx* ctx, const void* wh, const void* wl, const floa
   a.err = ctx->d_err;
   const int mtiles = (M + kTcBM - 1) / kTcBM, ntiles = (N + bn - 1) / bn;
   switch (bn) {
-    case 32: return launch_tc_gemm_bn<32>(ctx, wh, wl, xh, xl, a, mtiles, ksplit, ntiles, st);
-    case 64: return launch_tc_gemm_bn<64>(ctx, wh, wl, xh, xl, a, mtiles, ksplit, ntiles, st);
-    case 128: return launch_tc_gemm_bn<128>(ctx, wh, wl, xh, xl, a, mtiles, ksplit, ntiles, st);
-    default: return launch_tc_gemm_bn<256>(ctx, wh, wl, xh, xl, a, mtiles, ksplit, ntiles, st);
+    case 32: return launch_tc_gemm_bn<32>(ctx, wmap, xh, xl, a, mtiles, ksplit, ntiles, st);
+    case 64: return launch_tc_gemm_bn<64>(ctx, wmap, xh, xl, a, mtiles, ksplit, ntiles, st);
+    case 128: return launch_tc_gemm_bn<128>(ctx, wmap, xh, xl, a, mtiles, ksplit, ntiles, st);
+    default: return launch_tc_gemm_bn<256>(ctx, wmap, xh, xl, a, mtiles, ksplit, ntiles, st);
   }
 }
 
@@ -666,7 +729,7 @@ fm_status launch_query_prep_tc(fm_ctx* ctx, const float* hidden, const int64_t* 
   while (ks_d * 2 <= ctx->splitk_max && (HID / kTcBK) % (ks_d * 2) == 0 && mtiles_d * bn_tiles * ks_d < ctx->num_sms)
     ks_d *= 2;
   launch_split(hidden, ctx->x_hi, ctx->x_lo, (int64_t)B * HID, st);
-  fm_status s = launch_tc_gemm(ctx, ctx->wmaps[0], ctx->wmaps[1], ctx->x_hi, ctx->x_lo, 1, Md, B, HID, ks_d, 0,
+  fm_status s = launch_tc_gemm(ctx, ctx->wmaps[0], ctx->x_hi, ctx->x_lo, 1, Md, B, HID, ks_d, 0,
                                ctx->a_part, st);
   if (s != FM_OK) return s;
   const float w_scale = (float)(1.0 / sqrt((double)c.head_dim * (double)c.n_heads));
@@ -676,7 +739,7 @@ fm_status launch_query_prep_tc(fm_ctx* ctx, const float* hidden, const int64_t* 
   note_launch();
   // up projection: two K splits (its partials buffer holds two)
   const int ks_u = (R / kTcBK) % 2 == 0 ? 2 : 1;
-  s = launch_tc_gemm(ctx, ctx->wmaps[2], ctx->wmaps[3], ctx->r_hi, ctx->r_lo, L, Mu, B, R, ks_u,
+  s = launch_tc_gemm(ctx, ctx->wmaps[1], ctx->r_hi, ctx->r_lo, L, Mu, B, R, ks_u,
                      kHeads * kHeadDim, ctx->up_part, st);
   if (s != FM_OK) return s;
   const int warps = B * L * kHeads;
@@ -692,23 +755,16 @@ fm_status prepare_tc_weights(fm_ctx* ctx) {
   const fm_config& c = ctx->cfg;
   const int L = c.n_layers, R = c.q_lora_rank, HID = c.hidden;
   const int Md = L * (R + kHeads), Mu = L * kHeads * kHeadDim;
-  ctx->tc_ok = 0;
-  launch_split(ctx->w_down, ctx->w_down_hi, ctx->w_down_lo, (int64_t)Md * HID, 0);
-  launch_split(ctx->w_up, ctx->w_up_hi, ctx->w_up_lo, (int64_t)Mu * R, 0);
-  const fm_status s = check_launch();
-  if (s != FM_OK) return s;
-  ctx->tc_ok = encode_weight_map(ctx->wmaps[0], ctx->w_down_hi, Md, HID) &&
-               encode_weight_map(ctx->wmaps[1], ctx->w_down_lo, Md, HID) &&
-               encode_weight_map(ctx->wmaps[2], ctx->w_up_hi, Mu, R) &&
-               encode_weight_map(ctx->wmaps[3], ctx->w_up_lo, Mu, R);
+  ctx->tc_ok = encode_weight_map(ctx->wmaps[0], ctx->w_down, Md, HID) &&
+               encode_weight_map(ctx->wmaps[1], ctx->w_up, Mu, R);
   return FM_OK;
 }
 
 fm_status launch_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* positions, int B,
                             float* q, float* fused_w, cudaStream_t st) {
-  // Past 8 rows the projections are bound by fp32 FMA on the CUDA cores; the
-  // tensor-core path then reads twice the weight bytes (hi and lo) at a far
-  // higher math rate.  Up to 8 rows the CUDA-core GEMVs read the weights once.
+  // Past 8 rows the projections are bound by fp32 FMA on the CUDA cores and
+  // the tensor-core path (three-pass TF32) takes over; up to 8 rows the
+  // CUDA-core GEMVs are bound by the weight bytes, which both paths read once.
   if (ctx->tc_ok && B > 8) return launch_query_prep_tc(ctx, hidden, positions, B, q, fused_w, st);
   const fm_config& c = ctx->cfg;
   const int M = c.n_layers * (c.q_lora_rank + c.n_heads);
