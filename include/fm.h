@@ -136,7 +136,12 @@ fm_status fm_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* positio
  * q, fused_w as written by fm_query_prep (any producer is fine).
  * scores    [L, B, N] fp32 device (written; 0.0f past n_valid).
  * The product k.q runs on the tensor cores with q split into q_pieces e4m3
- * terms (per-head power-of-two scaling) and the keys used as stored. */
+ * terms (per-head power-of-two scaling) and the keys used as stored.
+ * The comp_k pointers may alias.  All layers reading one key tensor is the
+ * README "Usage" signature taken literally (one compressed_k scored by the
+ * three layers' queries).  The pass loads a tile's layers one after another,
+ * so with aliased pointers the repeats come from L2 and HBM reads the keys
+ * once. */
 fm_status fm_score(fm_ctx* ctx, const uint8_t* const* comp_k, int64_t row_stride_bytes,
                    const int32_t* n_valid, int B, int N, const float* q, const float* fused_w,
                    float* scores, cudaStream_t stream);

@@ -224,3 +224,21 @@ def test_argument_errors(retr, weights):
     assert lib.fm_score_fused(retr.handle, arr, 256 * 132, None, 2, 256, P(q), P(w), 7, 0.0, None,
                               P(ens), None, st) == fm.FM_ERR_INVALID_ARG
     retr.fm_sync_status()
+
+
+def test_shared_keys_across_layers(retr, weights):
+    """One compressed_k scored by all three layers' queries (the README "Usage"
+    signature taken literally): the layers' pointers alias one key tensor."""
+    case = H.make_case(3, 1001, [1001, 517, 129], seed=21, weights=weights)
+    shared = case.comp_k[0].to(DEV)
+    case.comp_k = [case.comp_k[0]] * 3  # the oracle scores the same keys for every layer
+    q, w = _run_query(retr, case)
+    s = retr.fm_score([shared] * 3, q, w, n_valid=case.n_valid.to(DEV), N=case.N).cpu().numpy()
+    want = H.oracle_scores(case)
+    assert np.abs(s - want).max() <= H.SCORE_TOL
+    ens, keep_thr, _ = retr.fm_score_fused([shared] * 3, q, w, mode="mean", threshold=0.5,
+                                           n_valid=case.n_valid.to(DEV), N=case.N)
+    ens = ens.cpu().numpy()
+    assert np.abs(ens - O.ensemble(want, "mean")).max() <= H.SCORE_TOL
+    np.testing.assert_array_equal(keep_thr.cpu().numpy(), O.select_threshold(ens, case.n_valid.numpy(), 0.5))
+    retr.fm_sync_status()
