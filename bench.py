@@ -50,10 +50,12 @@ def parse():
     ap.add_argument("--shared-keys", action="store_true",
                     help="one compressed_k tensor scored by all three layers' queries (the README "
                          "Usage signature taken literally); reports against the fp8 tensor peak")
-    ap.add_argument("--path", default="retrieve", choices=["retrieve", "recall", "level2"],
+    ap.add_argument("--path", default="retrieve", choices=["retrieve", "recall", "level2", "decode"],
                     help="retrieve: the scoring path (default); recall: keep mask -> index lists -> "
                          "gather of the kept chunks' records into a resident buffer; level2: the "
-                         "per-step top-512 over a resident set of 4096 chunks per row, one CUDA graph")
+                         "per-step top-512 over a resident set of 4096 chunks per row, one CUDA graph; "
+                         "decode: the toy sparse decode loop (retrieval every 64 steps, attention over the "
+                         "kept chunks every step)")
     return ap.parse_args()
 
 
@@ -504,6 +506,78 @@ def run_level2(args):
             "gpu_launches_per_step": "one graph launch", "clocks": sampler.summary()}
 
 
+# -------------------------------------------------------------- decode path
+def run_decode(args):
+    """The README's toy decode loop on the 64-row workload (64 rows x 262144
+    chunks per layer, top-4096): one timed unit is a retrieval cycle, i.e. 64
+    decode steps of which the first runs the retriever over all chunks; every
+    step runs the sparse attention over the 4096 kept chunks and the state
+    update.  The attention kernel is also timed alone (L2 flushed first)."""
+    from learned_kv_chunk_b200 import fm
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = G.WORKLOADS[4]
+    inp = G.make_query_inputs(wl)
+    B, N, L, K = wl.B, wl.N, G.N_LAYERS, wl.top_k
+    r = fm.Retriever(inp.weights, device=0, max_batch=B, q_pieces=args.q_pieces)
+    hidden = inp.hidden.to(dev)
+    q, _ = r.fm_query_prep(hidden, inp.positions.to(dev))
+    plant = q[:, :, 0, :].permute(1, 0, 2).contiguous().cpu()
+    keys = G.make_keys(wl.seed(G.SEED_KEYS), [int(x) for x in inp.n_valid], N, L, plant, device=dev)
+    n_valid = inp.n_valid.to(dev)
+    dec = fm.ToySparseDecoder(r, keys, n_valid, hidden, inp.positions, top_k=K, mode=wl.mode)
+    stream = torch.cuda.current_stream()
+    interval = dec.interval
+    for _ in range(max(3, args.warmup)):
+        dec.step()
+    while dec.t % interval:
+        dec.step()
+    torch.cuda.synchronize()
+    r.fm_sync_status()
+    cycles = max(1, args.steps // interval) if args.steps >= interval else 1
+    sampler = ClockSampler(0)
+    launches0 = fm.fm_launch_count()
+    with sampler:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(cycles * interval):
+            dec.step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        t_cycle = a.elapsed_time(b) / cycles
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        flush_buf = torch.empty(max(2 * l2, 1 << 28) // 4, device=dev, dtype=torch.float32)
+        ws = torch.empty(int(fm.lib().fm_decode_attention_workspace_bytes(B, K)), device=dev, dtype=torch.uint8)
+        out = torch.empty(B, 32, 128, device=dev)
+        t_attn = _timed_flushed(lambda: fm.fm_decode_attention(dec.hidden.view(B, 32, 128), dec.mem, dec.idx,
+                                                                dec.count, out=out, workspace=ws),
+                                20, flush_buf, stream)
+    launches = fm.fm_launch_count() - launches0
+    r.fm_sync_status()
+    kept = int(dec.count.clamp(max=K).sum())
+    flops = kept * 32 * 128 * 4  # q.x and p.x: one multiply-add each per (chunk, head, dim)
+    alu_peak = 148 * 128 * 2 * 1965e6 / 1e12  # fp32 lanes x 2 FLOP x max SM clock
+    ach = flops / (t_attn / 1e3) / 1e12
+    r.close()
+    return {"metric": "toy sparse decode tokens/sec (retrieval every 64 steps, attention over kept chunks)",
+            "value": B * interval / (t_cycle / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": cycles * interval,
+            "warmup": max(3, args.warmup), "ms_per_step": t_cycle / interval, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 (attention), e4m3 (retrieval)",
+            "data": "synthetic (seeded generator, random-init weights)",
+            "config": {"workload": "decode_B64_N262144_top4096_interval64", "rows": B, "chunks_per_row": N,
+                       "kept_per_row": K, "retrieval_interval": interval, "attention_heads": 32,
+                       "l2": "cycle inputs larger than L2 (6.64 GB of keys per retrieval); attention timed "
+                             "alone after a 256 MB L2 flush"},
+            "cycle_ms": round(t_cycle, 4),
+            "roofline": {"bound": "alu", "achieved": round(ach, 2), "peak": round(alu_peak, 1), "unit": "TFLOP/s",
+                         "frac": round(ach / alu_peak, 4), "traffic": None,
+                         "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz",
+                         "kernel": "sparse attention over the kept chunks (partial + combine)",
+                         "kernel_ms": round(t_attn, 4), "alg_flops_per_launch": flops},
+            "gpu_launches": launches, "clocks": sampler.summary()}
+
+
 def recall_oracle_sample(keep, src, K, rows=1):
     """The recall oracle (compaction + gather, plain loops) on the first rows."""
     import oracle.recall as OR
@@ -604,6 +678,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.path == "decode":
+        if rank == 0:
+            print(json.dumps(run_decode(args)), flush=True)
+        return
     if args.path == "level2":
         if rank == 0:
             print(json.dumps(run_level2(args)), flush=True)

@@ -331,6 +331,39 @@ fm_status fm_level2_copy_scores(const fm_level2* step, float* dst, cudaStream_t 
 /* Waits for the device and frees the step. */
 fm_status fm_level2_destroy(fm_level2* step);
 
+/* ------------------------------------------------------- toy sparse decode
+ * README "Toy inference reference": every decode step runs a sparse memory
+ * attention over the N compressed chunks in which the chunks the last
+ * retrieval did not keep get -inf logits; every 64 steps the retriever
+ * refreshes the keep mask.  The toy decoder is not defined by the pages; these
+ * calls take the plainest weight-free reading:
+ *   query   the step's hidden state [4096] as 32 heads of 128 (q [B, 32, 128]);
+ *   memory  chunk i's vector x_i = e4m3(bytes[0:128]) * f32le(bytes[128:132]),
+ *           used as key and value;
+ *   o_h     = sum_i softmax_i(q_h . x_i / sqrt(128)) x_i over the kept chunks
+ *           (the others' logits are -inf); a row with no kept chunk gives 0;
+ *   update  hidden' = RMSNorm(hidden + o), no gain. */
+
+/* Bytes of device workspace fm_decode_attention needs. */
+size_t fm_decode_attention_workspace_bytes(int B, int max_sel);
+
+/* The sparse attention, reading only the kept chunks: idx/count as written by
+ * fm_compact_mask for the keep mask (the first min(count[b], max_sel) entries
+ * of idx[b] are the kept chunk indices; an index outside [0, n_mem) counts as
+ * masked).  q [B, 32, 128] fp32 device, 16-byte aligned; mem: the chunk
+ * records [B, n_mem, 132] uint8 device, row b at mem + b*row_stride_bytes
+ * (4-byte aligned, row_stride_bytes >= n_mem*132, a multiple of 4);
+ * out [B, 32, 128] fp32 device (written); ws: the workspace, 16-byte aligned. */
+fm_status fm_decode_attention(const float* q, const uint8_t* mem, int64_t row_stride_bytes, int n_mem,
+                              const int32_t* idx, const int32_t* count, int B, int max_sel, float* out,
+                              void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* The toy decoder's state update: hidden_out[b] = RMSNorm(hidden[b] + attn_out[b])
+ * with eps and no gain; H = 4096 (the attention output flattened head-major).
+ * All [B, H] fp32 device; hidden_out may alias hidden. */
+fm_status fm_toy_decoder_update(const float* hidden, const float* attn_out, int B, int H, float eps,
+                                float* hidden_out, cudaStream_t stream);
+
 /* Synchronises `stream` and returns FM_ERR_DEVICE if a kernel launched on this
  * context recorded an error since the last call (the record is cleared),
  * FM_ERR_CUDA if the stream reports a CUDA error, FM_OK otherwise. */

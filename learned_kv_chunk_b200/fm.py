@@ -82,6 +82,9 @@ def _load():
         "fm_level2_launch": (I, [P, P]),
         "fm_level2_copy_scores": (I, [P, P, P]),
         "fm_level2_destroy": (I, [P]),
+        "fm_decode_attention_workspace_bytes": (S, [I, I]),
+        "fm_decode_attention": (I, [P, P, I64, I, P, P, I, I, P, P, S, P]),
+        "fm_toy_decoder_update": (I, [P, P, I, I, F, P, P]),
         "fm_topk_shard_begin": (I, [P, I, I, I, P, P, S, P]),
         "fm_topk_shard_hist": (I, [P, I, I, I, P, P, S, P]),
         "fm_topk_shard_pick": (I, [I, I, I, P, P, S, P]),
@@ -316,6 +319,93 @@ class Level2Step:
             self.close()
         except Exception:
             pass
+
+
+def fm_decode_attention(q: torch.Tensor, mem: torch.Tensor, idx: torch.Tensor, count: torch.Tensor,
+                        out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """The toy decoder's sparse attention over the kept chunks: q [B, 32, 128]
+    fp32 (the hidden state [B, 4096] viewed as 32 heads), mem [B, N, 132]
+    uint8 chunk records, idx/count from fm_compact_mask.  Returns o [B, 32, 128]."""
+    _need(q, torch.float32, "q")
+    _need(mem, torch.uint8, "mem")
+    _need(idx, torch.int32, "idx")
+    _need(count, torch.int32, "count")
+    B, n_mem, rec = mem.shape
+    if rec != 132:
+        raise ValueError("mem must be [B, N, 132] uint8")
+    max_sel = idx.shape[1]
+    out = out if out is not None else torch.empty(B, 32, 128, device=q.device, dtype=torch.float32)
+    nbytes = int(_lib.fm_decode_attention_workspace_bytes(B, max_sel))
+    ws = workspace if workspace is not None else torch.empty(nbytes, device=q.device, dtype=torch.uint8)
+    _check(_lib.fm_decode_attention(_ptr(q), _ptr(mem), n_mem * 132, n_mem, _ptr(idx), _ptr(count), B, max_sel,
+                                    _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "fm_decode_attention")
+    return out
+
+
+def fm_toy_decoder_update(hidden: torch.Tensor, attn_out: torch.Tensor, eps: float = 1e-6,
+                          out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """hidden' = RMSNorm(hidden + attn_out) (no gain); out may be hidden itself."""
+    _need(hidden, torch.float32, "hidden")
+    _need(attn_out, torch.float32, "attn_out")
+    B, H = hidden.shape
+    out = out if out is not None else torch.empty_like(hidden)
+    _check(_lib.fm_toy_decoder_update(_ptr(hidden), _ptr(attn_out), B, H, float(eps), _ptr(out),
+                                      _stream(stream)), "fm_toy_decoder_update")
+    return out
+
+
+class ToySparseDecoder:
+    """The README's toy decode loop ("Toy inference reference") on synthetic
+    inputs: every `interval` (64) steps the retriever scores all chunks of the
+    three layers for the current hidden state and the keep mask (top-K, or
+    sigmoid > threshold) is compacted into index lists; every step the toy
+    decoder attends over the kept chunks of the memory layer and updates its
+    hidden state (fm_decode_attention, fm_toy_decoder_update).  Positions
+    advance by one token per step from `positions`."""
+
+    def __init__(self, retriever: "Retriever", comp_k: Sequence[torch.Tensor], n_valid: torch.Tensor,
+                 hidden: torch.Tensor, positions: torch.Tensor, top_k: Optional[int] = 512,
+                 threshold: Optional[float] = None, mode: str = "max", interval: int = 64,
+                 memory_layer: int = 0):
+        if (top_k is None) == (threshold is None):
+            raise ValueError("give exactly one of top_k and threshold")
+        self.r, self.comp_k, self.n_valid = retriever, list(comp_k), n_valid
+        self.B, self.N = comp_k[0].shape[0], comp_k[0].shape[1]
+        dev = hidden.device
+        self.hidden = hidden.clone()
+        self.positions0 = positions.detach().to("cpu", torch.int64)
+        self.top_k, self.threshold, self.mode, self.interval = top_k, threshold, mode, int(interval)
+        self.mem = self.comp_k[memory_layer]
+        self.max_sel = int(top_k) if top_k is not None else self.N
+        self.idx = torch.empty(self.B, self.max_sel, device=dev, dtype=torch.int32)
+        self.count = torch.empty(self.B, device=dev, dtype=torch.int32)
+        self.attn = torch.empty(self.B, 32, 128, device=dev, dtype=torch.float32)
+        self._cws = torch.empty(int(_lib.fm_compact_workspace_bytes(self.B, self.N)), device=dev,
+                                dtype=torch.uint8)
+        self._aws = torch.empty(int(_lib.fm_decode_attention_workspace_bytes(self.B, self.max_sel)), device=dev,
+                                dtype=torch.uint8)
+        self.t = 0
+        self.keep = None
+        self.ens = None
+
+    def retrieve(self):
+        pos = (self.positions0 + self.t).to(self.hidden.device)
+        ens, keep_topk, keep_thr = self.r.retrieve(self.hidden, self.comp_k, pos, self.n_valid, self.mode,
+                                                   self.top_k, self.threshold, self.N)
+        self.ens = ens
+        self.keep = keep_topk if self.top_k is not None else keep_thr
+        fm_compact_mask(self.keep, self.max_sel, idx=self.idx, count=self.count, workspace=self._cws)
+
+    def step(self):
+        """One decode step; returns the new hidden state [B, 4096]."""
+        if self.t % self.interval == 0:
+            self.retrieve()
+        fm_decode_attention(self.hidden.view(self.B, 32, 128), self.mem, self.idx, self.count, out=self.attn,
+                            workspace=self._aws)
+        fm_toy_decoder_update(self.hidden, self.attn.view(self.B, -1), out=self.hidden)
+        self.t += 1
+        return self.hidden
 
 
 class TopKShard:

@@ -207,3 +207,59 @@ def test_recall_pins_catch_planted_mistake(monkeypatch, name, fn):
         except Exception:  # noqa: BLE001 - any failure counts as detection
             caught.append(pin.__name__)
     assert caught, f"no pin caught the mutation {name}:{fn.__name__}"
+
+
+# -------------------------------------------------------------- toy decode
+import math  # noqa: E402
+
+import oracle.decode as OD  # noqa: E402
+
+
+def _attn_generic(q, x, keep, scale=True, mask_value=-np.inf, normalise=True, over_heads=False):
+    q = np.asarray(q, np.float64)
+    x = np.asarray(x, np.float64)
+    B, H, D = q.shape
+    out = np.zeros((B, H, D))
+    for b in range(B):
+        if not keep[b].any():
+            continue
+        lg = q[b] @ x[b].T / (math.sqrt(D) if scale else 1.0)
+        lg = np.where(keep[b][None, :], lg, mask_value)
+        ax = 0 if over_heads else 1
+        e = np.exp(lg - lg.max(axis=ax, keepdims=True))
+        p = e / e.sum(axis=ax, keepdims=True) if normalise else e
+        out[b] = p @ x[b]
+    return out
+
+
+def _update_no_residual(hidden, o, eps=1e-6):
+    return OD.__dict__["_orig_toy_update"](np.zeros_like(hidden), o, eps)
+
+
+def _step_dim_major(hidden, x, keep):
+    B = hidden.shape[0]
+    q = np.asarray(hidden, np.float64).reshape(B, 128, 32).transpose(0, 2, 1)
+    return OD.toy_update(hidden, OD.masked_attention(q, x, keep))
+
+
+DECODE_MUTATIONS = [
+    ("masked_attention", lambda q, x, k: _attn_generic(q, x, k, scale=False)),
+    ("masked_attention", lambda q, x, k: _attn_generic(q, x, k, mask_value=0.0)),
+    ("masked_attention", lambda q, x, k: _attn_generic(q, x, k, normalise=False)),
+    ("masked_attention", lambda q, x, k: _attn_generic(q, x, k, over_heads=True)),
+    ("toy_update", _update_no_residual),
+    ("toy_step", _step_dim_major),
+]
+
+
+@pytest.mark.parametrize("name,fn", DECODE_MUTATIONS, ids=[f"{n}:{i}" for i, (n, _) in enumerate(DECODE_MUTATIONS)])
+def test_decode_pins_catch_planted_mistake(monkeypatch, name, fn):
+    monkeypatch.setitem(OD.__dict__, "_orig_" + name, getattr(OD, name))
+    monkeypatch.setattr(OD, name, fn)
+    caught = []
+    for pin in PINS:
+        try:
+            pin()
+        except Exception:  # noqa: BLE001 - any failure counts as detection
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the mutation {name}"

@@ -453,3 +453,88 @@ def test_gather_matches_fancy_indexing():
         m = min(int(count[b]), 20)
         assert np.array_equal(out[b, :m], src[b][np.flatnonzero(keep[b])[:m]])  # library routine
         assert not out[b, m:].any()
+
+
+# -------------------------------------------------------------- toy decode
+import oracle.decode as OD  # noqa: E402
+
+
+def _vecs(seed, B, N, D=128):
+    return np.random.default_rng(seed).standard_normal((B, N, D))
+
+
+def test_attention_single_kept_chunk_returns_it():
+    x = _vecs(1, 2, 7)
+    q = np.random.default_rng(2).standard_normal((2, 32, 128))
+    keep = np.zeros((2, 7), bool)
+    keep[0, 3] = True
+    keep[1, 6] = True
+    o = OD.masked_attention(q, x, keep)
+    np.testing.assert_allclose(o[0], np.broadcast_to(x[0, 3], (32, 128)), rtol=1e-14)
+    np.testing.assert_allclose(o[1], np.broadcast_to(x[1, 6], (32, 128)), rtol=1e-14)
+
+
+def test_attention_two_chunks_closed_form():
+    # q = 2 e_0 and x_1 = 3 e_0, x_2 = -e_0 + e_5: logits 6/sqrt(128) and -2/sqrt(128)
+    q = np.zeros((1, 32, 128))
+    q[0, :, 0] = 2.0
+    x = np.zeros((1, 3, 128))
+    x[0, 1, 0] = 3.0
+    x[0, 2, 0] = -1.0
+    x[0, 2, 5] = 1.0
+    x[0, 0, :] = 1e6  # a masked chunk: must not matter
+    keep = np.array([[False, True, True]])
+    p1 = 1.0 / (1.0 + math.exp(-(6.0 + 2.0) / math.sqrt(128)))
+    want = p1 * x[0, 1] + (1 - p1) * x[0, 2]
+    o = OD.masked_attention(q, x, keep)
+    np.testing.assert_allclose(o[0, 7], want, rtol=1e-13, atol=1e-15)
+
+
+def test_attention_masked_chunks_do_not_matter_and_empty_row_is_zero():
+    rng = np.random.default_rng(5)
+    x = _vecs(6, 2, 40)
+    q = rng.standard_normal((2, 32, 128))
+    keep = rng.random((2, 40)) < 0.4
+    keep[1] = False
+    o = OD.masked_attention(q, x, keep)
+    x2 = x.copy()
+    x2[~keep] = rng.standard_normal(((~keep).sum(), 128)) * 1e3
+    np.testing.assert_allclose(OD.masked_attention(q, x2, keep), o, rtol=1e-12, atol=1e-12)
+    assert (o[1] == 0).all()
+    # softmax weights of the kept chunks: the output is a convex combination
+    sub = x[0, keep[0]]
+    assert (o[0] <= sub.max(axis=0) + 1e-12).all() and (o[0] >= sub.min(axis=0) - 1e-12).all()
+
+
+def test_attention_heads_are_independent_and_equal_vectors_give_the_vector():
+    x = np.tile(_vecs(7, 1, 1), (1, 9, 1))
+    q = np.random.default_rng(8).standard_normal((1, 32, 128))
+    o = OD.masked_attention(q, x, np.ones((1, 9), bool))
+    np.testing.assert_allclose(o[0], np.broadcast_to(x[0, 0], (32, 128)), rtol=1e-13)
+    # a query aligned with chunk j for head 5 only: head 5 weights chunk j most
+    x = _vecs(9, 1, 6) / 10
+    q = np.zeros((1, 32, 128))
+    q[0, 5] = 40.0 * x[0, 2] / np.linalg.norm(x[0, 2])
+    o = OD.masked_attention(q, x, np.ones((1, 6), bool))
+    assert np.argmin(np.linalg.norm(x[0] - o[0, 5], axis=1)) == 2
+    np.testing.assert_allclose(o[0, 4], x[0].mean(axis=0), rtol=1e-12)  # head 4: zero query, uniform weights
+
+
+def test_toy_step_is_rmsnorm_of_residual():
+    rng = np.random.default_rng(10)
+    h = rng.standard_normal((2, 4096))
+    x = _vecs(11, 2, 30)
+    keep = rng.random((2, 30)) < 0.5
+    out = OD.toy_step(h, x, keep)
+    o = OD.masked_attention(h.reshape(2, 32, 128), x, keep).reshape(2, 4096)
+    v = h + o
+    np.testing.assert_allclose(np.sqrt(np.mean(out * out, axis=1)), np.sqrt(np.mean(v * v, axis=1) /
+                               (np.mean(v * v, axis=1) + 1e-6)), rtol=1e-12)
+    cos = (out * v).sum(1) / np.linalg.norm(out, axis=1) / np.linalg.norm(v, axis=1)
+    np.testing.assert_allclose(cos, 1.0, rtol=1e-12)
+    # head h of the query is hidden[h*128:(h+1)*128]: one kept chunk makes o = x for every head
+    keep1 = np.zeros((2, 30), bool)
+    keep1[:, 4] = True
+    out1 = OD.toy_step(h, x, keep1)
+    want = h + np.tile(x[:, 4], (1, 32))
+    np.testing.assert_allclose(out1, want / np.sqrt(np.mean(want * want, 1, keepdims=True) + 1e-6), rtol=1e-12)
