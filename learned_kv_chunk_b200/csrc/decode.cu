@@ -85,21 +85,38 @@ __global__ void __launch_bounds__(kAThreads) sparse_attn_partial_kernel(
     const int h = i / (kAD / 4), d4 = i % (kAD / 4);
     *reinterpret_cast<float4*>(&S.q[h][4 * d4]) = __ldg(qr + i);
   }
-  // gather + dequantize: warp w takes records w, w+8, ...; lane l the 4 codes l
+  // gather + dequantize: warp w takes records w + 8k (k < 16), lane l the 4
+  // codes l of each; all 16 records' loads are issued before any is used
   const uint8_t* row = mem + (size_t)b * row_stride;
   const int32_t* ids = idx + (size_t)b * max_sel + c0;
-  for (int c = warp; c < kSeg; c += kAThreads / 32) {
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    const int id = c < nc ? ids[c] : -1;
-    const bool ok = id >= 0 && id < n_mem;  // an index outside the memory counts as masked
-    if (lane == 0) S.valid[c] = ok ? 1 : 0;
-    if (ok) {
-      const uint8_t* rec = row + (int64_t)id * kRecord;
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(rec + 4 * lane);
-      const float s = __uint_as_float(*reinterpret_cast<const uint32_t*>(rec + 128));
-      dequant4(w, s, v);
+  {
+    constexpr int kPer = kSeg / (kAThreads / 32);
+    int id[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int c = warp + 8 * k;
+      id[k] = c < nc ? __ldg(ids + c) : -1;
     }
-    *reinterpret_cast<float4*>(&S.x[c][4 * lane]) = make_float4(v[0], v[1], v[2], v[3]);
+    uint32_t w[kPer], sc[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      w[k] = 0u;
+      sc[k] = 0u;
+      if (id[k] >= 0 && id[k] < n_mem) {  // an index outside the memory counts as masked
+        const uint8_t* rec = row + (int64_t)id[k] * kRecord;
+        w[k] = __ldg(reinterpret_cast<const uint32_t*>(rec + 4 * lane));
+        sc[k] = __ldg(reinterpret_cast<const uint32_t*>(rec + 128));
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int c = warp + 8 * k;
+      const bool ok = id[k] >= 0 && id[k] < n_mem;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (ok) dequant4(w[k], __uint_as_float(sc[k]), v);
+      if (lane == 0) S.valid[c] = ok ? 1 : 0;
+      *reinterpret_cast<float4*>(&S.x[c][4 * lane]) = make_float4(v[0], v[1], v[2], v[3]);
+    }
   }
   __syncthreads();
   // logits: thread t -> heads hg + 8i, chunks cg + 32j (i, j < 4)
@@ -183,30 +200,27 @@ __global__ void __launch_bounds__(kAThreads) sparse_attn_partial_kernel(
   }
 }
 
-// Merges the segments of row blockIdx.x: o_h = sum_s e^(m_s - M) o_s / sum_s e^(m_s - M) l_s.
-__global__ void __launch_bounds__(kAThreads) sparse_attn_combine_kernel(const float* __restrict__ part_o,
-                                                                        const float* __restrict__ part_ml,
-                                                                        int nseg, float* __restrict__ out) {
-  const int b = blockIdx.x;
+// Merges the segments of (head blockIdx.x, row blockIdx.y), thread d one
+// output dim: o = sum_s e^(m_s - M) o_s / sum_s e^(m_s - M) l_s.
+__global__ void __launch_bounds__(kAD) sparse_attn_combine_kernel(const float* __restrict__ part_o,
+                                                                  const float* __restrict__ part_ml, int nseg,
+                                                                  float* __restrict__ out) {
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const float* pml = part_ml + (size_t)b * nseg * kAH * 2;
   const float* po = part_o + (size_t)b * nseg * kAH * kAD;
-  float* o = out + (size_t)b * kAH * kAD;
-  for (int i = threadIdx.x; i < kAH * kAD; i += kAThreads) {
-    const int h = i / kAD;
-    float M = -INFINITY;
-    for (int s = 0; s < nseg; ++s) M = fmaxf(M, pml[((size_t)s * kAH + h) * 2]);
-    float num = 0.f, den = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < nseg; ++s) {
-        const float ms = pml[((size_t)s * kAH + h) * 2];
-        if (ms == -INFINITY) continue;
-        const float w = expf(ms - M);
-        num = fmaf(w, po[(size_t)s * kAH * kAD + i], num);
-        den = fmaf(w, pml[((size_t)s * kAH + h) * 2 + 1], den);
-      }
+  float M = -INFINITY;
+  for (int s = 0; s < nseg; ++s) M = fmaxf(M, __ldg(pml + ((size_t)s * kAH + h) * 2));
+  float num = 0.f, den = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < nseg; ++s) {
+      const float ms = __ldg(pml + ((size_t)s * kAH + h) * 2);
+      if (ms == -INFINITY) continue;
+      const float w = expf(ms - M);
+      num = fmaf(w, __ldg(po + ((size_t)s * kAH + h) * kAD + d), num);
+      den = fmaf(w, __ldg(pml + ((size_t)s * kAH + h) * 2 + 1), den);
     }
-    o[i] = den > 0.f ? num / den : 0.f;
   }
+  out[((size_t)b * kAH + h) * kAD + d] = den > 0.f ? num / den : 0.f;
 }
 
 // hidden'[b] = RMSNorm(hidden[b] + o[b]) (eps, no gain); one CTA per row.
@@ -271,7 +285,7 @@ extern "C" fm_status fm_decode_attention(const float* q, const uint8_t* mem, int
   }
   sparse_attn_partial_kernel<<<dim3(nseg, B), kAThreads, sizeof(AttnSmem), stream>>>(
       q, mem, row_stride_bytes, n_mem, idx, count, max_sel, nseg, part_o, part_ml);
-  sparse_attn_combine_kernel<<<B, kAThreads, 0, stream>>>(part_o, part_ml, nseg, out);
+  sparse_attn_combine_kernel<<<dim3(kAH, B), kAD, 0, stream>>>(part_o, part_ml, nseg, out);
   note_launch();
   note_launch();
   return check_launch();
