@@ -175,35 +175,58 @@ __global__ void split_tf32_kernel(const float* __restrict__ x, float* __restrict
 }
 
 // ------------------------------------------------ tensor-core skinny GEMM
-// part[s][n][m] = sum over K split s of W[m][k] X[n][k] at fp32-level accuracy
-// on the tensor cores: each operand is split as hi = tf32(v), lo = v - hi and
-// the product is taken as hi*hi + hi*lo + lo*hi (three TF32 MMAs, fp32
-// accumulation in TMEM).  X (a few hundred KB) arrives already split; W, the
-// bulk of the bytes, streams in as fp32 once and is split inside the CTA:
+// part[s][n][m] = W[m][:] . X[n][:] over one stretch of K, at fp32-level
+// accuracy on the tensor cores: each operand is split as hi = tf32(v),
+// lo = v - hi and the product is taken as hi*hi + hi*lo + lo*hi (TF32 MMAs,
+// fp32 accumulation in TMEM).  X (a few hundred KB) arrives already split; W,
+// the bulk of the bytes, streams in as fp32 once and is split in the CTA.
 //
-//   warp 0 lane 0   TMA producer: per stage the fp32 W tile (128 rows x 32)
-//                   and the X hi / lo tiles (BN rows x 32), 128B-swizzled
-//   warps 4..7      split: thread t reads row t of the W tile, writes its hi
-//                   and lo parts into the stage's TMEM columns (the MMA's A
-//                   operand), then reads out the accumulator at the end
-//   warp 1 lane 0   MMA issuer: A from TMEM, B (X hi / lo) from shared memory
+// Stream-K: the (tile, 32-wide K block) units of the whole product, tiles
+// being 128 rows of W x BN rows of X, are dealt out in equal contiguous
+// ranges to one persistent CTA per SM, so no CTA waits on a wave tail and the
+// pipeline runs across tile boundaries.  A CTA's run of units inside one tile
+// is a segment; its partial goes to slot (CTA - first CTA of the tile), and
+// the consumer sums the tile's StreamK::slots partials (a fixed order:
+// deterministic).
 //
-// A stage's TMEM columns are reused only after its shared-memory stage was
-// refilled, which waits for the MMAs of the previous use to retire.  One CTA
-// per (128 rows of W, K split, BN columns of X).
-constexpr int kTcThreads = 256;
-constexpr int kTcBM = 128;                              // rows of W per CTA (MMA M)
-constexpr int kTcBK = 32;                               // K per stage: 32 fp32 = one 128-byte row
+//   warp 0 lane 0   TMA producer: per unit the fp32 W tile (128 x 32) and the
+//                   X hi / lo tiles (BN x 32 each, adjacent), 128B-swizzled
+//   warps 4..7      split: thread t reads row t of the W tile and writes its
+//                   hi and lo parts into the stage's TMEM columns (A operand)
+//   warp 1 lane 0   MMA issuer: A from TMEM, B from shared memory:
+//                   hi x [Xhi; Xlo] (N = 2 BN) + lo x Xhi (N = BN)
+//   warps 8..11     epilogue: per segment, accumulator halves summed
+//                   (hi.Xhi + lo.Xhi | hi.Xlo) and stored to the slot
+//
+// TMEM: the accumulator buffer(s) of 2 BN columns, then 64 columns (hi, lo) per
+// stage.  A stage's TMEM columns are rewritten only after its shared-memory
+// stage was refilled, which waits for the MMAs of the previous use to retire.
+constexpr int kTcThreads = 384;
+constexpr int kTcBM = 128;                              // rows of W per tile (MMA M)
+constexpr int kTcBK = 32;                               // K per unit: 32 fp32 = one 128-byte row
 constexpr uint32_t kTcWTile = kTcBM * kTcBK * 4;        // 16 KB
 constexpr int kTcSplitWarp0 = 4;                        // warps 4..7: TMEM lane quarters 0..3
+constexpr int kTcEpiWarp0 = 8;                          // warps 8..11
+
+struct StreamK {
+  int KB;       // K blocks per tile
+  int mtiles;   // tiles along M; tile t = ntile * mtiles + mtile
+  int bn;       // X rows per tile
+  int G;        // CTAs
+  int64_t U;    // units = tiles * KB
+  __host__ __device__ int64_t start(int c) const { return U * c / G; }
+  __host__ __device__ int cta_of(int64_t u) const { return (int)(((int64_t)G * (u + 1) - 1) / U); }
+  __host__ __device__ int first_cta(int t) const { return cta_of((int64_t)t * KB); }
+  __host__ __device__ int slots(int t) const { return cta_of((int64_t)t * KB + KB - 1) - first_cta(t) + 1; }
+};
 
 struct TcGemmArgs {
-  int M, N, K;          // W [M, K]; X [N, K] (one layer of it); part [split][N][M]
-  int kb_per_split;     // K blocks of 32 per split (every split has exactly this many)
+  int M, N, K;          // W [M, K]; X [N, K] (one layer of it); part [slot][N][M]
   int rows_per_layer;   // W rows per X layer (the up projection); 0: X has one layer
   float* part;
   int64_t split_stride;
   int* err;
+  StreamK sk;
 };
 
 __host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
@@ -226,30 +249,34 @@ __device__ __forceinline__ void umma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, u
 }
 
 template <int BN>
-constexpr uint32_t tc_stage_bytes() { return kTcWTile + 2u * BN * kTcBK * 4; }
-
-// TMEM: the accumulator in columns [0, BN), then 64 columns (hi, lo) per stage.
-template <int BN>
-constexpr int tc_tmem_stages() { return (512 - BN) / 64; }
+struct TcCfg {
+  static constexpr int kAccBufs = BN <= 64 ? 2 : 1;
+  static constexpr int kAccCols = 2 * BN;
+  static constexpr int kStages = (512 - kAccBufs * kAccCols) / 64;  // TMEM A stages = smem stages
+  static constexpr uint32_t kStageBytes = kTcWTile + 2u * BN * kTcBK * 4;
+  static constexpr uint32_t kSmem = kStages * kStageBytes + (3 * kStages + 4) * 8 + 16 + 1024;
+};
 
 template <int BN>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap w_map, const __grid_constant__ CUtensorMap x_hi,
-                   const __grid_constant__ CUtensorMap x_lo, TcGemmArgs a, int S) {
+                   const __grid_constant__ CUtensorMap x_lo, TcGemmArgs a) {
+  using C = TcCfg<BN>;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   constexpr uint32_t kXTile = BN * kTcBK * 4;
-  constexpr uint32_t kStage = tc_stage_bytes<BN>();
+  constexpr uint32_t kStage = C::kStageBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * kStage);
   uint64_t* split = full + S;
   uint64_t* empty = split + S;
-  uint64_t* done = empty + S;
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* acc_full = empty + S;    // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kTcBM, n0 = blockIdx.z * BN;
-  const int kb0 = blockIdx.y * a.kb_per_split, nkb = a.kb_per_split;
-  const int layer = a.rows_per_layer ? m0 / a.rows_per_layer : 0;
+  const StreamK& sk = a.sk;
+  const int64_t u0 = sk.start(blockIdx.x), u1 = sk.start(blockIdx.x + 1);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -257,7 +284,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&split[i], 4);  // one arrival per split warp
       mbar_init(&empty[i], 1);
     }
-    mbar_init(done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);  // one arrival per epilogue warp
+    }
     *sAbort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -269,14 +299,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sTmem;
+  const uint32_t a_col0 = (uint32_t)(C::kAccBufs * C::kAccCols);
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
     uint32_t stage = 0, phase = 0, issued = 0;
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int64_t u = u0; u < u1; ++u) {
       if (!mbar_wait_bounded(&empty[stage], phase ^ 1, sAbort, a.err)) break;
+      const int t = (int)(u / sk.KB), kb = (int)(u - (int64_t)t * sk.KB);
+      const int m0 = (t % sk.mtiles) * kTcBM, n0 = (t / sk.mtiles) * BN;
+      const int layer = a.rows_per_layer ? m0 / a.rows_per_layer : 0;
+      const int k = kb * kTcBK;
       uint8_t* st = smem + (size_t)stage * kStage;
-      const int k = (kb0 + kb) * kTcBK;
       mbar_arrive_expect_tx(&full[stage], kStage);
       tma_load_2d(st, &w_map, k, m0, &full[stage]);
       tma_load_3d(st + kTcWTile, &x_hi, k, layer, n0, &full[stage]);
@@ -292,34 +326,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = idesc_tf32_f32(kTcBM, BN);
-    uint32_t stage = 0, phase = 0;
-    for (int kb = 0; kb < nkb; ++kb) {
-      if (!mbar_wait_bounded(&split[stage], phase, sAbort, a.err)) break;
+    constexpr uint32_t idesc2 = idesc_tf32_f32(kTcBM, 2 * BN), idesc1 = idesc_tf32_f32(kTcBM, BN);
+    uint32_t stage = 0, phase = 0, buf = 0;
+    uint32_t par = 0;  // bit b: parity of accumulator buffer b's uses
+    bool ok = true;
+    for (int64_t u = u0; u < u1 && ok;) {
+      const int t = (int)(u / sk.KB);
+      const int64_t seg_end = min(u1, (int64_t)(t + 1) * sk.KB);
+      if (!mbar_wait_bounded(&acc_empty[buf], ((par >> buf) & 1u) ^ 1u, sAbort, a.err)) break;
       tc_fence_after();
-      const uint32_t base = smem_u32(smem + (size_t)stage * kStage);
-      const uint64_t dxh = sdesc_kmajor_sw128(base + kTcWTile);
-      const uint64_t dxl = sdesc_kmajor_sw128(base + kTcWTile + kXTile);
-      const uint32_t a_hi = tmem + (uint32_t)BN + stage * 64u, a_lo = a_hi + 32u;
+      const uint32_t d = tmem + buf * (uint32_t)C::kAccCols;
+      for (bool first = true; u < seg_end; ++u, first = false) {
+        if (!mbar_wait_bounded(&split[stage], phase, sAbort, a.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t base = smem_u32(smem + (size_t)stage * kStage);
+        const uint64_t dx = sdesc_kmajor_sw128(base + kTcWTile);  // [Xhi; Xlo]: 2 BN rows
+        const uint32_t a_hi = tmem + a_col0 + stage * 64u, a_lo = a_hi + 32u;
 #pragma unroll
-      for (int k = 0; k < kTcBK / 8; ++k) {  // K = 8 tf32 per MMA: 8 TMEM columns, 32 smem bytes
-        const uint64_t o = 2u * (uint32_t)k;  // +32 bytes in the 16-byte address field
-        const uint32_t c = 8u * (uint32_t)k;
-        umma_tf32_ts(tmem, a_hi + c, dxh + o, idesc, (kb > 0 || k > 0) ? 1u : 0u);
-        umma_tf32_ts(tmem, a_hi + c, dxl + o, idesc, 1u);
-        umma_tf32_ts(tmem, a_lo + c, dxh + o, idesc, 1u);
+        for (int k = 0; k < kTcBK / 8; ++k) {  // K = 8 tf32 per MMA: 8 TMEM columns, 32 smem bytes
+          const uint64_t o = 2u * (uint32_t)k;  // +32 bytes in the 16-byte address field
+          const uint32_t c = 8u * (uint32_t)k;
+          umma_tf32_ts(d, a_hi + c, dx + o, idesc2, (first && k == 0) ? 0u : 1u);
+          umma_tf32_ts(d, a_lo + c, dx + o, idesc1, 1u);
+        }
+        umma_commit(&empty[stage]);  // the stage may be refilled once these MMAs retire
+        if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
       }
-      umma_commit(&empty[stage]);  // the stage may be refilled once these MMAs retire
-      if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
+      if (!ok) break;
+      umma_commit(&acc_full[buf]);
+      par ^= 1u << buf;
+      if (C::kAccBufs == 2) buf ^= 1u;
     }
-    umma_commit(done);
-  } else if (warp >= kTcSplitWarp0) {
+  } else if (warp >= kTcSplitWarp0 && warp < kTcEpiWarp0) {
     // --------------------------------------------------------------- split
     const int q = warp - kTcSplitWarp0;  // TMEM lane quarter
     const int r = q * 32 + lane;         // row of the W tile
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     uint32_t stage = 0, phase = 0;
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int64_t u = u0; u < u1; ++u) {
       // every lane waits (each needs the TMA data visible); the warp leaves
       // together if any lane's wait ran out, before the .aligned TMEM stores
       const bool ok = mbar_wait_bounded(&full[stage], phase, sAbort, a.err);
@@ -339,7 +383,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           lo[4 * c + i] = __float_as_uint(e[i] - h);
         }
       }
-      const uint32_t col = (uint32_t)BN + stage * 64u;
+      const uint32_t col = a_col0 + stage * 64u;
       tmem_st32_wait(lane_base + col, hi);
       tmem_st32_wait(lane_base + col + 32u, lo);
       tc_fence_before();
@@ -347,26 +391,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) mbar_arrive(&split[stage]);
       if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
     }
-    // ---------------------------------------------------------- epilogue
-    int good = 1;
-    if (lane == 0) good = mbar_wait_bounded(done, 0, sAbort, a.err) && !*sAbort;
-    good = __shfl_sync(0xffffffffu, good, 0);
-    tc_fence_after();
-    if (good) {
-      const int m = m0 + r;
-      float* out = a.part + (int64_t)blockIdx.y * a.split_stride;
+  } else if (warp >= kTcEpiWarp0) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp - kTcEpiWarp0;
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    uint32_t buf = 0;
+    uint32_t par = 0;  // bit b: parity of accumulator buffer b's uses
+    for (int64_t u = u0; u < u1;) {
+      const int t = (int)(u / sk.KB);
+      u = min(u1, (int64_t)(t + 1) * sk.KB);
+      int good = 1;
+      if (lane == 0) good = mbar_wait_bounded(&acc_full[buf], (par >> buf) & 1u, sAbort, a.err);
+      good = __shfl_sync(0xffffffffu, good, 0);
+      if (!good) break;
+      tc_fence_after();
+      const int m = (t % sk.mtiles) * kTcBM + q * 32 + lane, n0 = (t / sk.mtiles) * BN;
+      float* out = a.part + (int64_t)((int)blockIdx.x - sk.first_cta(t)) * a.split_stride;
+      const uint32_t dcol = buf * (uint32_t)C::kAccCols;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32_wait(lane_base + (uint32_t)c0, v);
+        uint32_t v[32], w[32];
+        tmem_ld32_wait(lane_base + dcol + (uint32_t)c0, v);        // hi.Xhi + lo.Xhi
+        tmem_ld32_wait(lane_base + dcol + (uint32_t)(BN + c0), w);  // hi.Xlo
         if (m < a.M) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int n = n0 + c0 + j;
-            if (n < a.N) out[(int64_t)n * a.M + m] = __uint_as_float(v[j]);
+            if (n < a.N) out[(int64_t)n * a.M + m] = __uint_as_float(v[j]) + __uint_as_float(w[j]);
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      par ^= 1u << buf;
+      if (C::kAccBufs == 2) buf ^= 1u;
     }
   }
   tc_fence_before();
@@ -379,7 +438,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // The up projection's K-split partials summed, then RoPE and the Hadamard:
 // one warp per (row, layer, head).
-__global__ void __launch_bounds__(kThreads) qup_finish_kernel(const float* __restrict__ part, int ksplit,
+__global__ void __launch_bounds__(kThreads) qup_finish_kernel(const float* __restrict__ part, StreamK sk,
                                                               int64_t split_stride, int B, int L,
                                                               const float* __restrict__ rope_cs,
                                                               float* __restrict__ q);
@@ -387,7 +446,7 @@ __global__ void __launch_bounds__(kThreads) qup_finish_kernel(const float* __res
 // One CTA per (row b, layer l): reduce the K splits, RMSNorm the wq_a part,
 // scale the weights_proj part into fused_w, and (layer 0) the RoPE table.
 __global__ void __launch_bounds__(kThreads) qnorm_kernel(
-    const float* __restrict__ a_part, int ksplit, int B, int L, int R, int H,
+    const float* __restrict__ a_part, int ksplit, StreamK sk, int B, int L, int R, int H,
     const float* __restrict__ q_norm, float eps, float w_scale, const int64_t* __restrict__ positions,
     const double* __restrict__ rope_freq, int rope_half, float* __restrict__ r_norm,
     float* __restrict__ fused_w, float* __restrict__ rope_cs, float* __restrict__ r_hi,
@@ -395,11 +454,26 @@ __global__ void __launch_bounds__(kThreads) qnorm_kernel(
   const int b = blockIdx.x, l = blockIdx.y;
   const int M = L * (R + H);
   const float* base = a_part + (size_t)b * M + (size_t)l * (R + H);
+  // partials of element i: ksplit (K splits), or its tile's stream-K slots,
+  // looked up per tile from a table built once
+  constexpr int kMaxTiles = 64;  // tiles in the table; a (row, layer) block spans (R + H) / 128 + 2
+  __shared__ int s_slots[kMaxTiles];
+  const int t0 = (l * (R + H)) / kTcBM;
+  if (ksplit <= 0)
+    for (int j = threadIdx.x; j < kMaxTiles; j += kThreads)
+      s_slots[j] = sk.slots((b / sk.bn) * sk.mtiles + t0 + j);
+  __syncthreads();
+  auto nparts = [&](int i) {
+    if (ksplit > 0) return ksplit;
+    const int j = (l * (R + H) + i) / kTcBM - t0;
+    return j < kMaxTiles ? s_slots[j] : sk.slots((b / sk.bn) * sk.mtiles + t0 + j);
+  };
   __shared__ float red[kThreads / 32];
   float ss = 0.f;
   for (int i = threadIdx.x; i < R; i += kThreads) {
     float a = 0.f;
-    for (int s = 0; s < ksplit; ++s) a += base[(size_t)s * B * M + i];
+    const int np = nparts(i);
+    for (int s = 0; s < np; ++s) a += base[(size_t)s * B * M + i];
     ss = fmaf(a, a, ss);
   }
 #pragma unroll
@@ -412,7 +486,8 @@ __global__ void __launch_bounds__(kThreads) qnorm_kernel(
   const float inv_rms = 1.0f / sqrtf(tot / (float)R + eps);
   for (int i = threadIdx.x; i < R; i += kThreads) {
     float a = 0.f;
-    for (int s = 0; s < ksplit; ++s) a += base[(size_t)s * B * M + i];
+    const int np = nparts(i);
+    for (int s = 0; s < np; ++s) a += base[(size_t)s * B * M + i];
     const float r = a * inv_rms * q_norm[(size_t)l * R + i];
     r_norm[((size_t)b * L + l) * R + i] = r;
     if (r_hi) {  // the split operand of the tensor-core up projection
@@ -423,7 +498,8 @@ __global__ void __launch_bounds__(kThreads) qnorm_kernel(
   }
   for (int h = threadIdx.x; h < H; h += kThreads) {
     float a = 0.f;
-    for (int s = 0; s < ksplit; ++s) a += base[(size_t)s * B * M + R + h];
+    const int np = nparts(R + h);
+    for (int s = 0; s < np; ++s) a += base[(size_t)s * B * M + R + h];
     fused_w[((size_t)b * L + l) * H + h] = a * w_scale;
   }
   if (l == 0 && threadIdx.x < rope_half) {
@@ -475,7 +551,7 @@ __device__ __forceinline__ void rope_wht_store(float x[4], int b, int l, int h, 
       make_float4(x[0] * inv_sqrt_d, x[1] * inv_sqrt_d, x[2] * inv_sqrt_d, x[3] * inv_sqrt_d);
 }
 
-__global__ void __launch_bounds__(kThreads) qup_finish_kernel(const float* __restrict__ part, int ksplit,
+__global__ void __launch_bounds__(kThreads) qup_finish_kernel(const float* __restrict__ part, StreamK sk,
                                                               int64_t split_stride, int B, int L,
                                                               const float* __restrict__ rope_cs,
                                                               float* __restrict__ q) {
@@ -484,8 +560,10 @@ __global__ void __launch_bounds__(kThreads) qup_finish_kernel(const float* __res
   const int lane = threadIdx.x & 31;
   const int h = idx % kHeads, bl = idx / kHeads, l = bl % L, b = bl / L;
   const float* src = part + (size_t)b * L * kHeads * kHeadDim + ((size_t)l * kHeads + h) * kHeadDim + lane * 4;
+  // one head's 128 rows of wq_b are one tile: its partials are the tile's slots
+  const int nslots = sk.slots((b / sk.bn) * sk.mtiles + l * kHeads + h);
   float4 acc = __ldg(reinterpret_cast<const float4*>(src));
-  for (int s = 1; s < ksplit; ++s) {
+  for (int s = 1; s < nslots; ++s) {
     const float4 v = __ldg(reinterpret_cast<const float4*>(src + (int64_t)s * split_stride));
     acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
   }
@@ -673,46 +751,62 @@ void launch_split(const float* x, float* hi, float* lo, int64_t n, cudaStream_t 
 
 template <int BN>
 fm_status launch_tc_gemm_bn(fm_ctx* ctx, const void* wmap, const void* xh, const void* xl, const TcGemmArgs& a,
-                            int mtiles, int ksplit, int ntiles, cudaStream_t st) {
+                            cudaStream_t st) {
   static int configured_dev = -1;
-  constexpr uint32_t stage = tc_stage_bytes<BN>();
-  int S = (int)((200u * 1024u) / stage);
-  S = S < 2 ? 2 : S;
-  if (S > tc_tmem_stages<BN>()) S = tc_tmem_stages<BN>();
-  const uint32_t smem = (uint32_t)S * stage + (uint32_t)(3 * S + 1) * 8 + 16 + 1024;
+  constexpr uint32_t smem = TcCfg<BN>::kSmem;
+  static_assert(smem <= 227u * 1024u, "shared memory");
   if (configured_dev != ctx->device) {
-    if (cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+    if (cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return check_launch();
     configured_dev = ctx->device;
   }
-  tc_gemm_kernel<BN><<<dim3(mtiles, ksplit, ntiles), kTcThreads, smem, st>>>(
-      *reinterpret_cast<const CUtensorMap*>(wmap), *reinterpret_cast<const CUtensorMap*>(xh),
-      *reinterpret_cast<const CUtensorMap*>(xl), a, S);
+  tc_gemm_kernel<BN><<<a.sk.G, kTcThreads, smem, st>>>(*reinterpret_cast<const CUtensorMap*>(wmap),
+                                                       *reinterpret_cast<const CUtensorMap*>(xh),
+                                                       *reinterpret_cast<const CUtensorMap*>(xl), a);
   note_launch();
   return check_launch();
 }
 
-// part[s][n][m] for W (fp32 map: [M, K]) against X (split maps) in K splits.
+// The stream-K partition of an M x N product over K for at most `G` CTAs,
+// with no tile split over more than `max_slots` CTAs.
+StreamK make_stream_k(int M, int N, int K, int bn, int G, int max_slots) {
+  StreamK sk;
+  sk.KB = K / kTcBK;
+  sk.mtiles = (M + kTcBM - 1) / kTcBM;
+  sk.bn = bn;
+  const int tiles = sk.mtiles * ((N + bn - 1) / bn);
+  sk.U = (int64_t)tiles * sk.KB;
+  sk.G = (int)(sk.U < G ? sk.U : G);
+  for (;;) {
+    int worst = 0;
+    for (int t = 0; t < tiles; ++t) worst = worst > sk.slots(t) ? worst : sk.slots(t);
+    if (worst <= max_slots || sk.G == 1) break;
+    --sk.G;
+  }
+  return sk;
+}
+
+// part[slot][n][m] for W (fp32 map: [M, K]) against X (split maps), stream-K.
 fm_status launch_tc_gemm(fm_ctx* ctx, const void* wmap, const float* x_hi, const float* x_lo, int x_layers,
-                         int M, int N, int K, int ksplit, int rows_per_layer, float* part, cudaStream_t st) {
-  const int bn = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+                         int M, int N, int K, int max_slots, int rows_per_layer, float* part, StreamK* sk_out,
+                         cudaStream_t st) {
+  const int bn = N <= 32 ? 32 : N <= 64 ? 64 : 128;
   alignas(64) unsigned char xh[128], xl[128];
   if (!encode_act_map(xh, x_hi, N, x_layers, K, bn) || !encode_act_map(xl, x_lo, N, x_layers, K, bn))
     return FM_ERR_CUDA;
   TcGemmArgs a;
   a.M = M; a.N = N; a.K = K;
-  a.kb_per_split = K / kTcBK / ksplit;
   a.rows_per_layer = rows_per_layer;
   a.part = part;
   a.split_stride = (int64_t)N * M;
   a.err = ctx->d_err;
-  const int mtiles = (M + kTcBM - 1) / kTcBM, ntiles = (N + bn - 1) / bn;
+  a.sk = make_stream_k(M, N, K, bn, ctx->num_sms, max_slots);
+  *sk_out = a.sk;
   switch (bn) {
-    case 32: return launch_tc_gemm_bn<32>(ctx, wmap, xh, xl, a, mtiles, ksplit, ntiles, st);
-    case 64: return launch_tc_gemm_bn<64>(ctx, wmap, xh, xl, a, mtiles, ksplit, ntiles, st);
-    case 128: return launch_tc_gemm_bn<128>(ctx, wmap, xh, xl, a, mtiles, ksplit, ntiles, st);
-    default: return launch_tc_gemm_bn<256>(ctx, wmap, xh, xl, a, mtiles, ksplit, ntiles, st);
+    case 32: return launch_tc_gemm_bn<32>(ctx, wmap, xh, xl, a, st);
+    case 64: return launch_tc_gemm_bn<64>(ctx, wmap, xh, xl, a, st);
+    default: return launch_tc_gemm_bn<128>(ctx, wmap, xh, xl, a, st);
   }
 }
 
@@ -722,29 +816,24 @@ fm_status launch_query_prep_tc(fm_ctx* ctx, const float* hidden, const int64_t* 
   const fm_config& c = ctx->cfg;
   const int L = c.n_layers, R = c.q_lora_rank, HID = c.hidden;
   const int Md = L * (R + kHeads), Mu = L * kHeads * kHeadDim;
-  const int bn_tiles = (B + 255) / 256;
-  // down projection: K splits until every SM has a CTA (splits divide K/32)
-  const int mtiles_d = (Md + kTcBM - 1) / kTcBM;
-  int ks_d = 1;
-  while (ks_d * 2 <= ctx->splitk_max && (HID / kTcBK) % (ks_d * 2) == 0 && mtiles_d * bn_tiles * ks_d < ctx->num_sms)
-    ks_d *= 2;
+  // down projection (stream-K; its partials buffer holds splitk_max slots)
   launch_split(hidden, ctx->x_hi, ctx->x_lo, (int64_t)B * HID, st);
-  fm_status s = launch_tc_gemm(ctx, ctx->wmaps[0], ctx->x_hi, ctx->x_lo, 1, Md, B, HID, ks_d, 0,
-                               ctx->a_part, st);
+  StreamK sk_d, sk_u;
+  fm_status s = launch_tc_gemm(ctx, ctx->wmaps[0], ctx->x_hi, ctx->x_lo, 1, Md, B, HID, ctx->splitk_max, 0,
+                               ctx->a_part, &sk_d, st);
   if (s != FM_OK) return s;
   const float w_scale = (float)(1.0 / sqrt((double)c.head_dim * (double)c.n_heads));
-  qnorm_kernel<<<dim3(B, L), kThreads, 0, st>>>(ctx->a_part, ks_d, B, L, R, c.n_heads, ctx->q_norm, c.rms_eps,
-                                                 w_scale, positions, ctx->rope_freq, c.rope_dim / 2,
+  qnorm_kernel<<<dim3(B, L), kThreads, 0, st>>>(ctx->a_part, 0, sk_d, B, L, R, c.n_heads, ctx->q_norm,
+                                                 c.rms_eps, w_scale, positions, ctx->rope_freq, c.rope_dim / 2,
                                                  ctx->r_norm, fused_w, ctx->rope_cs, ctx->r_hi, ctx->r_lo);
   note_launch();
-  // up projection: two K splits (its partials buffer holds two)
-  const int ks_u = (R / kTcBK) % 2 == 0 ? 2 : 1;
-  s = launch_tc_gemm(ctx, ctx->wmaps[1], ctx->r_hi, ctx->r_lo, L, Mu, B, R, ks_u,
-                     kHeads * kHeadDim, ctx->up_part, st);
+  // up projection (stream-K; its partials buffer holds two slots)
+  s = launch_tc_gemm(ctx, ctx->wmaps[1], ctx->r_hi, ctx->r_lo, L, Mu, B, R, 2, kHeads * kHeadDim, ctx->up_part,
+                     &sk_u, st);
   if (s != FM_OK) return s;
   const int warps = B * L * kHeads;
   qup_finish_kernel<<<(warps + kThreads / 32 - 1) / (kThreads / 32), kThreads, 0, st>>>(
-      ctx->up_part, ks_u, (int64_t)B * Mu, B, L, ctx->rope_cs, q);
+      ctx->up_part, sk_u, (int64_t)B * Mu, B, L, ctx->rope_cs, q);
   note_launch();
   return check_launch();
 }
@@ -786,7 +875,7 @@ fm_status launch_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* pos
 
   const float w_scale = (float)(1.0 / sqrt((double)c.head_dim * (double)c.n_heads));
   qnorm_kernel<<<dim3(B, c.n_layers), kThreads, 0, st>>>(
-      ctx->a_part, ksplit, B, c.n_layers, c.q_lora_rank, c.n_heads, ctx->q_norm, c.rms_eps,
+      ctx->a_part, ksplit, StreamK{}, B, c.n_layers, c.q_lora_rank, c.n_heads, ctx->q_norm, c.rms_eps,
       w_scale, positions, ctx->rope_freq, c.rope_dim / 2, ctx->r_norm, fused_w, ctx->rope_cs, nullptr,
       nullptr);
   note_launch();
