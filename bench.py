@@ -223,19 +223,23 @@ def run_ours(args, rank, world, local_rank):
     flush = key_bytes < 4 * l2
     flush_buf = torch.empty(max(2 * l2, 1 << 28) // 4, device=dev, dtype=torch.float32) if flush else None
 
-    ev_sc = []
+    ev_sc = []  # per timed step: events before prep, before scoring, after scoring, after top-K
 
     def step(timed=False):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if timed else None
+        if timed:
+            ev[0].record(stream)
         r.fm_query_prep(hidden, positions, q=qb, fused_w=wb)
         if timed:
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
+            ev[1].record(stream)
         r.fm_score_fused(keys, qb, wb, mode=wl.mode, threshold=wl.threshold, n_valid=n_valid, N=N,
                          ens=ens, keep_thr=keep_thr)
         if timed:
-            b.record(stream)
-            ev_sc.append((a, b))
+            ev[2].record(stream)
         fm.fm_select_topk(ens, wl.top_k, n_valid, out=keep, workspace=ws)
+        if timed:
+            ev[3].record(stream)
+            ev_sc.append(ev)
 
     for _ in range(args.warmup):
         step()
@@ -272,7 +276,10 @@ def run_ours(args, rank, world, local_rank):
         barrier()
     launches = fm.fm_launch_count() - launches0
     r.fm_sync_status()
-    score_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_sc]))
+    score_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev_sc]))
+    stages_ms = {"query_prep": round(float(np.mean([e[0].elapsed_time(e[1]) for e in ev_sc])), 4),
+                 "scoring_pass": round(score_ms, 4),
+                 "topk": round(float(np.mean([e[2].elapsed_time(e[3]) for e in ev_sc])), 4)}
 
     elapsed_max = max_over_ranks(elapsed_ms, world, dev)
     ms_per_step = elapsed_max / args.steps
@@ -328,7 +335,7 @@ def run_ours(args, rank, world, local_rank):
     r.close()
     return dict(value=value, ms_per_step=ms_per_step, roofline=roofline, e2e=e2e, cpu=cpu,
                 clocks=sampler.summary(), launches=launches, decisions=decisions, flush=flush,
-                key_bytes=key_bytes)
+                key_bytes=key_bytes, stages_ms=stages_ms)
 
 
 # ------------------------------------------------------------ recall path
@@ -600,6 +607,17 @@ def _oracle_threads():
         return os.cpu_count()
 
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return None
+
+
 def cpu_baseline_sample(inp, keys, wl, q_row=0):
     """The CPU oracle, as it stands, on one row of the workload (all chunks,
     3 layers, query prep, ensemble, top-K)."""
@@ -617,6 +635,7 @@ def cpu_baseline_sample(inp, keys, wl, q_row=0):
     O.select_topk(e, np.array([n]), wl.top_k)
     dt = time.perf_counter() - t0
     return {"value": n / dt, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+            "cpu_model": _cpu_model(), "host_cpus": len(os.sched_getaffinity(0)),
             "sample": f"row {b} of the workload: {n} chunks x 3 layers, query prep, ensemble, "
                       f"top-{wl.top_k} ({dt:.1f} s)"}
 
@@ -712,7 +731,8 @@ def main():
            "dtype": "e4m3",
            "data": "synthetic (seeded generator, random-init weights)",
            "config": config_of(wl, world, res["flush"], res["key_bytes"], args.shared_keys),
-           "roofline": res["roofline"], "e2e": res["e2e"], "gpu_launches": res["launches"],
+           "roofline": res["roofline"], "stages_ms": res["stages_ms"], "e2e": res["e2e"],
+           "gpu_launches": res["launches"],
            "clocks": res["clocks"], "cpu_baseline": res["cpu"]}
     print(json.dumps(out), flush=True)
 
