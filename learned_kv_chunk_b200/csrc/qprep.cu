@@ -469,11 +469,33 @@ __global__ void __launch_bounds__(kThreads) qnorm_kernel(
     return j < kMaxTiles ? s_slots[j] : sk.slots((b / sk.bn) * sk.mtiles + t0 + j);
   };
   __shared__ float red[kThreads / 32];
-  float ss = 0.f;
-  for (int i = threadIdx.x; i < R; i += kThreads) {
-    float a = 0.f;
+  // the split sums of this thread's first kKeep elements stay in registers
+  // for the second loop; the partial loads of one element issue together
+  constexpr int kKeep = 8;
+  auto reduce = [&](int i) {
     const int np = nparts(i);
-    for (int s = 0; s < np; ++s) a += base[(size_t)s * B * M + i];
+    float a = 0.f;
+    if (np <= 16) {
+      float v[16];
+#pragma unroll
+      for (int s = 0; s < 16; ++s) v[s] = s < np ? __ldg(base + (size_t)s * B * M + i) : 0.f;
+#pragma unroll
+      for (int s = 0; s < 16; ++s) a += v[s];
+    } else {
+      for (int s = 0; s < np; ++s) a += base[(size_t)s * B * M + i];
+    }
+    return a;
+  };
+  float kept[kKeep];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < kKeep; ++k) {
+    const int i = threadIdx.x + k * kThreads;
+    kept[k] = i < R ? reduce(i) : 0.f;
+    ss = fmaf(kept[k], kept[k], ss);
+  }
+  for (int i = threadIdx.x + kKeep * kThreads; i < R; i += kThreads) {
+    const float a = reduce(i);
     ss = fmaf(a, a, ss);
   }
 #pragma unroll
@@ -484,10 +506,7 @@ __global__ void __launch_bounds__(kThreads) qnorm_kernel(
 #pragma unroll
   for (int w = 0; w < kThreads / 32; ++w) tot += red[w];
   const float inv_rms = 1.0f / sqrtf(tot / (float)R + eps);
-  for (int i = threadIdx.x; i < R; i += kThreads) {
-    float a = 0.f;
-    const int np = nparts(i);
-    for (int s = 0; s < np; ++s) a += base[(size_t)s * B * M + i];
+  auto emit = [&](int i, float a) {
     const float r = a * inv_rms * q_norm[(size_t)l * R + i];
     r_norm[((size_t)b * L + l) * R + i] = r;
     if (r_hi) {  // the split operand of the tensor-core up projection
@@ -495,11 +514,15 @@ __global__ void __launch_bounds__(kThreads) qnorm_kernel(
       r_hi[((size_t)b * L + l) * R + i] = hi;
       r_lo[((size_t)b * L + l) * R + i] = r - hi;
     }
+  };
+#pragma unroll
+  for (int k = 0; k < kKeep; ++k) {
+    const int i = threadIdx.x + k * kThreads;
+    if (i < R) emit(i, kept[k]);
   }
+  for (int i = threadIdx.x + kKeep * kThreads; i < R; i += kThreads) emit(i, reduce(i));
   for (int h = threadIdx.x; h < H; h += kThreads) {
-    float a = 0.f;
-    const int np = nparts(R + h);
-    for (int s = 0; s < np; ++s) a += base[(size_t)s * B * M + R + h];
+    const float a = reduce(R + h);
     fused_w[((size_t)b * L + l) * H + h] = a * w_scale;
   }
   if (l == 0 && threadIdx.x < rope_half) {
