@@ -248,6 +248,30 @@ __device__ __forceinline__ void umma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
+// Two 32-lane x 32-column TMEM stores (thread i writes lane base+i of each),
+// then one wait that covers both.
+__device__ __forceinline__ void tmem_st32x2_wait(uint32_t taddr0, const uint32_t* v, uint32_t taddr1,
+                                                 const uint32_t* w) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%33], "
+      "{%34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, "
+      "%50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr0),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+      "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+      "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31]),
+      "r"(taddr1),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15]),
+      "r"(w[16]), "r"(w[17]), "r"(w[18]), "r"(w[19]), "r"(w[20]), "r"(w[21]), "r"(w[22]), "r"(w[23]),
+      "r"(w[24]), "r"(w[25]), "r"(w[26]), "r"(w[27]), "r"(w[28]), "r"(w[29]), "r"(w[30]), "r"(w[31])
+      : "memory");
+}
+
 template <int BN>
 struct TcCfg {
   static constexpr int kAccBufs = BN <= 64 ? 2 : 1;
@@ -384,8 +408,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       const uint32_t col = a_col0 + stage * 64u;
-      tmem_st32_wait(lane_base + col, hi);
-      tmem_st32_wait(lane_base + col + 32u, lo);
+      tmem_st32x2_wait(lane_base + col, hi, lane_base + col + 32u, lo);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&split[stage]);
