@@ -108,3 +108,22 @@ def test_host_side_argument_rejection(lib):
     out = P(0x1234)
     assert lib.fm_create(None, None, 0, ctypes.byref(out)) == INVALID
     assert out.value is None
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/fm.h is a C ABI: it compiles as strict C99 (and as C++), with
+    every declared type usable from C."""
+    import shutil
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_fm.c"
+    src.write_text('#include "fm.h"\n'
+                   "int main(void) {\n"
+                   "  fm_config c; fm_config_default(&c);\n"
+                   "  fm_layer_weights w; fm_level2_desc d; (void)w; (void)d;\n"
+                   "  return (int)(fm_topk_workspace_bytes(1, 10) == 0) + (int)FM_TOPK_SHARD_BINS * 0;\n"
+                   "}\n")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
+                        "-I", os.path.dirname(HEADER), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
