@@ -112,3 +112,32 @@ def test_level2_rejects_bad_descriptors():
                           torch.zeros(9, dtype=torch.int32, device=DEV), k=8)  # B > max_batch
     finally:
         r.close()
+
+
+def test_level2_ties_take_the_lowest_slots():
+    """Identical resident records give identical scores: the top-k must keep
+    the first k slots of each row (ties to the lower slot), and a row with
+    fewer resident chunks than k keeps them all."""
+    weights = G.make_weights(779, 3)
+    r = fm.Retriever(weights, device=0, max_batch=8, q_pieces=2)
+    try:
+        B, R, k = 3, 1024, 100
+        rec = G.make_keys(80, [1], 4, 3, None)  # one record per layer
+        res_keys = [t[:, :1].expand(B, R, 132).contiguous().to(DEV) for t in rec]
+        ids = (torch.arange(R, dtype=torch.int32) * 7 + 3).repeat(B, 1).contiguous().to(DEV)
+        count = torch.tensor([R, 1000, 60], dtype=torch.int32, device=DEV)
+        step = fm.Level2Step(r, res_keys, ids, count, k=k)
+        step.hidden.copy_(G.make_hidden(81, B).to(DEV))
+        step.positions.copy_(torch.full((B,), 4096, dtype=torch.int64, device=DEV))
+        step.launch()
+        torch.cuda.synchronize()
+        out = step.out_ids.cpu().numpy()
+        idh = ids.cpu().numpy()
+        np.testing.assert_array_equal(out[0], idh[0, :k])
+        np.testing.assert_array_equal(out[1], idh[1, :k])
+        np.testing.assert_array_equal(out[2, :60], idh[2, :60])
+        assert (out[2, 60:] == -1).all()
+        np.testing.assert_array_equal(step.out_count.cpu().numpy(), [k, k, 60])
+        step.close()
+    finally:
+        r.close()
