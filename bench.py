@@ -215,7 +215,7 @@ def run_ours(args, rank, world, local_rank):
     ens = torch.empty(B, N, device=dev, dtype=torch.float32)
     keep = torch.empty(B, N, device=dev, dtype=torch.bool)
     keep_thr = torch.empty(B, N, device=dev, dtype=torch.bool) if wl.threshold is not None else None
-    ws = torch.empty(fm.fm_topk_workspace_bytes(B, N), device=dev, dtype=torch.uint8)
+    ws = torch.empty(fm.fm_topk_workspace_bytes_fast(B, N), device=dev, dtype=torch.uint8)
     qb = torch.empty(B, L, 64, 128, device=dev)
     wb = torch.empty(B, L, 64, device=dev)
     stream = torch.cuda.current_stream()

@@ -169,14 +169,25 @@ fm_status fm_score_fused(fm_ctx* ctx, const uint8_t* const* comp_k, int64_t row_
 /* Bytes of device workspace fm_select_topk needs for B rows of N chunks. */
 size_t fm_topk_workspace_bytes(int B, int N);
 
+/* Bytes of workspace with which fm_select_topk can take its candidate path:
+ * a threshold from a sample of each row, one pass that lists the scores above
+ * it, and the selection among those in shared memory, instead of three
+ * histogram passes and a mask pass over all scores.  The mask is the same
+ * (exact) either way; rows the candidate path cannot finish (too few or too
+ * many candidates, or the K-th value tied with values not kept) go through
+ * the histogram passes.  Taken when the workspace given is at least this
+ * large and 2k + 1024 <= min(16384, max(256, N / 16)). */
+size_t fm_topk_workspace_bytes_fast(int B, int N);
+
 /* Top-K keep mask (README "Usage" select_topk(top_k=K); toy loop "top-K"):
  * keep[b,n] = 1 for the min(k, n_b) largest ens[b, 0:n_b], equal scores taken
  * in increasing chunk index; 0 elsewhere.  Scores must be >= 0 (sigmoid
  * outputs); NaN ranks below every number.
  * ens [B, N] fp32 device; n_valid [B] int32 device or NULL; k >= 1;
  * keep [B, N] uint8 device (written);
- * ws device workspace of at least fm_topk_workspace_bytes(B, N) bytes,
- * 16-byte aligned, owned by the caller; its contents on entry do not matter. */
+ * ws device workspace of at least fm_topk_workspace_bytes(B, N) bytes (the
+ * faster candidate path needs fm_topk_workspace_bytes_fast(B, N)), 16-byte
+ * aligned, owned by the caller; its contents on entry do not matter. */
 fm_status fm_select_topk(const float* ens, const int32_t* n_valid, int B, int N, int k,
                          uint8_t* keep, void* ws, size_t ws_bytes, cudaStream_t stream);
 

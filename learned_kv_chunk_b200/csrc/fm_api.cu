@@ -286,6 +286,11 @@ size_t fm_topk_workspace_bytes(int B, int N) {
   return topk_workspace_bytes(B, N);
 }
 
+size_t fm_topk_workspace_bytes_fast(int B, int N) {
+  if (B < 1 || N < 1) return 0;
+  return topk_workspace_bytes_fast(B, N);
+}
+
 fm_status fm_select_topk(const float* ens, const int32_t* n_valid, int B, int N, int k,
                          uint8_t* keep, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (!ens || !keep || !ws || B < 1 || N < 1 || k < 1 || B > 65535) return FM_ERR_INVALID_ARG;

@@ -95,6 +95,9 @@ fm_status launch_ensemble(const float* scores, int L, int B, int N, int mode, fl
 fm_status launch_threshold(const float* ens, const int32_t* n_valid, int B, int N, float thr,
                            uint8_t* keep, cudaStream_t stream);
 size_t topk_workspace_bytes(int B, int N);
+// With the candidate fast path's buffers (launch_topk takes that path when
+// the workspace is this large).
+size_t topk_workspace_bytes_fast(int B, int N);
 fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, int k, uint8_t* keep,
                       void* ws, size_t ws_bytes, cudaStream_t stream);
 size_t compact_workspace_bytes(int B, int N);

@@ -21,6 +21,7 @@
 #include <new>
 
 #include "fm_internal.cuh"
+#include "select_block.cuh"
 
 struct fm_level2 {
   fm_ctx* ctx;
@@ -49,46 +50,8 @@ namespace {
 // then an ordered scan that writes the kept slots' chunk ids in slot order
 // (equal keys taken in increasing slot).  The general top-K (grid-wide passes
 // with a block per 8192 scores) pays six launches of one block per row here.
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = kBlkThreads;
 constexpr int kSelMaxR = 8192;
-
-// Order-preserving key of a score: larger float -> larger key; +0 and -0
-// equal; NaN lowest.
-__device__ __forceinline__ uint32_t sel_key(float x) {
-  if (x != x) return 0u;
-  const uint32_t u = (x == 0.f) ? 0u : __float_as_uint(x);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Block-wide exclusive scan of one int per thread (kSelThreads threads);
-// returns the exclusive prefix and, through *total, the sum.
-__device__ __forceinline__ int sel_scan(int v, int* s_warp, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
-  }
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int x = lane < kSelThreads / 32 ? s_warp[lane] : 0;
-    int y = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, y, o);
-      if (lane >= o) y += u;
-    }
-    if (lane < kSelThreads / 32) s_warp[lane] = y - x;  // exclusive over warps
-    if (lane == kSelThreads / 32 - 1) s_warp[kSelThreads / 32] = y;
-  }
-  __syncthreads();
-  const int r = s_warp[warp] + incl - v;
-  *total = s_warp[kSelThreads / 32];
-  __syncthreads();
-  return r;
-}
 
 __global__ void __launch_bounds__(kSelThreads) level2_select_kernel(const float* __restrict__ ens,
                                                                     const int32_t* __restrict__ resident_count,
@@ -99,53 +62,19 @@ __global__ void __launch_bounds__(kSelThreads) level2_select_kernel(const float*
   __shared__ uint32_t s_hist[2048];
   __shared__ int s_warp[kSelThreads / 32 + 1];
   __shared__ uint32_t s_pick[2];
+  const BlockSelScratch sc{s_hist, s_warp, s_pick};
   const int b = blockIdx.x, t = threadIdx.x;
   const int nv = max(0, min(resident_count[b], R));
   const float* row = ens + (size_t)b * R;
-  for (int i = t; i < nv; i += kSelThreads) s_key[i] = sel_key(row[i]);
+  for (int i = t; i < nv; i += kSelThreads) s_key[i] = block_order_key(row[i]);
   const bool all = k >= nv;
   uint32_t T = 0u;
   int need = 0;  // keys equal to T to keep
   if (!all) {
-    uint32_t prefix = 0u, want = (uint32_t)k;
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0), nbits = pass == 2 ? 10 : 11;
-      const int nb = 1 << nbits, hi = shift + nbits;
-      for (int i = t; i < nb; i += kSelThreads) s_hist[i] = 0u;
-      __syncthreads();
-      for (int i = t; i < nv; i += kSelThreads) {
-        const uint32_t key = s_key[i];
-        if (hi >= 32 || (key >> hi) == (prefix >> hi)) atomicAdd(&s_hist[(key >> shift) & (nb - 1)], 1u);
-      }
-      __syncthreads();
-      // thread t owns bins [t*per, (t+1)*per) in descending digit order
-      const int per = nb / kSelThreads;
-      uint32_t mine = 0;
-      for (int j = 0; j < per; ++j) mine += s_hist[nb - 1 - (t * per + j)];
-      int tot;
-      const uint32_t before = (uint32_t)sel_scan((int)mine, s_warp, &tot);
-      if (before < want && before + mine >= want) {
-        uint32_t acc = before;
-        for (int j = 0; j < per; ++j) {
-          const int d = nb - 1 - (t * per + j);
-          const uint32_t c = s_hist[d];
-          if (acc + c >= want) {
-            s_pick[0] = prefix | ((uint32_t)d << shift);
-            s_pick[1] = want - acc;
-            break;
-          }
-          acc += c;
-        }
-      }
-      __syncthreads();
-      prefix = s_pick[0];
-      want = s_pick[1];
-      __syncthreads();
-    }
-    T = prefix;
-    need = (int)want;
+    __syncthreads();
+    block_kth_largest(s_key, nv, (uint32_t)k, sc, &T, &need);
   }
+  __syncthreads();
   // ordered compaction: thread t scans the contiguous slots [lo, hi)
   const int span = (nv + kSelThreads - 1) / kSelThreads;
   const int lo = min(nv, t * span), hi = min(nv, lo + span);
@@ -156,10 +85,10 @@ __global__ void __launch_bounds__(kSelThreads) level2_select_kernel(const float*
       gt += s_key[i] > T ? 1 : 0;
     }
   int tot;
-  const int eq_before = all ? 0 : sel_scan(eq, s_warp, &tot);
+  const int eq_before = all ? 0 : block_exclusive_scan(eq, s_warp, &tot);
   const int keep_eq = all ? 0 : max(0, min(eq, need - eq_before));
   const int kept = all ? hi - lo : gt + keep_eq;
-  int pos = sel_scan(kept, s_warp, &tot);
+  int pos = block_exclusive_scan(kept, s_warp, &tot);
   int32_t* out = out_ids + (size_t)b * k;
   const int32_t* ids = resident_ids + (size_t)b * R;
   int eq_seen = 0;

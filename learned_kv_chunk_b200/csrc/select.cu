@@ -21,11 +21,13 @@
 // same global histogram.  Ties at T are ranked across shards by an exclusive
 // sum of the per-shard tie counts in shard order (one all-gather).
 #include "fm_internal.cuh"
+#include "select_block.cuh"
 
 namespace fm {
 namespace {
 
 constexpr int kThreads = 512;  // top-K blocks: 8192 chunks each, so few per-block merges per row
+static_assert(kThreads == kBlkThreads, "the block scans assume the selection block size");
 constexpr int kPerThread = 16;
 constexpr int kChunk = kThreads * kPerThread;  // elements per block slice
 constexpr int kBins0 = 2048, kBins1 = 2048, kBins2 = 1024;
@@ -35,7 +37,8 @@ static_assert(kShardBins >= kBins0 && kShardBins >= kBins1 && kShardBins >= kBin
 constexpr int kShift[3] = {21, 10, 0};
 constexpr int kBits[3] = {11, 11, 10};
 
-enum : int { kModeEmpty = 0, kModeAll = 1, kModeSelect = 2 };
+// kModeFast: the candidate path below; kModeDone: the row's mask is written.
+enum : int { kModeEmpty = 0, kModeAll = 1, kModeSelect = 2, kModeFast = 3, kModeDone = 4 };
 
 // Per-row state (in the workspace).
 struct RowState {
@@ -72,6 +75,50 @@ __host__ __device__ inline Workspace carve(void* ws, int B, int nblk) {
 __host__ __device__ inline size_t ws_bytes(int B, int nblk) {
   return align256(sizeof(RowState) * (size_t)B) + align256(sizeof(uint32_t) * (size_t)B * kHistWords) +
          align256(sizeof(int) * (size_t)B * nblk);
+}
+
+// ------------------------------------------------- the candidate fast path
+// Exact top-K with one full pass over the scores.  A CTA per row takes an
+// evenly spread sample of up to kSample scores and sets the threshold tau to
+// the sample's key of rank 2K * S / n + 16 (about the 2K-th largest score of
+// the row).  One pass over the row then writes the mask's zeros and appends
+// every valid score >= tau, with its index, to the row's candidate list.  If
+// the list holds at least K entries (and fits), the K largest scores of the row
+// are all in it -- every other score is below tau, hence below every
+// candidate -- and a CTA per row selects them in shared memory and sets their
+// mask bytes.  A row whose list is too short or too long, or whose K-th value
+// is tied with values it does not keep (the tie order needs the chunk order),
+// falls back to the histogram passes, which run after and skip finished rows.
+constexpr int kSample = 8192;
+constexpr int kCandMax = 16384;  // a candidate list in one CTA's shared memory: 128 KB
+
+__host__ __device__ inline int cand_cap(int N) {
+  const int c = (N + 15) / 16;
+  return c < 256 ? 256 : (c > kCandMax ? kCandMax : c);
+}
+
+struct FastWs {
+  uint32_t* tau;   // [B]
+  int* cnt;        // [B] candidates found (may exceed the capacity)
+  uint32_t* ckey;  // [B, C]
+  int* cidx;       // [B, C]
+};
+
+__host__ __device__ inline FastWs carve_fast(void* ws, int B, int nblk, int C) {
+  uint8_t* p = static_cast<uint8_t*>(ws) + ws_bytes(B, nblk);
+  FastWs f;
+  f.tau = reinterpret_cast<uint32_t*>(p);
+  p += align256(sizeof(uint32_t) * (size_t)B);
+  f.cnt = reinterpret_cast<int*>(p);
+  p += align256(sizeof(int) * (size_t)B);
+  f.ckey = reinterpret_cast<uint32_t*>(p);
+  p += align256(sizeof(uint32_t) * (size_t)B * C);
+  f.cidx = reinterpret_cast<int*>(p);
+  return f;
+}
+
+__host__ __device__ inline size_t fast_ws_bytes(int B, int nblk, int C) {
+  return ws_bytes(B, nblk) + 2 * align256(sizeof(int) * (size_t)B) + 2 * align256(sizeof(int) * (size_t)B * C);
 }
 
 // Order-preserving key: larger float -> larger key; +0 and -0 equal; NaN lowest.
@@ -114,14 +161,14 @@ __global__ void threshold_kernel(const float* __restrict__ ens, const int32_t* _
 }
 
 // --------------------------------------------------------------- top-K
-__global__ void topk_init_kernel(Workspace w, const int32_t* __restrict__ n_valid, int N, int k) {
+__global__ void topk_init_kernel(Workspace w, const int32_t* __restrict__ n_valid, int N, int k, int fast) {
   const int b = blockIdx.x;
   uint32_t* h = w.hist + (size_t)b * kHistWords;
   for (int i = threadIdx.x; i < kHistWords; i += blockDim.x) h[i] = 0u;
   if (threadIdx.x == 0) {
     RowState s = {};
     s.nv = row_nvalid(n_valid, b, N);
-    s.mode = s.nv == 0 ? kModeEmpty : (k >= s.nv ? kModeAll : kModeSelect);
+    s.mode = s.nv == 0 ? kModeEmpty : (k >= s.nv ? kModeAll : (fast ? kModeFast : kModeSelect));
     s.prefix = 0u;
     s.remaining = min(k, s.nv);
     w.state[b] = s;
@@ -314,6 +361,7 @@ __global__ void __launch_bounds__(kThreads) topk_mask_kernel(Workspace w, const 
   const int b = blockIdx.y;
   const RowState* st = w.state + b;
   const int mode = st->mode, nv = st->nv;
+  if (mode == kModeDone) return;  // written by the candidate path
   const uint32_t T = st->prefix;
   const bool split_tie = mode == kModeSelect && st->need_eq != st->cnt_eq;
   const int need = st->need_eq;
@@ -388,6 +436,194 @@ __global__ void __launch_bounds__(kThreads) topk_mask_kernel(Workspace w, const 
   }
 }
 
+// Fast path, per row: the sample and the threshold tau; zeroes the list.
+__global__ void __launch_bounds__(kBlkThreads) topk_sample_kernel(Workspace w, FastWs f,
+                                                                  const float* __restrict__ ens, int N) {
+  extern __shared__ uint32_t s_key[];  // [kSample]
+  __shared__ uint32_t s_hist[2048];
+  __shared__ int s_warp[kBlkThreads / 32 + 1];
+  __shared__ uint32_t s_pick[2];
+  const int b = blockIdx.x, t = threadIdx.x;
+  const RowState* st = w.state + b;
+  if (st->mode != kModeFast) return;  // uniform across the block
+  const int nv = st->nv, K = st->remaining;
+  const int S = nv < kSample ? nv : kSample;
+  const float* row = ens + (size_t)b * N;
+  {  // all of a thread's strided loads in flight at once
+    constexpr int kPer = kSample / kBlkThreads;
+    float v[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int j = t + q * kBlkThreads;
+      v[q] = j < S ? __ldg(row + (int64_t)j * nv / S) : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int j = t + q * kBlkThreads;
+      if (j < S) s_key[j] = order_key(v[q]);
+    }
+  }
+  const int64_t r = (2 * (int64_t)K * S + nv - 1) / nv + 16;
+  uint32_t tau = 0u;  // 0: every valid score is a candidate
+  if (r < S) {
+    __syncthreads();
+    int need;
+    block_kth_largest(s_key, S, (uint32_t)r, BlockSelScratch{s_hist, s_warp, s_pick}, &tau, &need);
+  }
+  if (t == 0) {
+    f.tau[b] = tau;
+    f.cnt[b] = 0;
+  }
+}
+
+// Fast path, grid-wide: writes the mask of the Fast / All / Empty rows (zeros
+// for Fast rows; their kept bytes are set per row afterwards) and appends the
+// valid scores >= tau of Fast rows to the row's list.
+__global__ void __launch_bounds__(kThreads) topk_collect_kernel(Workspace w, FastWs f, int C,
+                                                                const float* __restrict__ ens, int N,
+                                                                uint8_t* __restrict__ keep) {
+  const int b = blockIdx.y;
+  const RowState* st = w.state + b;
+  const int mode = st->mode;
+  if (mode != kModeFast && mode != kModeAll && mode != kModeEmpty) return;
+  const int nv = st->nv;
+  const int64_t base = (int64_t)blockIdx.x * kChunk;
+  const float* row = ens + (int64_t)b * N;
+  uint8_t* out = keep + (int64_t)b * N;
+  if ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(keep) & 3u) == 0) {
+#pragma unroll
+    for (int i = 0; i < kPerThread / 4; ++i) {
+      const int64_t n = base + ((int64_t)i * kThreads + threadIdx.x) * 4;
+      if (n >= N) break;
+      uint32_t word = 0;
+      if (mode == kModeAll)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) word |= (n + c < nv ? 1u : 0u) << (8 * c);
+      *reinterpret_cast<uint32_t*>(out + n) = word;
+    }
+  } else {
+    for (int i = 0; i < kPerThread; ++i) {
+      const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
+      if (n >= N) break;
+      out[n] = (mode == kModeAll && n < nv) ? 1 : 0;
+    }
+  }
+  if (mode != kModeFast) return;  // uniform across the block
+  const uint32_t tau = f.tau[b];
+  uint32_t key[kPerThread];
+  uint32_t is_cand = 0;  // bit i: element i of this thread is a candidate
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
+    key[i] = order_key(n < nv ? __ldg(row + n) : 0.f);
+    if (n < nv && key[i] >= tau) is_cand |= 1u << i;
+  }
+  // one atomic per block: the block's candidates go to one range of the list
+  __shared__ int s_warp[kThreads / 32 + 1];
+  __shared__ int s_base;
+  int total;
+  const int before = block_exclusive_scan(__popc(is_cand), s_warp, &total);
+  if (threadIdx.x == 0) s_base = total ? atomicAdd(f.cnt + b, total) : 0;
+  __syncthreads();
+  int pos = s_base + before;
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    if (is_cand & (1u << i)) {
+      if (pos < C) {
+        f.ckey[(size_t)b * C + pos] = key[i];
+        f.cidx[(size_t)b * C + pos] = (int)(base + (int64_t)i * kThreads + threadIdx.x);
+      }
+      ++pos;
+    }
+  }
+}
+
+// The whole row by one CTA from global memory (the candidate path's fallback):
+// the K-th largest key T of ens[b, 0:nv), then the mask of [0, N) with the keys
+// equal to T taken in chunk order.  Three reads of the row by one SM: slow for
+// the row, but only rows the candidate path cannot finish take it.
+__device__ void row_select_in_block(const float* __restrict__ row, int nv, int N, int K, uint8_t* __restrict__ out,
+                                    BlockSelScratch sc) {
+  uint32_t T;
+  int need;
+  block_kth_largest_of([row](int i) { return order_key(__ldg(row + i)); }, nv, (uint32_t)K, sc, &T, &need);
+  // ordered mask: thread t takes kSpan consecutive chunks of each tile
+  constexpr int kSpan = 16;
+  constexpr int kTileN = kBlkThreads * kSpan;
+  int taken = 0;  // keys == T kept in earlier tiles
+  for (int c0 = 0; c0 < N; c0 += kTileN) {
+    const int lo = c0 + threadIdx.x * kSpan;
+    int eq = 0;
+    for (int j = 0; j < kSpan; ++j) {
+      const int n = lo + j;
+      if (n < nv && order_key(__ldg(row + n)) == T) ++eq;
+    }
+    int tile_eq;
+    const int eq_before = taken + block_exclusive_scan(eq, sc.warp, &tile_eq);
+    int rank = eq_before;
+    for (int j = 0; j < kSpan; ++j) {
+      const int n = lo + j;
+      if (n >= N) break;
+      uint8_t k = 0;
+      if (n < nv) {
+        const uint32_t key = order_key(__ldg(row + n));
+        k = (key > T || (key == T && rank++ < need)) ? 1 : 0;
+      }
+      out[n] = k;
+    }
+    taken += tile_eq;
+  }
+}
+
+// Fast path, per row: the K largest of the candidate list, or the whole row
+// by this CTA when the list cannot give them.
+__global__ void __launch_bounds__(kBlkThreads) topk_fastsel_kernel(Workspace w, FastWs f, const float* __restrict__ ens,
+                                                                   int C, int N, uint8_t* __restrict__ keep) {
+  extern __shared__ uint32_t s_dyn[];  // keys [C], then indices [C]
+  __shared__ uint32_t s_hist[2048];
+  __shared__ int s_warp[kBlkThreads / 32 + 1];
+  __shared__ uint32_t s_pick[2];
+  const int b = blockIdx.x, t = threadIdx.x;
+  RowState* st = w.state + b;
+  const int mode = st->mode;
+  __syncthreads();  // every thread has read the mode before thread 0 may change it
+  if (mode == kModeAll || mode == kModeEmpty) {  // the collect pass wrote their masks
+    if (t == 0) st->mode = kModeDone;
+    return;
+  }
+  if (mode != kModeFast) return;
+  const int cnt = f.cnt[b], K = st->remaining;
+  const BlockSelScratch sc{s_hist, s_warp, s_pick};
+  uint8_t* out = keep + (int64_t)b * N;
+  if (cnt < K || cnt > C) {  // too few candidates (tau too high) or too many to hold
+    row_select_in_block(ens + (int64_t)b * N, st->nv, N, K, out, sc);
+    if (t == 0) st->mode = kModeDone;
+    return;
+  }
+  uint32_t* keys = s_dyn;
+  int* idx = reinterpret_cast<int*>(s_dyn + C);
+  for (int i = t; i < cnt; i += kBlkThreads) {
+    keys[i] = f.ckey[(size_t)b * C + i];
+    idx[i] = f.cidx[(size_t)b * C + i];
+  }
+  __syncthreads();
+  uint32_t T;
+  int need;
+  block_kth_largest(keys, cnt, (uint32_t)K, sc, &T, &need);
+  int eq = 0;
+  for (int i = t; i < cnt; i += kBlkThreads) eq += keys[i] == T ? 1 : 0;
+  int eq_total;
+  block_exclusive_scan(eq, s_warp, &eq_total);
+  if (eq_total != need) {  // the K-th value is tied with values not kept: rank them by chunk order
+    row_select_in_block(ens + (int64_t)b * N, st->nv, N, K, out, sc);
+    if (t == 0) st->mode = kModeDone;
+    return;
+  }
+  for (int i = t; i < cnt; i += kBlkThreads)
+    if (keys[i] >= T) out[idx[i]] = 1;
+  if (t == 0) st->mode = kModeDone;
+}
+
 }  // namespace
 
 fm_status launch_ensemble(const float* scores, int L, int B, int N, int mode, float* ens,
@@ -414,19 +650,44 @@ size_t topk_workspace_bytes(int B, int N) {
   return ws_bytes(B, nblk);
 }
 
+size_t topk_workspace_bytes_fast(int B, int N) {
+  const int nblk = (int)(((int64_t)N + kChunk - 1) / kChunk);
+  return fast_ws_bytes(B, nblk, cand_cap(N));
+}
+
 fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, int k, uint8_t* keep,
                       void* ws, size_t ws_size, cudaStream_t st) {
   const int nblk = (int)(((int64_t)N + kChunk - 1) / kChunk);
   if (ws_size < ws_bytes(B, nblk)) return FM_ERR_INVALID_ARG;
   Workspace w = carve(ws, B, nblk);
-  topk_init_kernel<<<B, 256, 0, st>>>(w, n_valid, N, k);
+  const int C = cand_cap(N);
+  const bool fast = ws_size >= fast_ws_bytes(B, nblk, C) && 2 * (int64_t)k + 1024 <= C;
+  topk_init_kernel<<<B, 256, 0, st>>>(w, n_valid, N, k, fast ? 1 : 0);
+  note_launch();
   dim3 grid(nblk, B);
+  if (fast) {
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+      if (cudaFuncSetAttribute(topk_fastsel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)(2 * sizeof(uint32_t) * kCandMax)) != cudaSuccess)
+        return check_launch();
+      configured_dev = dev;
+    }
+    const FastWs f = carve_fast(ws, B, nblk, C);
+    topk_sample_kernel<<<B, kBlkThreads, sizeof(uint32_t) * kSample, st>>>(w, f, ens, N);
+    topk_collect_kernel<<<grid, kThreads, 0, st>>>(w, f, C, ens, N, keep);
+    topk_fastsel_kernel<<<B, kBlkThreads, 2 * sizeof(uint32_t) * (size_t)C, st>>>(w, f, ens, C, N, keep);
+    for (int i = 0; i < 3; ++i) note_launch();
+    return check_launch();  // every row is finished by the candidate path or its in-block fallback
+  }
   topk_hist_kernel<0, true><<<grid, kThreads, 0, st>>>(w, ens, N, nullptr);
   topk_hist_kernel<1, true><<<grid, kThreads, 0, st>>>(w, ens, N, nullptr);
   topk_hist_kernel<2, true><<<grid, kThreads, 0, st>>>(w, ens, N, nullptr);
   topk_eqcount_kernel<<<grid, kThreads, 0, st>>>(w, ens, N, nblk, nullptr);
   topk_mask_kernel<<<grid, kThreads, 0, st>>>(w, ens, N, nblk, keep, nullptr, 0, B);
-  for (int i = 0; i < 6; ++i) note_launch();
+  for (int i = 0; i < 5; ++i) note_launch();
   return check_launch();
 }
 

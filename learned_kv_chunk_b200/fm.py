@@ -72,6 +72,7 @@ def _load():
         "fm_ensemble": (I, [P, I, I, I, I, P, P]),
         "fm_score_fused": (I, [P, P, I64, P, I, I, P, P, I, F, P, P, P, P]),
         "fm_topk_workspace_bytes": (S, [I, I]),
+        "fm_topk_workspace_bytes_fast": (S, [I, I]),
         "fm_select_topk": (I, [P, P, I, I, I, P, P, S, P]),
         "fm_select_threshold": (I, [P, P, I, I, F, P, P]),
         "fm_select_topk_static": (I, [P, P, I, I, I, P, P]),
@@ -147,6 +148,10 @@ def fm_topk_workspace_bytes(B: int, N: int) -> int:
     return int(_lib.fm_topk_workspace_bytes(B, N))
 
 
+def fm_topk_workspace_bytes_fast(B: int, N: int) -> int:
+    return int(_lib.fm_topk_workspace_bytes_fast(B, N))
+
+
 def _comp_k_array(comp_k: Sequence[torch.Tensor]):
     for i, t in enumerate(comp_k):
         _need(t, torch.uint8, f"comp_k[{i}]")
@@ -182,7 +187,7 @@ def fm_select_topk(ens: torch.Tensor, k: int, n_valid: Optional[torch.Tensor] = 
     if n_valid is not None:
         _need(n_valid, torch.int32, "n_valid")
     keep = out if out is not None else torch.empty(B, N, device=ens.device, dtype=torch.bool)
-    nbytes = fm_topk_workspace_bytes(B, N)
+    nbytes = fm_topk_workspace_bytes_fast(B, N)
     ws = workspace if workspace is not None else torch.empty(nbytes, device=ens.device, dtype=torch.uint8)
     _check(_lib.fm_select_topk(_ptr(ens), _ptr(n_valid), B, N, int(k), _ptr(keep), _ptr(ws),
                                ws.numel(), _stream(stream)), "fm_select_topk")

@@ -242,3 +242,28 @@ def test_shared_keys_across_layers(retr, weights):
     assert np.abs(ens - O.ensemble(want, "mean")).max() <= H.SCORE_TOL
     np.testing.assert_array_equal(keep_thr.cpu().numpy(), O.select_threshold(ens, case.n_valid.numpy(), 0.5))
     retr.fm_sync_status()
+
+
+def test_topk_candidate_path_and_its_fallbacks():
+    """Rows of 262144 scores, K = 4096, a workspace large enough for the
+    candidate path: ordinary scores (the path finishes the row), large scores
+    placed only where the threshold sample looks (too few candidates: the row
+    falls back to the histogram passes), all scores equal (too many
+    candidates), and a K-th value tied across the cut (ties need chunk order):
+    every mask must equal the selection rule."""
+    B, N, K = 4, 262144, 4096
+    g = torch.Generator().manual_seed(12)
+    ens = torch.rand(B, N, generator=g) * 0.5
+    sampled = (torch.arange(8192, dtype=torch.int64) * N) // 8192
+    ens[1, sampled] = 0.9 + torch.rand(8192, generator=g) * 0.05  # only sampled positions are large
+    ens[2] = 0.5
+    ens[3] = torch.randint(0, 8, (N,), generator=g).float() / 8.0  # heavy ties at the K-th value
+    nv = torch.tensor([N, N, N - 17, 200000], dtype=torch.int32)
+    ws = torch.zeros(fm.fm_topk_workspace_bytes_fast(B, N), device=DEV, dtype=torch.uint8)
+    keep = fm.fm_select_topk(ens.to(DEV), K, nv.to(DEV), workspace=ws)
+    torch.cuda.synchronize()
+    H.check_topk_against_rule(keep.cpu().numpy(), ens.numpy(), nv.numpy(), K)
+    # the same rows through the histogram passes only (a workspace too small for the candidate path)
+    ws_min = torch.zeros(fm.fm_topk_workspace_bytes(B, N), device=DEV, dtype=torch.uint8)
+    keep_min = fm.fm_select_topk(ens.to(DEV), K, nv.to(DEV), workspace=ws_min)
+    assert torch.equal(keep.cpu(), keep_min.cpu())
