@@ -173,10 +173,11 @@ size_t fm_topk_workspace_bytes(int B, int N);
  * a threshold from a sample of each row, one pass that lists the scores above
  * it, and the selection among those in shared memory, instead of three
  * histogram passes and a mask pass over all scores.  The mask is the same
- * (exact) either way; rows the candidate path cannot finish (too few or too
- * many candidates, or the K-th value tied with values not kept) go through
- * the histogram passes.  Taken when the workspace given is at least this
- * large and 2k + 1024 <= min(16384, max(256, N / 16)). */
+ * (exact) either way; a row the candidate list cannot finish (too few or too
+ * many candidates, or the K-th value tied with values not kept) is selected
+ * by one CTA over the whole row, ties in chunk order.  Taken when the
+ * workspace given is at least this large and
+ * 2k + 1024 <= min(16384, max(256, N / 16)). */
 size_t fm_topk_workspace_bytes_fast(int B, int N);
 
 /* Top-K keep mask (README "Usage" select_topk(top_k=K); toy loop "top-K"):
@@ -198,8 +199,8 @@ fm_status fm_select_topk(const float* ens, const int32_t* n_valid, int B, int N,
 
 /* fm_select_topk for callers that cannot allocate device memory: the same
  * keep mask, with the scratch taken from a fixed array inside the library
- * instead of a caller workspace.  The paper has no counterpart; this is an
- * integration entry point.  Callers that need it: a serving process whose
+ * instead of a caller workspace.  The README's interface has no counterpart;
+ * this is an integration entry point.  Callers that need it: a serving process whose
  * device memory is all handed to its KV-cache pool at start-up, a plugin that
  * must leave device memory to its host framework's allocator, a decode loop
  * that cannot afford the device synchronisation cudaMalloc/cudaFree may cause.
