@@ -127,3 +127,20 @@ def test_header_is_plain_c(tmp_path):
     r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
                         "-I", os.path.dirname(HEADER), str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_topk_fast_workspace_sizing(lib):
+    """The candidate path's workspace adds, per row, a threshold, a count and a
+    list of min(16384, max(256, N/16)) (key, index) pairs to the base workspace;
+    the base one alone still fits the no-allocation scratch for 64 x 262144."""
+    f, g = lib.fm_topk_workspace_bytes, lib.fm_topk_workspace_bytes_fast
+    for fn in (f, g):
+        fn.restype = ctypes.c_size_t
+        fn.argtypes = [ctypes.c_int, ctypes.c_int]
+    assert g(0, 10) == 0 and g(1, 0) == 0
+    for B, N in [(1, 4096), (64, 262144), (8, 65536), (32, 131072), (3, 1 << 22)]:
+        cap = min(16384, max(256, (N + 15) // 16))
+        extra = g(B, N) - f(B, N)
+        assert extra >= 2 * 4 * B * cap and extra <= 2 * 4 * B * cap + 4 * 256, (B, N, extra)
+        assert g(B, N) % 256 == 0
+    assert f(64, 262144) <= (4 << 20) < g(64, 262144)
