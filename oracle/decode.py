@@ -10,8 +10,7 @@ compressed chunks, the chunks the last retrieval did not keep having their
 attention logits set to -inf; every 64 steps the retriever scores all chunks,
 ensembles the layers and selects the keep mask (top-K or sigmoid > thresh).
 
-The toy decoder is not defined by the pages.  Readings (each listed in
-DESIGN.md):
+The toy decoder is not defined by the pages.  Readings taken here:
   * the query is the step's hidden state [4096] taken as 32 heads of 128;
   * the memory is the chunks' dequantized compressed records (the only
     per-chunk data the toy has), used as keys and values;

@@ -12,7 +12,7 @@ function below restates one arrow of the Architecture figure in the order the
 figure gives it.  Arithmetic is fp64 except where the README fixes fp32 (the
 key dequantisation `fp8_values.view(float8_e4m3).float() * scale`).
 
-Readings of points the pages leave open (each listed in the design doc):
+Readings of points the pages leave open:
   * linear maps are bias-free, weights stored [out, in];
   * RMSNorm is x * (mean(x^2) + eps)^-1/2 * g;
   * RoPE acts on the last 64 dims in half-split pairs (64+j, 96+j); YaRN
@@ -21,6 +21,11 @@ Readings of points the pages leave open (each listed in the design doc):
   * the Hadamard transform is the Sylvester (natural) order, scaled by
     128^-1/2, applied to q only;
   * e4m3 is the OCP "fn" variant (bias 7, no infinities, S.1111.111 = NaN);
+  * the per-chunk scale multiplies the codes before the head dot products, so
+    the relu sees the scaled dot product whatever the scale's sign;
+  * a NaN code or scale makes the chunk's score NaN (relu, sigmoid and the
+    ensembles carry NaN, as torch's do); top-K ranks NaN below every number,
+    ties by chunk index, and NaN > thr is false;
   * top-K ties go to the lower chunk index, K >= n keeps every valid chunk;
     the threshold test is strict (score > thr);
   * chunks past a row's valid length score 0 and are never kept.

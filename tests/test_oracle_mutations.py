@@ -87,6 +87,39 @@ def _score_transposed_q(comp_k, q, w):
     return O.sigmoid(np.maximum(k[:, : qt.shape[1]] @ qt.T, 0) @ w)
 
 
+def _score_scale_after_relu(comp_k, q, w):
+    codes, scale = O.split_records(comp_k, q.shape[-1])
+    k8 = O.e4m3_decode(codes).astype(np.float64)
+    return O.sigmoid((np.maximum(k8 @ q.T, 0) * scale[:, None]) @ w)
+
+
+def _score_relu_drops_nan(comp_k, q, w):
+    k = O.dequant(comp_k, q.shape[-1]).astype(np.float64)
+    return O.sigmoid(np.fmax(k @ q.T, 0) @ w)
+
+
+def _ensemble_max_drops_nan(scores, mode="max"):
+    s = np.asarray(scores, np.float64)
+    return np.fmax.reduce(s, axis=0) if mode == "max" else O.__dict__["_orig_ensemble"](s, mode)
+
+
+def _topk_nan_high(ens, n_valid, k):
+    ens = np.asarray(ens, np.float64)
+    keep = np.zeros(ens.shape, bool)
+    for b in range(ens.shape[0]):
+        n = int(n_valid[b])
+        key = np.where(np.isnan(ens[b, :n]), np.inf, ens[b, :n])
+        order = np.lexsort((np.arange(n), -key))
+        keep[b, order[:min(k, n)]] = True
+    return keep
+
+
+def _threshold_nan_kept(ens, n_valid, thr):
+    ens = np.asarray(ens)
+    valid = np.arange(ens.shape[1])[None, :] < np.asarray(n_valid).reshape(-1, 1)
+    return valid & ~(ens <= thr)
+
+
 def _ensemble_sum(scores, mode="max"):
     s = np.asarray(scores, np.float64)
     return s.max(0) if mode == "max" else s.sum(0)
@@ -128,9 +161,14 @@ MUTATIONS = [
     ("score_chunks", _score_relu_after_weight),
     ("score_chunks", _score_no_scale),
     ("score_chunks", _score_transposed_q),
+    ("score_chunks", _score_scale_after_relu),
+    ("score_chunks", _score_relu_drops_nan),
     ("ensemble", _ensemble_sum),
+    ("ensemble", _ensemble_max_drops_nan),
     ("select_topk", _topk_ties_high),
+    ("select_topk", _topk_nan_high),
     ("select_threshold", _threshold_ge),
+    ("select_threshold", _threshold_nan_kept),
     ("query_prep", _fused_w_wrong_scale),
 ]
 

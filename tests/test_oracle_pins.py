@@ -297,6 +297,60 @@ def test_score_scale_applies_inside_relu():
     np.testing.assert_allclose(s, [1 / (1 + math.exp(-1.0)), 0.5], rtol=1e-15)
 
 
+def test_score_negative_scale_applies_inside_relu():
+    # README "compressed_k format": the scale is a plain fp32, so it may be
+    # negative; the key is codes * scale and the relu acts on k . q_h.  With
+    # s = -0.5 and codes (1, -2) the key is (-0.5, 1): head dots (-0.5, 1),
+    # relu (0, 1), logit 3 * 1 = 3.  Scaling after the relu would give
+    # s * relu((1, -2)) = (-0.5, 0) and logit -1.
+    q = np.zeros((2, 128))
+    q[0, 0] = q[1, 1] = 1.0
+    codes = np.zeros(128, np.uint8)
+    codes[0], codes[1] = 0x38, 0xC0  # 1.0, -2.0
+    rec = np.stack([_record(codes, -0.5), _record(codes, 0.5)])
+    s = O.score_chunks(rec, q, np.array([2.0, 3.0]))
+    # s = +0.5: key (0.5, -1), relu (0.5, 0), logit 1
+    np.testing.assert_allclose(s, [1 / (1 + math.exp(-3.0)), 1 / (1 + math.exp(-1.0))], rtol=1e-15)
+
+
+def test_nan_codes_and_scales_give_nan_scores():
+    # OCP E4M3 "fn": S.1111.111 is NaN.  A NaN element makes every head dot
+    # NaN, and relu and sigmoid carry it (as the README's torch ops do), so the
+    # chunk's score is NaN; a NaN scale does the same.  Other chunks are
+    # untouched.
+    q = np.ones((3, 128))
+    w = np.array([0.5, -0.25, 1.0])
+    base = np.full(128, 0x30, np.uint8)  # 0.5
+    bad_pos, bad_neg = base.copy(), base.copy()
+    bad_pos[17], bad_neg[100] = 0x7F, 0xFF
+    rec = np.stack([_record(base, 0.01), _record(bad_pos, 0.01), _record(bad_neg, 0.01),
+                    _record(base, float("nan"))])
+    s = O.score_chunks(rec, q, w)
+    assert np.isfinite(s[0]) and np.all(np.isnan(s[1:]))
+    k = 0.5 * float(np.float32(0.01))  # the scale is stored as fp32
+    np.testing.assert_allclose(s[0], 1 / (1 + math.exp(-(0.5 - 0.25 + 1.0) * 128 * k)), rtol=1e-12)
+
+
+def test_ensemble_carries_nan():
+    s = np.array([[0.2, 0.3], [np.nan, 0.9], [0.7, 0.1]])
+    for mode in ("max", "mean"):
+        e = O.ensemble(s, mode)
+        assert np.isnan(e[0]) and np.isfinite(e[1])
+
+
+def test_topk_and_threshold_rank_nan_below_every_number():
+    nan = float("nan")
+    ens = np.array([[0.2, nan, 0.1, 0.0, nan, 0.7]])
+    n = np.array([6])
+    assert O.select_topk(ens, n, 3)[0].tolist() == [True, False, True, False, False, True]
+    assert O.select_topk(ens, n, 4)[0].tolist() == [True, False, True, True, False, True]
+    # NaNs come last, in index order; K >= n keeps every valid chunk
+    assert O.select_topk(ens, n, 5)[0].tolist() == [True, True, True, True, False, True]
+    assert O.select_topk(ens, n, 6)[0].all()
+    assert O.select_threshold(ens, n, 0.05)[0].tolist() == [True, False, True, False, False, True]
+    assert not O.select_threshold(ens, n, -1.0)[0, [1, 4]].any()
+
+
 def test_score_degenerate_cases_and_range():
     rng = np.random.default_rng(6)
     q = rng.normal(size=(64, 128))
