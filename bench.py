@@ -34,6 +34,7 @@ from gen import synthetic as G  # noqa: E402
 
 METRIC = "retriever chunks scored/sec (3-layer ensemble + top-K)"
 UNIT = "chunks/s"
+NOMINAL_HBM_GBS = 8000.0  # the nominal HBM3e figure the target is stated against
 
 
 def parse():
@@ -42,7 +43,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", type=int, default=4)
+    ap.add_argument("--workload", default="4",
+                    help="index of the synthetic workload (0-4), or 'all': one JSON line per workload")
     ap.add_argument("--q-pieces", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -59,22 +61,28 @@ def parse():
     return ap.parse_args()
 
 
-def recorded_traffic(decisions: int):
-    """DRAM bytes per scoring launch from the committed ncu summary, scaled to
-    this launch's decisions; None once the kernel source differs from the one
-    the counters were taken on."""
+def scoring_kernel_sha1() -> str:
+    """sha1 of the scoring kernel's device source: score_tc.cu followed by the
+    device part of fm_internal.cuh (from its `#if defined(__CUDACC__)` line)."""
     import hashlib
-    import re
+    src = os.path.join(ROOT, "learned_kv_chunk_b200", "csrc")
+    m = hashlib.sha1()
+    m.update(open(os.path.join(src, "score_tc.cu"), "rb").read())
+    header = open(os.path.join(src, "fm_internal.cuh"), "rb").read()
+    m.update(header[header.index(b"#if defined(__CUDACC__)"):])
+    return m.hexdigest()
+
+
+def recorded_traffic(decisions: int):
+    """DRAM bytes per scoring launch from the committed ncu counters
+    (profiles/score_kernel_B8xN65536.json), scaled to this launch's decisions;
+    None once the kernel source differs from the one they were taken on."""
     try:
-        text = open(os.path.join(ROOT, "profiles", "score_kernel_B8xN65536.md")).read()
-        sha = re.search(r"kernel_source_sha1: ([0-9a-f]{40})", text).group(1)
-        per = float(re.search(r"traffic_bytes_per_decision: ([0-9.]+)", text).group(1))
-        src = os.path.join(ROOT, "learned_kv_chunk_b200", "csrc")
-        m = hashlib.sha1()
-        m.update(open(os.path.join(src, "score_tc.cu"), "rb").read())
-        header = open(os.path.join(src, "fm_internal.cuh"), "rb").read()
-        m.update(header[header.index(b"#if defined(__CUDACC__)"):])  # the header's device code
-        return int(per * decisions) if m.hexdigest() == sha else None
+        with open(os.path.join(ROOT, "profiles", "score_kernel_B8xN65536.json")) as f:
+            rec = json.load(f)
+        if rec["kernel_source_sha1"] != scoring_kernel_sha1():
+            return None
+        return int(float(rec["traffic_bytes_per_decision"]) * decisions)
     except Exception:
         return None
 
@@ -187,12 +195,11 @@ def job_throughput(decisions_per_rank: int, world: int, steps: int, elapsed_max_
 
 
 # -------------------------------------------------------------- our arm
-def run_ours(args, rank, world, local_rank):
+def run_ours(args, wl, rank, world, local_rank):
     from learned_kv_chunk_b200 import fm
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = G.WORKLOADS[args.workload]
     inp = G.make_query_inputs(wl)
     B, N, L = wl.B, wl.N, G.N_LAYERS
     r = fm.Retriever(inp.weights, device=local_rank, max_batch=max(64, B), q_pieces=args.q_pieces)
@@ -291,6 +298,7 @@ def run_ours(args, rank, world, local_rank):
     if not args.shared_keys:
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                     "frac": round(achieved / hbm_peak, 4), "traffic": recorded_traffic(decisions),
+                    "frac_of_nominal_8000": round(achieved / NOMINAL_HBM_GBS, 4),
                     "kernel": "score_kernel (fused scoring pass, via fm_score_fused)",
                     "kernel_ms": round(score_ms, 4), "peak_kind": peak_kind,
                     "alg_bytes_per_launch": alg_bytes}
@@ -306,7 +314,7 @@ def run_ours(args, rank, world, local_rank):
                     "alg_flops_per_launch": flops, "hbm_alg_bytes_per_launch": alg_bytes,
                     "hbm_achieved_gbs": round(achieved, 1), "hbm_frac": round(achieved / hbm_peak, 4)}
 
-    # end to end through the host-buffer API: H2D of the step's inputs, D2H of the mask
+    # end to end through the C ABI's host-buffer call: H2D of the step's inputs, D2H of the masks
     e2e = None
     if not args.no_e2e and not args.shared_keys:
         hk = [k.cpu().pin_memory() for k in keys]
@@ -325,12 +333,22 @@ def run_ours(args, rank, world, local_rank):
         d2h = B * N * (2 if wl.threshold is not None else 1)
         e2e = {"value": job_throughput(decisions, world, args.e2e_steps, et_max), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "steps": args.e2e_steps}
+               "steps": args.e2e_steps,
+               "call": "fm_retrieve_host (C ABI): pinned host inputs in, host masks out, one step per call"}
         del hk
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_sample(inp, keys, wl, q_row=0)
+        if wl.index == 0:  # the small workload's oracle is also timed on one core
+            try:
+                import threadpoolctl
+                with threadpoolctl.threadpool_limits(1):
+                    one = cpu_baseline_sample(inp, keys, wl, q_row=0)
+                cpu["single_thread"] = {"value": one["value"], "unit": UNIT, "cores": 1,
+                                        "sample": one["sample"]}
+            except Exception as e:  # noqa: BLE001
+                cpu["single_thread"] = {"unavailable": str(e)}
 
     r.close()
     return dict(value=value, ms_per_step=ms_per_step, roofline=roofline, e2e=e2e, cpu=cpu,
@@ -641,11 +659,10 @@ def cpu_baseline_sample(inp, keys, wl, q_row=0):
 
 
 # ---------------------------------------------------------- reference arm
-def run_reference(args):
+def run_reference(args, wl):
     """The CPU oracle on the host cores: each step scores a bounded sample
     (one row's query prep + 8192 chunks x 3 layers + ensemble + top-K)."""
     import oracle.retriever as O
-    wl = G.WORKLOADS[args.workload]
     inp = G.make_query_inputs(wl)
     layers = [{k: v.numpy().astype(np.float64) for k, v in w_.items()} for w_ in inp.weights]
     M = min(8192, wl.N)
@@ -710,21 +727,27 @@ def main():
             print(json.dumps(run_recall_reference(args) if args.impl == "reference" else run_recall(args)),
                   flush=True)
         return
+    wls = G.WORKLOADS if args.workload == "all" else [G.WORKLOADS[int(args.workload)]]
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args)), flush=True)
+            for wl in wls:
+                print(json.dumps(run_reference(args, wl)), flush=True)
         return
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        res = run_ours(args, rank, world, local_rank)
+        for wl in wls:
+            res = run_ours(args, wl, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(result_line(args, wl, world, res)), flush=True)
+            torch.cuda.empty_cache()
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()
-    if rank != 0:
-        return
-    wl = G.WORKLOADS[args.workload]
+
+
+def result_line(args, wl, world, res):
     out = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -734,7 +757,7 @@ def main():
            "roofline": res["roofline"], "stages_ms": res["stages_ms"], "e2e": res["e2e"],
            "gpu_launches": res["launches"],
            "clocks": res["clocks"], "cpu_baseline": res["cpu"]}
-    print(json.dumps(out), flush=True)
+    return out
 
 
 if __name__ == "__main__":

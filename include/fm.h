@@ -139,9 +139,8 @@ fm_status fm_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* positio
  * terms (per-head power-of-two scaling) and the keys used as stored.
  * The comp_k pointers may alias.  All layers reading one key tensor is the
  * README "Usage" signature taken literally (one compressed_k scored by the
- * three layers' queries).  The pass loads a tile's layers one after another,
- * so with aliased pointers the repeats come from L2 and HBM reads the keys
- * once. */
+ * three layers' queries): when every layer's pointer is the same, the pass
+ * copies each 128-chunk key tile once and runs every layer's product from it. */
 fm_status fm_score(fm_ctx* ctx, const uint8_t* const* comp_k, int64_t row_stride_bytes,
                    const int32_t* n_valid, int B, int N, const float* q, const float* fused_w,
                    float* scores, cudaStream_t stream);
@@ -169,7 +168,9 @@ fm_status fm_score_fused(fm_ctx* ctx, const uint8_t* const* comp_k, int64_t row_
 /* Bytes of device workspace fm_select_topk needs for B rows of N chunks. */
 size_t fm_topk_workspace_bytes(int B, int N);
 
-/* Bytes of workspace with which fm_select_topk can take its candidate path:
+/* Bytes of workspace with which fm_select_topk can take its candidate path
+ * on rows of more than 16384 chunks (shorter rows take the one-kernel form
+ * described at fm_select_topk):
  * a threshold from a sample of each row, one pass that lists the scores above
  * it, and the selection among those in shared memory, instead of three
  * histogram passes and a mask pass over all scores.  The mask is the same
@@ -188,7 +189,10 @@ size_t fm_topk_workspace_bytes_fast(int B, int N);
  * keep [B, N] uint8 device (written);
  * ws device workspace of at least fm_topk_workspace_bytes(B, N) bytes (the
  * faster candidate path needs fm_topk_workspace_bytes_fast(B, N)), 16-byte
- * aligned, owned by the caller; its contents on entry do not matter. */
+ * aligned, owned by the caller; its contents on entry do not matter.
+ * Rows of up to 16384 chunks are selected by one kernel, one CTA per row
+ * holding the row's keys in shared memory; it leaves the workspace
+ * untouched.  Longer rows take the candidate path or the histogram passes. */
 fm_status fm_select_topk(const float* ens, const int32_t* n_valid, int B, int N, int k,
                          uint8_t* keep, void* ws, size_t ws_bytes, cudaStream_t stream);
 
@@ -212,10 +216,64 @@ fm_status fm_select_topk(const float* ens, const int32_t* n_valid, int B, int N,
  * stream capture.  Every call on a device shares the one array and the call's
  * first kernel re-initialises what it uses: calls whose kernels overlap on the
  * GPU (different streams or threads) race and give wrong masks; order them.
+ * Rows of up to 16384 chunks take fm_select_topk's one-kernel form, which
+ * uses none of the array; longer rows take its candidate path when the array
+ * also holds the candidate lists (fm_topk_workspace_bytes_fast(B, N) <=
+ * FM_TOPK_STATIC_SCRATCH_BYTES, and the rule on k given there), otherwise the
+ * histogram form; the mask is the same either way.
  * Returns FM_ERR_UNSUPPORTED, launching nothing, when
  * fm_topk_workspace_bytes(B, N) > FM_TOPK_STATIC_SCRATCH_BYTES. */
 fm_status fm_select_topk_static(const float* ens, const int32_t* n_valid, int B, int N, int k,
                                 uint8_t* keep, cudaStream_t stream);
+
+/* ------------------------------------------------- whole path from host memory
+ * README "Usage" composed for a caller whose inputs live in host memory: the
+ * inputs are copied to device staging buffers, the path runs (fm_query_prep,
+ * fm_score_fused, fm_select_topk), and the masks are copied back. */
+typedef struct fm_host_batch {
+  int B;                      /* rows, 1..max_batch */
+  int N;                      /* chunks per row */
+  const float* hidden;        /* [B, HID] fp32 host */
+  const int64_t* positions;   /* [B] int64 host */
+  const uint8_t* comp_k[4];   /* per layer (n_layers used): [B, N_pad, 132] host, row b at
+                                 comp_k[l] + b * row_stride_bytes */
+  int64_t row_stride_bytes;   /* as fm_score (a multiple of 16, >= ceil4(N) * 132) */
+  const int32_t* n_valid;     /* [B] int32 host, or NULL (= N for all) */
+  int mode;                   /* FM_ENSEMBLE_MAX or FM_ENSEMBLE_MEAN */
+  int top_k;                  /* >= 1 with keep_topk, else ignored */
+  float thr;                  /* threshold, used with keep_thr */
+  uint8_t* keep_topk;         /* [B, N] host (written) or NULL: the top-K mask */
+  uint8_t* keep_thr;          /* [B, N] host (written) or NULL: the threshold mask */
+} fm_host_batch;
+
+/* Device buffers the call stages through, owned by the caller (the call
+ * allocates nothing).  Sizes for the batch's B and N: */
+typedef struct fm_device_staging {
+  uint8_t* comp_k[4];         /* per layer, B * row_stride_bytes bytes, 16-byte aligned */
+  float* hidden;              /* [B, HID], 16-byte aligned */
+  int64_t* positions;         /* [B] */
+  int32_t* n_valid;           /* [B] (used when the batch has n_valid) */
+  float* q;                   /* [B, L, H, D], 16-byte aligned */
+  float* fused_w;             /* [B, L, H] */
+  float* ens;                 /* [B, N] */
+  uint8_t* keep_topk;         /* [B, N] (used with keep_topk) */
+  uint8_t* keep_thr;          /* [B, N] (used with keep_thr) */
+  void* topk_ws;              /* fm_topk_workspace_bytes(B, N) bytes or more (the candidate path
+                                 takes fm_topk_workspace_bytes_fast), 16-byte aligned */
+  size_t topk_ws_bytes;
+} fm_device_staging;
+
+/* The whole path for one batch in host memory, asynchronous on `stream`: one
+ * cudaMemcpyAsync per input buffer (host to the staging buffers), query prep,
+ * the fused scoring pass with the ensemble and the threshold mask, top-K,
+ * then one cudaMemcpyAsync per requested mask back to the host.  The host
+ * masks hold their values once `stream` has reached the end of the call
+ * (fm_sync_status waits for it); the host inputs must stay unchanged until
+ * then.  Pinned host memory (cudaHostAlloc) keeps the copies asynchronous;
+ * pageable memory works, with the runtime staging the copies.  Argument and
+ * alignment errors are reported before anything is copied. */
+fm_status fm_retrieve_host(fm_ctx* ctx, const fm_host_batch* batch, const fm_device_staging* dev,
+                           cudaStream_t stream);
 
 /* Threshold keep mask (README "Usage" select_topk(threshold=t)):
  * keep[b,n] = (n < n_b) && (ens[b,n] > thr).  Shapes as fm_select_topk. */
@@ -389,6 +447,29 @@ int fm_last_cuda_error(void);
 
 /* Number of kernel launches issued by this process since load (all calls). */
 uint64_t fm_launch_count(void);
+
+/* ---------------------------------------------------- failure-path test hooks
+ * The pages have no counterpart; these exist so that tests can drive the
+ * library's error paths without faulting or hanging a GPU. */
+
+/* Makes the n-th device allocation from now (n >= 1, counted over all threads)
+ * made by fm_create or fm_level2_create fail as an out-of-memory cudaMalloc
+ * would; those calls then free what they had allocated and return
+ * FM_ERR_OOM.  n <= 0 turns the hook off. */
+void fm_debug_fail_alloc(int n);
+
+/* Number of device allocations currently held by live contexts and Level-2
+ * steps (what fm_destroy / fm_level2_destroy will free). */
+int64_t fm_debug_live_allocations(void);
+
+/* The next scoring launch on `ctx` (fm_score, fm_score_fused) never loads its
+ * query operand and bounds each of its waits by wait_limit_ns (1 ..
+ * 2e9 ns) instead of the usual 2 s: the wait for the query runs out, the
+ * kernel's roles stop at their next wait, copies already in flight land, and
+ * the launch ends with the context's error word set.  fm_sync_status then
+ * returns FM_ERR_DEVICE and clears it; the context stays usable.  No result
+ * of that launch is valid.  Call it only on a context no other thread uses. */
+fm_status fm_debug_stall_next_score(fm_ctx* ctx, uint64_t wait_limit_ns);
 
 /* Diagnostic: the raw tensor-core dot products of one 128-chunk tile of layer
  * `layer`, row b, tile t (chunks t*128 .. t*128+127), before the per-chunk

@@ -274,15 +274,11 @@ extern "C" fm_status fm_decode_attention(const float* q, const uint8_t* mem, int
   const int nseg = attn_segments(max_sel);
   float* part_o = static_cast<float*>(ws);
   float* part_ml = part_o + (size_t)B * nseg * kAH * kAD;
-  static int configured_dev = -1;
+  static PerDeviceOnce smem_set;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (configured_dev != dev) {
-    if (cudaFuncSetAttribute(sparse_attn_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(AttnSmem)) != cudaSuccess)
-      return check_launch();
-    configured_dev = dev;
-  }
+  if (fm_status s = smem_limit_once(smem_set, dev, sparse_attn_partial_kernel, (int)sizeof(AttnSmem)))
+    return s;
   sparse_attn_partial_kernel<<<dim3(nseg, B), kAThreads, sizeof(AttnSmem), stream>>>(
       q, mem, row_stride_bytes, n_mem, idx, count, max_sel, nseg, part_o, part_ml);
   sparse_attn_combine_kernel<<<dim3(kAH, B), kAD, 0, stream>>>(part_o, part_ml, nseg, out);

@@ -13,6 +13,8 @@ namespace {
 
 thread_local int g_last_cuda_error = 0;
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int64_t> g_fail_alloc_in{0};  // > 0: allocations until the one that is made to fail
+std::atomic<int64_t> g_live_allocs{0};
 
 fm_status cuda_fail(cudaError_t e) {
   g_last_cuda_error = (int)e;
@@ -75,6 +77,21 @@ fm_status check_keys(const fm_ctx* ctx, const uint8_t* const* comp_k, int64_t ro
 }
 
 }  // namespace
+
+cudaError_t dev_alloc(void** p, size_t bytes) {
+  *p = nullptr;
+  int64_t n = g_fail_alloc_in.load();
+  while (n > 0 && !g_fail_alloc_in.compare_exchange_weak(n, n - 1)) {
+  }
+  if (n == 1) return cudaErrorMemoryAllocation;  // this is the allocation the test asked to fail
+  const cudaError_t e = cudaMalloc(p, bytes);
+  if (e == cudaSuccess) g_live_allocs.fetch_add(1);
+  return e;
+}
+
+void dev_free(void* p) {
+  if (p && cudaFree(p) == cudaSuccess) g_live_allocs.fetch_sub(1);
+}
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
@@ -159,7 +176,7 @@ fm_status fm_create(const fm_config* cfg, const fm_layer_weights* w, int device,
   };
   fm_status st = FM_OK;
   for (auto& a : allocs) {
-    if (cudaMalloc(a.p, a.bytes) != cudaSuccess) {
+    if (dev_alloc(a.p, a.bytes) != cudaSuccess) {
       cudaGetLastError();
       st = FM_ERR_OOM;
       break;
@@ -206,8 +223,7 @@ fm_status fm_destroy(fm_ctx* c) {
   void* ptrs[] = {c->w_down, c->q_norm, c->w_up,   c->rope_freq, c->a_part, c->r_norm, c->rope_cs,
                   c->qpack,  c->wprime, c->qexp,   c->d_err,     c->x_hi,   c->x_lo,   c->r_hi,
                   c->r_lo,   c->up_part};
-  for (void* p : ptrs)
-    if (p) cudaFree(p);
+  for (void* p : ptrs) dev_free(p);
   cudaSetDevice(prev);
   delete c;
   return FM_OK;
@@ -250,6 +266,12 @@ static fm_status score_common(fm_ctx* c, const uint8_t* const* comp_k, int64_t r
   a.thr = thr;
   a.mode = mode;
   a.err = c->d_err;
+  a.wait_ns = kWaitLimitNs;
+  if (c->debug_stall) {  // one launch only
+    a.wait_ns = c->debug_wait_ns;
+    a.withhold_query = 1;
+    c->debug_stall = 0;
+  }
   a.dbg_out = dbg_out;
   a.dbg_layer = dbg_layer;
   a.dbg_b = dbg_b;
@@ -351,6 +373,48 @@ fm_status fm_topk_shard_mask(const float* ens_local, int B, int N, const int32_t
   return launch_topk_shard_mask(ens_local, B, N, eq_all, shard, keep_local, ws, ws_bytes, stream);
 }
 
+fm_status fm_retrieve_host(fm_ctx* c, const fm_host_batch* in, const fm_device_staging* d,
+                           cudaStream_t stream) {
+  if (!c || !in || !d) return FM_ERR_INVALID_ARG;
+  const int B = in->B, N = in->N, L = c->cfg.n_layers;
+  if (B < 1 || B > c->cfg.max_batch || N < 1 || !in->hidden || !in->positions) return FM_ERR_INVALID_ARG;
+  if (!in->keep_topk && !in->keep_thr) return FM_ERR_INVALID_ARG;
+  if (in->keep_topk && (in->top_k < 1 || !d->keep_topk || !d->topk_ws)) return FM_ERR_INVALID_ARG;
+  if (in->keep_thr && !d->keep_thr) return FM_ERR_INVALID_ARG;
+  if (in->mode != FM_ENSEMBLE_MAX && in->mode != FM_ENSEMBLE_MEAN) return FM_ERR_INVALID_ARG;
+  if (!d->hidden || !d->positions || !d->q || !d->fused_w || !d->ens || (in->n_valid && !d->n_valid))
+    return FM_ERR_INVALID_ARG;
+  for (int l = 0; l < L; ++l)
+    if (!in->comp_k[l]) return FM_ERR_INVALID_ARG;
+  if (fm_status s = check_keys(c, d->comp_k, in->row_stride_bytes, B, N)) return s;
+  if (!aligned(d->hidden, 16) || !aligned(d->q, 16) || !aligned(d->positions, 8) || !aligned(d->fused_w, 4) ||
+      !aligned(d->ens, 4) || (d->n_valid && !aligned(d->n_valid, 4)) || (d->topk_ws && !aligned(d->topk_ws, 16)))
+    return FM_ERR_ALIGNMENT;
+  if (in->keep_topk && d->topk_ws_bytes < topk_workspace_bytes(B, N)) return FM_ERR_INVALID_ARG;
+  const size_t mask = (size_t)B * N;
+  cudaError_t e = cudaSuccess;
+  auto copy = [&](void* dst, const void* src, size_t bytes, cudaMemcpyKind kind) {
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dst, src, bytes, kind, stream);
+  };
+  copy(d->hidden, in->hidden, sizeof(float) * (size_t)B * c->cfg.hidden, cudaMemcpyHostToDevice);
+  copy(d->positions, in->positions, sizeof(int64_t) * (size_t)B, cudaMemcpyHostToDevice);
+  if (in->n_valid) copy(d->n_valid, in->n_valid, sizeof(int32_t) * (size_t)B, cudaMemcpyHostToDevice);
+  for (int l = 0; l < L; ++l)
+    copy(d->comp_k[l], in->comp_k[l], (size_t)B * (size_t)in->row_stride_bytes, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  const int32_t* nv = in->n_valid ? d->n_valid : nullptr;
+  fm_status s = fm_query_prep(c, d->hidden, d->positions, B, d->q, d->fused_w, stream);
+  if (s == FM_OK)
+    s = fm_score_fused(c, d->comp_k, in->row_stride_bytes, nv, B, N, d->q, d->fused_w, in->mode, in->thr,
+                       nullptr, d->ens, in->keep_thr ? d->keep_thr : nullptr, stream);
+  if (s == FM_OK && in->keep_topk)
+    s = fm_select_topk(d->ens, nv, B, N, in->top_k, d->keep_topk, d->topk_ws, d->topk_ws_bytes, stream);
+  if (s != FM_OK) return s;
+  if (in->keep_topk) copy(in->keep_topk, d->keep_topk, mask, cudaMemcpyDeviceToHost);
+  if (in->keep_thr) copy(in->keep_thr, d->keep_thr, mask, cudaMemcpyDeviceToHost);
+  return e == cudaSuccess ? FM_OK : record_cuda_error(e);
+}
+
 fm_status fm_sync_status(fm_ctx* c, cudaStream_t stream) {
   if (!c) return FM_ERR_INVALID_ARG;
   cudaError_t e = cudaStreamSynchronize(stream);
@@ -381,6 +445,17 @@ const char* fm_strerror(fm_status s) {
 int fm_last_cuda_error(void) { return g_last_cuda_error; }
 
 uint64_t fm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void fm_debug_fail_alloc(int n) { g_fail_alloc_in.store(n > 0 ? n : 0); }
+
+int64_t fm_debug_live_allocations(void) { return g_live_allocs.load(); }
+
+fm_status fm_debug_stall_next_score(fm_ctx* c, uint64_t wait_limit_ns) {
+  if (!c || wait_limit_ns == 0 || wait_limit_ns > kWaitLimitNs) return FM_ERR_INVALID_ARG;
+  c->debug_wait_ns = wait_limit_ns;
+  c->debug_stall = 1;
+  return FM_OK;
+}
 
 fm_status fm_debug_tile_dots(fm_ctx* c, const uint8_t* const* comp_k, int64_t row_stride, int B,
                              int N, const float* q, const float* fused_w, int layer, int b, int t,

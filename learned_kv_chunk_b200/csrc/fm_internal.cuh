@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/fm.h"
 
 namespace fm {
@@ -52,15 +54,59 @@ struct fm_ctx {
   float* r_hi; float* r_lo;            // [max_batch, L, R] RMSNorm output, split
   float* up_part;                      // [2, max_batch, L*H*D] K-split partial sums of wq_b . r
   alignas(64) unsigned char wmaps[2][128];  // TMA tensor maps (fp32): w_down, w_up
+  // test hook (fm_debug_stall_next_score): the next scoring launch withholds
+  // its query operand and bounds its waits by debug_wait_ns
+  int debug_stall;
+  uint64_t debug_wait_ns;
 };
 
 namespace fm {
+
+// Device allocations of fm_create and fm_level2_create go through these two,
+// so that a test can make the n-th one fail (fm_debug_fail_alloc) and count
+// the allocations still held (fm_debug_live_allocations).
+cudaError_t dev_alloc(void** p, size_t bytes);
+void dev_free(void* p);
+
+// Bound of every wait inside a kernel when no test hook shortens it.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // launch helpers (fm_api.cu)
 void note_launch();
 fm_status check_launch();
 // Records `e` for fm_last_cuda_error and returns FM_ERR_CUDA.
 fm_status record_cuda_error(cudaError_t e);
+
+// A set-up step to run once per device (a kernel's dynamic shared-memory
+// limit): run(device, fn) calls fn() until it has returned FM_OK on that
+// device and skips it afterwards.  Several host threads may call run() at
+// once; two of them may both run fn() the first time, so fn() must be
+// idempotent.  Devices past 63 run fn() on every call.
+class PerDeviceOnce {
+ public:
+  template <typename F>
+  fm_status run(int device, F&& fn) {
+    const bool tracked = device >= 0 && device < 64;
+    const uint64_t bit = tracked ? (uint64_t)1 << device : 0;
+    if (tracked && (done_.load(std::memory_order_acquire) & bit)) return FM_OK;
+    const fm_status s = fn();
+    if (s == FM_OK && tracked) done_.fetch_or(bit, std::memory_order_acq_rel);
+    return s;
+  }
+
+ private:
+  std::atomic<uint64_t> done_{0};
+};
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` once per device.
+template <typename K>
+fm_status smem_limit_once(PerDeviceOnce& once, int device, K* kernel, int bytes) {
+  return once.run(device, [&]() -> fm_status {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    return e == cudaSuccess ? FM_OK : record_cuda_error(e);
+  });
+}
 
 // kernels' host entry points
 fm_status launch_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* positions, int B,
@@ -84,6 +130,8 @@ struct ScoreArgs {
   float thr;
   int mode;                // FM_ENSEMBLE_*
   int* err;
+  uint64_t wait_ns;        // bound of every wait (kWaitLimitNs unless a test shortens it)
+  int withhold_query;      // test hook: the query operand is never loaded, so its wait runs out
   // diagnostic dump of one tile's raw accumulators
   float* dbg_out;          // [128, 192] or null
   int dbg_layer, dbg_b, dbg_t;
@@ -100,6 +148,13 @@ size_t topk_workspace_bytes(int B, int N);
 size_t topk_workspace_bytes_fast(int B, int N);
 fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, int k, uint8_t* keep,
                       void* ws, size_t ws_bytes, cudaStream_t stream);
+// The one-kernel form for rows of up to 16 * 16384 chunks (a thread-block
+// cluster per row, no workspace): its cluster size for N, 0 past that bound;
+// whether fm_select_topk takes it for N.
+int topk_cluster_size(int N);
+bool topk_use_cluster(int N);
+fm_status launch_topk_cluster(const float* ens, const int32_t* n_valid, int B, int N, int k, uint8_t* keep,
+                              cudaStream_t stream);
 size_t compact_workspace_bytes(int B, int N);
 fm_status launch_compact(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx, int32_t* count,
                          void* ws, cudaStream_t stream);
@@ -121,6 +176,39 @@ fm_status launch_topk_shard_mask(const float* ens, int B, int N, const int32_t* 
 
 // ------------------------------------------------------------ PTX wrappers
 #if defined(__CUDACC__)
+
+// Launches `kernel` so that it may start while the kernel ahead of it in
+// `stream` is still running (programmatic dependent launch): the kernel must
+// pass grid_dependency_wait() before it touches memory that kernel writes.
+// Inside a stream capture the launch is a plain one.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = cap == cudaStreamCaptureStatusNone ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Waits until the kernels this one was launched after (launch_overlapped)
+// have finished and their writes are visible; returns at once otherwise.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Lets a kernel launched after this one with launch_overlapped start now.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -483,6 +571,16 @@ __device__ __forceinline__ void tmem_ld16x3_wait(uint32_t t0, uint32_t t1, uint3
       : FM_TMEM_REGS16(a), FM_TMEM_REGS16(b), FM_TMEM_REGS16(c)
       : "r"(t0), "r"(t1), "r"(t2)
       : "memory");
+}
+
+// max(a, b) that is NaN when either operand is NaN (fmaxf returns the other
+// operand instead).  relu(x) = fmax_nan(x, 0) and the max ensemble use it, so
+// a NaN key element or scale carries through to the chunk's score, as it does
+// through the README's torch operations.
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
 }
 
 // Packed fp32x2 arithmetic (sm_100): one instruction for two lanes of data.

@@ -153,8 +153,7 @@ void release(fm_level2* s) {
   if (s->exec) cudaGraphExecDestroy(s->exec);
   if (s->graph) cudaGraphDestroy(s->graph);
   void* ptrs[] = {s->q, s->fused_w, s->ens, s->keep, s->slots, s->slot_count, s->topk_ws, s->compact_ws};
-  for (void* p : ptrs)
-    if (p) cudaFree(p);
+  for (void* p : ptrs) dev_free(p);
   delete s;
 }
 
@@ -204,7 +203,7 @@ extern "C" fm_status fm_level2_create(fm_ctx* ctx, const fm_level2_desc* d, cuda
       {&s->compact_ws, compact_workspace_bytes(B, R)},
   };
   for (auto& a : allocs) {
-    if (cudaMalloc(a.p, a.bytes) != cudaSuccess) {
+    if (dev_alloc(a.p, a.bytes) != cudaSuccess) {
       cudaGetLastError();
       release(s);
       cudaSetDevice(prev);

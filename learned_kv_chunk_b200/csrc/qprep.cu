@@ -462,74 +462,184 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // The up projection's K-split partials summed, then RoPE and the Hadamard:
 // one warp per (row, layer, head).
 __global__ void __launch_bounds__(kThreads) qup_finish_kernel(const float* __restrict__ part, StreamK sk,
-                                                              int64_t split_stride, int B, int L,
+                                                              int nsplit, int64_t split_stride, int B, int L,
                                                               const float* __restrict__ rope_cs,
                                                               float* __restrict__ q);
 
 // One CTA per (row b, layer l): reduce the K splits, RMSNorm the wq_a part,
 // scale the weights_proj part into fused_w, and (layer 0) the RoPE table.
-__global__ void __launch_bounds__(kThreads) qnorm_kernel(
+// ------------------------------------------------ GEMV for up to 8 rows
+// part[s, b, m] = sum over the s-th K slice of W[m, k] X[b, layer(m), k], for
+// B <= TB <= 8 rows of X: bound by the bytes of W, each read once.  A warp owns
+// 4 consecutive rows of W and one K slice; lane j streams the float4 columns
+// k = 4j + 128i of its 4 rows with kGemvUnroll slices of loads in flight, the
+// CTA's X slice sits in shared memory, and the 4 x TB sums are reduced across
+// the warp by a butterfly in which every exchange halves the values a lane
+// holds (4 TB - 1 shuffles in all) and lane j ends with sum number j.
+constexpr int kGemvWarps = 8;
+constexpr int kGemvRows = 4;  // rows of W per warp
+constexpr int kGemvUnroll = 4;
+
+template <int TB>
+__global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(
+    const float* __restrict__ W, int M, int K, int kslice, const float* __restrict__ X,
+    int64_t x_row_stride, int64_t x_layer_stride, int rows_per_layer, int B, float* __restrict__ part) {
+  extern __shared__ __align__(16) float Xs[];  // [TB][kslice]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_cta = blockIdx.x * kGemvWarps * kGemvRows;
+  const int m0 = m_cta + warp * kGemvRows;
+  const int s = blockIdx.y;
+  const int k0 = s * kslice;
+  const int layer = rows_per_layer > 0 ? m_cta / rows_per_layer : 0;
+  const bool rows_ok = m0 + kGemvRows <= M;
+  // W does not depend on the kernel ahead: start its first slices now.  The
+  // register ring w holds kGemvUnroll slices (slice i in w[i % kGemvUnroll]);
+  // a slot is reloaded with slice i + kGemvUnroll as soon as slice i is used.
+  float4 w[kGemvUnroll][kGemvRows];
+  const float* wrow = W + (size_t)m0 * K + k0 + 4 * lane;
+  auto load_slice = [&](float4* dst, int i) {
+#pragma unroll
+    for (int r = 0; r < kGemvRows; ++r)
+      dst[r] = (rows_ok && i * 128 < kslice)
+                   ? __ldg(reinterpret_cast<const float4*>(wrow + (size_t)r * K + i * 128))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+#pragma unroll
+  for (int u = 0; u < kGemvUnroll; ++u) load_slice(w[u], u);
+  grid_dependency_wait();  // X is written by the kernel ahead
+  const float* xsrc = X + (size_t)layer * x_layer_stride + k0;
+  for (int i = threadIdx.x; i < TB * kslice / 4; i += kGemvWarps * 32) {
+    const int b = (i * 4) / kslice, k = (i * 4) % kslice;
+    reinterpret_cast<float4*>(Xs)[i] =
+        b < B ? __ldg(reinterpret_cast<const float4*>(xsrc + (size_t)b * x_row_stride + k))
+              : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
+  float acc[kGemvRows * TB];
+#pragma unroll
+  for (int v = 0; v < kGemvRows * TB; ++v) acc[v] = 0.f;
+  const int nslices = kslice / 128;
+  for (int i0 = 0; i0 < nslices; i0 += kGemvUnroll) {
+#pragma unroll
+    for (int u = 0; u < kGemvUnroll; ++u) {
+      const int i = i0 + u;
+      if (i >= nslices) break;
+#pragma unroll
+      for (int b = 0; b < TB; ++b) {
+        const float4 x = *reinterpret_cast<const float4*>(Xs + (size_t)b * kslice + i * 128 + 4 * lane);
+#pragma unroll
+        for (int r = 0; r < kGemvRows; ++r) {
+          float a = acc[r * TB + b];
+          a = fmaf(w[u][r].x, x.x, a);
+          a = fmaf(w[u][r].y, x.y, a);
+          a = fmaf(w[u][r].z, x.z, a);
+          a = fmaf(w[u][r].w, x.w, a);
+          acc[r * TB + b] = a;
+        }
+      }
+      load_slice(w[u], i + kGemvUnroll);
+    }
+  }
+  // butterfly: at stride h, the lanes with bit h set keep the upper half of
+  // their values and the others the lower half, each adding its partner's copy
+  constexpr int V = kGemvRows * TB;
+#pragma unroll
+  for (int h = V / 2; h >= 1; h >>= 1) {
+    const bool upper = (lane & h) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = upper ? acc[i] : acc[i + h];
+      const float keep = upper ? acc[i + h] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, h);
+    }
+  }
+#pragma unroll
+  for (int h = V; h < 32; h <<= 1) acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], h);
+  if (lane < V && rows_ok) {
+    const int r = lane / TB, b = lane % TB;
+    if (b < B) part[((size_t)s * B + b) * M + m0 + r] = acc[0];
+  }
+}
+
+constexpr int kNormThreads = 1024;  // one thread per element of a (row, layer) block, two past 1024
+
+__global__ void __launch_bounds__(kNormThreads) qnorm_kernel(
     const float* __restrict__ a_part, int ksplit, StreamK sk, int B, int L, int R, int H,
     const float* __restrict__ q_norm, float eps, float w_scale, const int64_t* __restrict__ positions,
     const double* __restrict__ rope_freq, int rope_half, float* __restrict__ r_norm,
     float* __restrict__ fused_w, float* __restrict__ rope_cs, float* __restrict__ r_hi,
     float* __restrict__ r_lo) {
+  grid_dependency_wait();  // the partial sums come from the kernel ahead
   const int b = blockIdx.x, l = blockIdx.y;
+  const int t = threadIdx.x;
   const int M = L * (R + H);
   const float* base = a_part + (size_t)b * M + (size_t)l * (R + H);
   // partials of element i: ksplit (K splits), or its tile's stream-K slots,
   // looked up per tile from a table built once
   constexpr int kMaxTiles = 64;  // tiles in the table; a (row, layer) block spans (R + H) / 128 + 2
   __shared__ int s_slots[kMaxTiles];
+  __shared__ float red[kNormThreads / 32];
   const int t0 = (l * (R + H)) / kTcBM;
   if (ksplit <= 0)
-    for (int j = threadIdx.x; j < kMaxTiles; j += kThreads)
-      s_slots[j] = sk.slots((b / sk.bn) * sk.mtiles + t0 + j);
+    for (int j = t; j < kMaxTiles; j += kNormThreads) s_slots[j] = sk.slots((b / sk.bn) * sk.mtiles + t0 + j);
+  // the row's RoPE table (layer 0's block): angles and cos/sin in fp64,
+  // rounded once; computed while the partial sums below are in flight
+  const int last_warp = kNormThreads - 32;
+  if (l == 0 && t >= last_warp && t - last_warp < rope_half) {
+    const int j = t - last_warp;
+    const double theta = (double)positions[b] * rope_freq[j];
+    double sn, cs;
+    sincos(theta, &sn, &cs);
+    rope_cs[((size_t)b * rope_half + j) * 2 + 0] = (float)cs;
+    rope_cs[((size_t)b * rope_half + j) * 2 + 1] = (float)sn;
+  }
   __syncthreads();
   auto nparts = [&](int i) {
     if (ksplit > 0) return ksplit;
     const int j = (l * (R + H) + i) / kTcBM - t0;
     return j < kMaxTiles ? s_slots[j] : sk.slots((b / sk.bn) * sk.mtiles + t0 + j);
   };
-  __shared__ float red[kThreads / 32];
-  // the split sums of this thread's first kKeep elements stay in registers
-  // for the second loop; the partial loads of one element issue together
-  constexpr int kKeep = 8;
-  auto reduce = [&](int i) {
-    const int np = nparts(i);
+  // elements t and t + 1024 of the block: every partial of both is loaded
+  // before any is summed
+  const int n = R + H;
+  constexpr int kMaxParts = 16;
+  float v0[kMaxParts], v1[kMaxParts];
+  const int i0 = t, i1 = t + kNormThreads;
+  const int np0 = i0 < n ? nparts(i0) : 0, np1 = i1 < n ? nparts(i1) : 0;
+#pragma unroll
+  for (int s = 0; s < kMaxParts; ++s) {
+    v0[s] = s < np0 ? __ldg(base + (size_t)s * B * M + i0) : 0.f;
+    v1[s] = s < np1 ? __ldg(base + (size_t)s * B * M + i1) : 0.f;
+  }
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+  for (int s = 0; s < kMaxParts; ++s) { a0 += v0[s]; a1 += v1[s]; }
+  for (int s = kMaxParts; s < np0; ++s) a0 += base[(size_t)s * B * M + i0];
+  for (int s = kMaxParts; s < np1; ++s) a1 += base[(size_t)s * B * M + i1];
+  auto sum_of = [&](int i) {  // elements past the first 2048 (ranks above 1984 only)
     float a = 0.f;
-    if (np <= 16) {
-      float v[16];
-#pragma unroll
-      for (int s = 0; s < 16; ++s) v[s] = s < np ? __ldg(base + (size_t)s * B * M + i) : 0.f;
-#pragma unroll
-      for (int s = 0; s < 16; ++s) a += v[s];
-    } else {
-      for (int s = 0; s < np; ++s) a += base[(size_t)s * B * M + i];
-    }
+    for (int s = 0, np = nparts(i); s < np; ++s) a += base[(size_t)s * B * M + i];
     return a;
   };
-  float kept[kKeep];
-  float ss = 0.f;
-#pragma unroll
-  for (int k = 0; k < kKeep; ++k) {
-    const int i = threadIdx.x + k * kThreads;
-    kept[k] = i < R ? reduce(i) : 0.f;
-    ss = fmaf(kept[k], kept[k], ss);
-  }
-  for (int i = threadIdx.x + kKeep * kThreads; i < R; i += kThreads) {
-    const float a = reduce(i);
+  float ss = (i0 < R ? a0 * a0 : 0.f) + (i1 < R ? a1 * a1 : 0.f);
+  for (int i = t + 2 * kNormThreads; i < R; i += kNormThreads) {
+    const float a = sum_of(i);
     ss = fmaf(a, a, ss);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  if ((t & 31) == 0) red[t >> 5] = ss;
   __syncthreads();
   float tot = 0.f;
 #pragma unroll
-  for (int w = 0; w < kThreads / 32; ++w) tot += red[w];
+  for (int w = 0; w < kNormThreads / 32; ++w) tot += red[w];
   const float inv_rms = 1.0f / sqrtf(tot / (float)R + eps);
   auto emit = [&](int i, float a) {
+    if (i >= n) return;
+    if (i >= R) {
+      fused_w[((size_t)b * L + l) * H + (i - R)] = a * w_scale;
+      return;
+    }
     const float r = a * inv_rms * q_norm[(size_t)l * R + i];
     r_norm[((size_t)b * L + l) * R + i] = r;
     if (r_hi) {  // the split operand of the tensor-core up projection
@@ -538,24 +648,9 @@ __global__ void __launch_bounds__(kThreads) qnorm_kernel(
       r_lo[((size_t)b * L + l) * R + i] = r - hi;
     }
   };
-#pragma unroll
-  for (int k = 0; k < kKeep; ++k) {
-    const int i = threadIdx.x + k * kThreads;
-    if (i < R) emit(i, kept[k]);
-  }
-  for (int i = threadIdx.x + kKeep * kThreads; i < R; i += kThreads) emit(i, reduce(i));
-  for (int h = threadIdx.x; h < H; h += kThreads) {
-    const float a = reduce(R + h);
-    fused_w[((size_t)b * L + l) * H + h] = a * w_scale;
-  }
-  if (l == 0 && threadIdx.x < rope_half) {
-    const int j = threadIdx.x;
-    const double theta = (double)positions[b] * rope_freq[j];
-    double sn, cs;
-    sincos(theta, &sn, &cs);
-    rope_cs[((size_t)b * rope_half + j) * 2 + 0] = (float)cs;
-    rope_cs[((size_t)b * rope_half + j) * 2 + 1] = (float)sn;
-  }
+  emit(i0, a0);
+  emit(i1, a1);
+  for (int i = t + 2 * kNormThreads; i < n; i += kNormThreads) emit(i, sum_of(i));
 }
 
 // RoPE on dims 64..127 (pairs (64+j, 96+j)) and the normalised Hadamard of
@@ -597,17 +692,21 @@ __device__ __forceinline__ void rope_wht_store(float x[4], int b, int l, int h, 
       make_float4(x[0] * inv_sqrt_d, x[1] * inv_sqrt_d, x[2] * inv_sqrt_d, x[3] * inv_sqrt_d);
 }
 
+// Sums the partials of wq_b . r (nsplit slices, or when nsplit is 0 the
+// stream-K slots of the head's tile), then RoPE and the Hadamard: one warp per
+// (b, l, h).
 __global__ void __launch_bounds__(kThreads) qup_finish_kernel(const float* __restrict__ part, StreamK sk,
-                                                              int64_t split_stride, int B, int L,
+                                                              int nsplit, int64_t split_stride, int B, int L,
                                                               const float* __restrict__ rope_cs,
                                                               float* __restrict__ q) {
+  grid_dependency_wait();  // the partials come from the kernel ahead
   const int idx = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);  // (b*L + l)*64 + h
   if (idx >= B * L * kHeads) return;
   const int lane = threadIdx.x & 31;
   const int h = idx % kHeads, bl = idx / kHeads, l = bl % L, b = bl / L;
   const float* src = part + (size_t)b * L * kHeads * kHeadDim + ((size_t)l * kHeads + h) * kHeadDim + lane * 4;
   // one head's 128 rows of wq_b are one tile: its partials are the tile's slots
-  const int nslots = sk.slots((b / sk.bn) * sk.mtiles + l * kHeads + h);
+  const int nslots = nsplit > 0 ? nsplit : sk.slots((b / sk.bn) * sk.mtiles + l * kHeads + h);
   float4 acc = __ldg(reinterpret_cast<const float4*>(src));
   for (int s = 1; s < nslots; ++s) {
     const float4 v = __ldg(reinterpret_cast<const float4*>(src + (int64_t)s * split_stride));
@@ -691,6 +790,7 @@ __global__ void __launch_bounds__(kThreads) qpack_kernel(const float* __restrict
                                                          uint8_t* __restrict__ qpack,
                                                          float* __restrict__ wprime,
                                                          int32_t* __restrict__ qexp) {
+  grid_launch_dependents();  // the scoring pass may start its key stream now
   const int idx = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);  // (b*L + l)*64 + h
   if (idx >= n) return;
   const int lane = threadIdx.x & 31;
@@ -722,6 +822,63 @@ __global__ void __launch_bounds__(kThreads) qpack_kernel(const float* __restrict
     wprime[idx] = fused_w[idx] * ldexpf(1.0f, -e);
     qexp[idx] = e;
   }
+}
+
+template <int TB>
+fm_status launch_gemv(const float* W, int M, int K, int ksplit, const float* X, int64_t x_row_stride,
+                      int64_t x_layer_stride, int rows_per_layer, int B, float* part, cudaStream_t st) {
+  const int kslice = K / ksplit;
+  const size_t smem = sizeof(float) * TB * (size_t)kslice;
+  static PerDeviceOnce smem_set;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (fm_status e = smem_limit_once(smem_set, dev, gemv_kernel<TB>, 64 * 1024)) return e;
+  const dim3 grid((M + kGemvWarps * kGemvRows - 1) / (kGemvWarps * kGemvRows), ksplit);
+  const cudaError_t e = launch_overlapped(gemv_kernel<TB>, grid, dim3(kGemvWarps * 32), smem, st, W, M, K,
+                                          kslice, X, x_row_stride, x_layer_stride, rows_per_layer, B, part);
+  note_launch();
+  return e == cudaSuccess ? FM_OK : record_cuda_error(e);
+}
+
+// The query chain for up to 8 rows: both projections as GEMVs bound by the
+// weights' bytes, the RMSNorm between them, then RoPE and the Hadamard.
+template <int TB>
+fm_status launch_query_prep_gemv(fm_ctx* ctx, const float* hidden, const int64_t* positions, int B,
+                                 float* q, float* fused_w, cudaStream_t st) {
+  const fm_config& c = ctx->cfg;
+  const int L = c.n_layers, R = c.q_lora_rank, HID = c.hidden;
+  const int Md = L * (R + kHeads), Mu = L * kHeads * kHeadDim;
+  // K slices of the down projection: enough CTAs for two per SM, slices of
+  // at least 1024 columns (a multiple of 128) that fit the shared X slice
+  int ks = 1;
+  const int row_blocks = (Md + kGemvWarps * kGemvRows - 1) / (kGemvWarps * kGemvRows);
+  while (ks * 2 <= ctx->splitk_max && HID % (ks * 2 * 128) == 0 && HID / (ks * 2) >= 1024 &&
+         row_blocks * ks < 2 * ctx->num_sms)
+    ks *= 2;
+  while (sizeof(float) * TB * (size_t)(HID / ks) > 64 * 1024 && ks * 2 <= ctx->splitk_max &&
+         HID % (ks * 2 * 128) == 0)
+    ks *= 2;
+  if (sizeof(float) * TB * (size_t)(HID / ks) > 64 * 1024 || sizeof(float) * TB * (size_t)R > 64 * 1024)
+    return FM_ERR_UNSUPPORTED;
+  fm_status s = launch_gemv<TB>(ctx->w_down, Md, HID, ks, hidden, HID, 0, 0, B, ctx->a_part, st);
+  if (s != FM_OK) return s;
+  const float w_scale = (float)(1.0 / sqrt((double)c.head_dim * (double)c.n_heads));
+  cudaError_t e = launch_overlapped(qnorm_kernel, dim3(B, L), dim3(kNormThreads), 0, st, (const float*)ctx->a_part,
+                                    ks, StreamK{}, B, L, R, (int)c.n_heads, (const float*)ctx->q_norm,
+                                    c.rms_eps, w_scale, positions, (const double*)ctx->rope_freq,
+                                    c.rope_dim / 2, ctx->r_norm, fused_w, ctx->rope_cs, (float*)nullptr,
+                                    (float*)nullptr);
+  note_launch();
+  if (e != cudaSuccess) return record_cuda_error(e);
+  s = launch_gemv<TB>(ctx->w_up, Mu, R, 1, ctx->r_norm, (int64_t)L * R, R, kHeads * kHeadDim, B, ctx->up_part,
+                      st);
+  if (s != FM_OK) return s;
+  const int warps = B * L * kHeads;
+  e = launch_overlapped(qup_finish_kernel, dim3((warps + kThreads / 32 - 1) / (kThreads / 32)), dim3(kThreads), 0,
+                        st, (const float*)ctx->up_part, StreamK{}, 1, (int64_t)B * Mu, B, L,
+                        (const float*)ctx->rope_cs, q);
+  note_launch();
+  return e == cudaSuccess ? check_launch() : record_cuda_error(e);
 }
 
 template <int TN>
@@ -798,15 +955,10 @@ void launch_split(const float* x, float* hi, float* lo, int64_t n, cudaStream_t 
 template <int BN>
 fm_status launch_tc_gemm_bn(fm_ctx* ctx, const void* wmap, const void* xh, const void* xl, const TcGemmArgs& a,
                             cudaStream_t st) {
-  static int configured_dev = -1;
+  static PerDeviceOnce smem_set;
   constexpr uint32_t smem = TcCfg<BN>::kSmem;
   static_assert(smem <= 227u * 1024u, "shared memory");
-  if (configured_dev != ctx->device) {
-    if (cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return check_launch();
-    configured_dev = ctx->device;
-  }
+  if (fm_status s = smem_limit_once(smem_set, ctx->device, tc_gemm_kernel<BN>, (int)smem)) return s;
   tc_gemm_kernel<BN><<<a.sk.G, kTcThreads, smem, st>>>(*reinterpret_cast<const CUtensorMap*>(wmap),
                                                        *reinterpret_cast<const CUtensorMap*>(xh),
                                                        *reinterpret_cast<const CUtensorMap*>(xl), a);
@@ -869,7 +1021,7 @@ fm_status launch_query_prep_tc(fm_ctx* ctx, const float* hidden, const int64_t* 
                                ctx->a_part, &sk_d, st);
   if (s != FM_OK) return s;
   const float w_scale = (float)(1.0 / sqrt((double)c.head_dim * (double)c.n_heads));
-  qnorm_kernel<<<dim3(B, L), kThreads, 0, st>>>(ctx->a_part, 0, sk_d, B, L, R, c.n_heads, ctx->q_norm,
+  qnorm_kernel<<<dim3(B, L), kNormThreads, 0, st>>>(ctx->a_part, 0, sk_d, B, L, R, c.n_heads, ctx->q_norm,
                                                  c.rms_eps, w_scale, positions, ctx->rope_freq, c.rope_dim / 2,
                                                  ctx->r_norm, fused_w, ctx->rope_cs, ctx->r_hi, ctx->r_lo);
   note_launch();
@@ -879,7 +1031,7 @@ fm_status launch_query_prep_tc(fm_ctx* ctx, const float* hidden, const int64_t* 
   if (s != FM_OK) return s;
   const int warps = B * L * kHeads;
   qup_finish_kernel<<<(warps + kThreads / 32 - 1) / (kThreads / 32), kThreads, 0, st>>>(
-      ctx->up_part, sk_u, (int64_t)B * Mu, B, L, ctx->rope_cs, q);
+      ctx->up_part, sk_u, 0, (int64_t)B * Mu, B, L, ctx->rope_cs, q);
   note_launch();
   return check_launch();
 }
@@ -901,6 +1053,10 @@ fm_status launch_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* pos
   // the tensor-core path (three-pass TF32) takes over; up to 8 rows the
   // CUDA-core GEMVs are bound by the weight bytes, which both paths read once.
   if (ctx->tc_ok && B > 8) return launch_query_prep_tc(ctx, hidden, positions, B, q, fused_w, st);
+  if (B == 1) return launch_query_prep_gemv<1>(ctx, hidden, positions, B, q, fused_w, st);
+  if (B == 2) return launch_query_prep_gemv<2>(ctx, hidden, positions, B, q, fused_w, st);
+  if (B <= 4) return launch_query_prep_gemv<4>(ctx, hidden, positions, B, q, fused_w, st);
+  if (B <= 8) return launch_query_prep_gemv<8>(ctx, hidden, positions, B, q, fused_w, st);
   const fm_config& c = ctx->cfg;
   const int M = c.n_layers * (c.q_lora_rank + c.n_heads);
   const int mtiles = (M + BM - 1) / BM;
@@ -920,7 +1076,7 @@ fm_status launch_query_prep(fm_ctx* ctx, const float* hidden, const int64_t* pos
     launch_qdown<8>(ctx, hidden, B, ksplit, st);
 
   const float w_scale = (float)(1.0 / sqrt((double)c.head_dim * (double)c.n_heads));
-  qnorm_kernel<<<dim3(B, c.n_layers), kThreads, 0, st>>>(
+  qnorm_kernel<<<dim3(B, c.n_layers), kNormThreads, 0, st>>>(
       ctx->a_part, ksplit, StreamK{}, B, c.n_layers, c.q_lora_rank, c.n_heads, ctx->q_norm, c.rms_eps,
       w_scale, positions, ctx->rope_freq, c.rope_dim / 2, ctx->r_norm, fused_w, ctx->rope_cs, nullptr,
       nullptr);

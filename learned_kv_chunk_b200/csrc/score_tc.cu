@@ -26,25 +26,28 @@
 //    reads with the accumulators, so no scale is read from global memory.  A
 //    stage goes back to the key loader as soon as it has been read, so the
 //    ring holds little besides keys in flight from HBM;
-//  * two single threads pace the pass: the key loader (its copies in flight
-//    set the HBM rate) and the MMA issuer (each tcgen05.mma, commit or
-//    mbarrier probe costs it tens of cycles, so an item is four MMAs with
-//    descriptors advanced by constant adds, and per-item work is kept off
-//    every role: scales travel through TMEM instead of as scattered global
-//    loads, which doubled the L2 request count).  Warp w runs on scheduler
-//    w % 4 and may only touch TMEM lanes 32*(w % 4) .. +31, so every
-//    scheduler hosts one transform warp and two epilogue warps;
-//  * warp roles (16 warps): 0 key loader, 1 MMA issuer, 2 TMEM owner + query
-//    loader, 4-7 transform, 8-11 and 12-15 two epilogue groups (one lane
+//  * single threads pace the pass: the key loader (its copies in flight set
+//    the HBM rate) and the MMA issuers (each tcgen05.mma, commit or mbarrier
+//    probe costs its thread tens of cycles, so an item is four MMAs with
+//    descriptors advanced by constant adds, two issuing threads on two
+//    schedulers share the items, and per-item work is kept off every role:
+//    scales travel through TMEM instead of as scattered global loads, which
+//    doubled the L2 request count).  Warp w runs on scheduler w % 4 and may
+//    only touch TMEM lanes 32*(w % 4) .. +31, so every scheduler hosts one
+//    transform warp and two epilogue warps;
+//  * warp roles (16 warps): 0 key loader, 1 and 3 MMA issuers (one per
+//    epilogue group), 2 TMEM owner + query loader, 4-7 transform, 8-11 and
+//    12-15 two epilogue groups (one lane
 //    quarter per warp, all 64 heads of a chunk row), each with one
 //    accumulator stage.  Units are taken in pairs from the same row,
 //    the first for group 0 and the second for group 1, and their items are
 //    issued layer by layer alternately, (u0,l0) (u1,l0) (u0,l1) (u1,l1) ...,
 //    so each group has a whole MMA to drain its stage before it is needed
 //    again.  Every ring index is advanced incrementally (no runtime division
-//    in any loop).
-#include <cstdlib>
-
+//    in any loop);
+//  * the pass is launched to overlap the query-packing kernel ahead of it:
+//    set-up and the key stream start at once, and only the query loader and
+//    the epilogue (the head weights) wait for the packing kernel's writes.
 #include "fm_internal.cuh"
 
 namespace fm {
@@ -55,29 +58,34 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kRawBytes = kTile * kRecord;  // 16896, a multiple of 128
 constexpr int kMmaM = kTile;                // MMA rows = TMEM lanes = chunks of a tile
 constexpr int kQuarters = 4;                // TMEM lane quarters (32 lanes, one warp each)
-constexpr int kWarpLoader = 0, kWarpMma = 1, kWarpQ = 2;
+constexpr int kWarpLoader = 0, kWarpMma = 1, kWarpQ = 2, kWarpMma2 = 3;
 constexpr int kWarpXform0 = 4, kWarpEpi0 = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACols = 32;  // 128 e4m3 bytes per row = 32 columns per key tile
 constexpr uint32_t kPieceBytes = kHeads * kHeadDim;  // one query piece of one layer
 
 // TMEM columns: accumulator of group g at [g * P*64, (g+1) * P*64), key tiles
-// after them, and the last 32 columns a ring of per-chunk scales (one column
-// per item, slot = item index mod 32).
+// after them, and the last 32 columns two rings of per-chunk scales, 16
+// columns per epilogue group: the scale of the g-th group's n-th key tile
+// (item, or unit with shared keys) in column kScaleCol + 16 g + n mod 16.
 constexpr uint32_t kScaleSlots = 32;
 constexpr uint32_t kScaleCol = kTmemCols - kScaleSlots;
+constexpr uint32_t kGroupSlots = kScaleSlots / 2;
 template <int P>
 constexpr uint32_t acc_cols() { return (uint32_t)P * kHeads; }
 template <int P>
 constexpr uint32_t a_col_base() { return 2u * acc_cols<P>(); }
 template <int P>
 constexpr uint32_t a_stages() { return (kScaleCol - a_col_base<P>()) / kACols; }  // 7 (P=2), 3 (P=3)
-// A scale slot is rewritten 32 items after it was written.  The item that
-// rewrites it waits for its key stage, i.e. for the MMA of the item NA before
-// it, and that MMA was issued only after both epilogue groups had loaded
-// (scale included) every item up to two before it; so NA + 2 < 32 keeps every
-// scale alive until it has been read.
-static_assert(a_stages<2>() + 2 < kScaleSlots && a_stages<3>() + 2 < kScaleSlots, "scale ring too short");
+// A group's scale slot is rewritten 16 of that group's key tiles later.  The
+// transform stores tile x only after the key stage of the tile NA before it
+// (in the CTA's order) was released, so after every tile up to x - NA had all
+// its MMAs issued.  With 16 > NA + 1, at least one tile of the same group lies
+// between the slot's previous tile y and x - NA, and that group's issuer
+// issued it only after the group's epilogue had released y -- scale included.
+// Each group's ring depends on its own epilogue only, whatever the other group
+// does (a row's lone last tile leaves the second group idle for that pair).
+static_assert(a_stages<2>() + 1 < kGroupSlots && a_stages<3>() + 1 < kGroupSlots, "scale ring too short");
 
 
 struct Layout {
@@ -211,7 +219,7 @@ __device__ __forceinline__ float head_sum32(const HeadCols<P>& c, const float* _
       float dx, dy;
       f2_unpack(d, dx, dy);
       const float2 ww = *reinterpret_cast<const float2*>(w + 2 * j);
-      const uint64_t rr = f2_pack(fmaxf(dx, 0.f), fmaxf(dy, 0.f));
+      const uint64_t rr = f2_pack(fmax_nan(dx, 0.f), fmax_nan(dy, 0.f));
       acc = f2_fma(rr, f2_pack(ww.x, ww.y), acc);  // one chain: fewer registers, same issue count
     }
     float a0, a1;
@@ -222,12 +230,16 @@ __device__ __forceinline__ float head_sum32(const HeadCols<P>& c, const float* _
   for (int i = 0; i < 32; ++i) {
     float d = fmaf(c.at(1, i), kInv16, c.at(0, i));
     if constexpr (P == 3) d = fmaf(c.at(2, i), kInv256, d);
-    acc = fmaf(fmaxf(d * s, 0.f), w[i], acc);
+    acc = fmaf(fmax_nan(d * s, 0.f), w[i], acc);
   }
   return acc;
 }
 
-template <int P, bool DUMP>
+// SK (shared keys): every layer's pointer is the same key tensor, so each
+// unit's tile is copied and stored into TMEM once and every layer's MMAs read
+// it; the key ring, the TMEM key stages and the scale slots then go per unit
+// instead of per (unit, layer).
+template <int P, bool DUMP, bool SK>
 __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int NR) {
   extern __shared__ uint8_t smem_raw[];
   constexpr uint32_t ACCW = acc_cols<P>();
@@ -236,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
   const Layout lay = make_layout(args.L, P, NR, NA);
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int L = args.L;
+  const int LK = SK ? 1 : L;  // key tiles copied per unit
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr uint32_t kQLayerBytes = (uint32_t)P * kPieceBytes;
 
@@ -265,8 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
     }
     for (int g = 0; g < 2; ++g) { mbar_init(&B_.acc_full[g], 1); mbar_init(&B_.acc_empty[g], kQuarters); }
     mbar_init(B_.q_full, 1);
-    mbar_init(B_.q_empty, 1);
-    mbar_init(B_.done, 1);
+    mbar_init(B_.q_empty, 2);                // both MMA issuers' commits
+    mbar_init(B_.done, 2);
     *sAbort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -312,14 +325,14 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       bool ok = true;
       for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); ok && pw.valid() && !*sAbort;
            pw.next()) {
-        for (int l = 0; l < L && ok; ++l) {
+        for (int l = 0; l < LK && ok; ++l) {
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             if (j == 1 && !pw.has1) break;
             const Unit U = j == 0 ? pw.u[0] : pw.u[1];
             const int nrem = min(kTile, U.nv - U.t * kTile);
             const uint32_t bytes = (uint32_t)((nrem + 3) & ~3) * kRecord;
-            ok = mbar_wait_bounded(&B_.raw_empty[raw.stage], raw.phase ^ 1, sAbort, args.err);
+            ok = mbar_wait_bounded(&B_.raw_empty[raw.stage], raw.phase ^ 1, sAbort, args.err, args.wait_ns);
             if (!ok) break;
             mbar_arrive_expect_tx(&B_.raw_full[raw.stage], bytes);
             const uint8_t* src = args.comp_k[l] + (int64_t)U.b * args.row_stride + (int64_t)U.t * kRawBytes;
@@ -339,13 +352,14 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
     }
   } else if (warp == kWarpQ) {
     // ------------------------------------------------ query operand loader
-    if (lane == 0) {
+    if (lane == 0 && !args.withhold_query) {
+      grid_dependency_wait();  // the query image is written by the packing kernel ahead
       int cur = -1;
       uint32_t loads = 0;
       for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); pw.valid() && !*sAbort; pw.next()) {
         const int b = pw.u[0].b;
         if (b == cur) continue;
-        if (loads > 0 && !mbar_wait_bounded(B_.q_empty, (loads - 1) & 1, sAbort, args.err)) break;
+        if (loads > 0 && !mbar_wait_bounded(B_.q_empty, (loads - 1) & 1, sAbort, args.err, args.wait_ns)) break;
         mbar_arrive_expect_tx(B_.q_full, (uint32_t)L * kQLayerBytes);
         for (int l = 0; l < L; ++l)
           bulk_g2s(sQ + (size_t)l * kQLayerBytes, args.qpack + ((size_t)b * L + l) * kQLayerBytes,
@@ -355,9 +369,16 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       }
       if (loads > 0) mbar_drain(B_.q_full, (loads - 1) & 1, args.err);
     }
-  } else if (warp == kWarpMma) {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp == kWarpMma || warp == kWarpMma2) {
+    // --------------------------------------------------------- MMA issuers
+    // Two issuing threads on two schedulers, one per epilogue group: thread
+    // `me` issues the items of group `me` (the pair's unit u[me]) into that
+    // group's accumulator.  A tcgen05.mma costs its issuing thread tens of
+    // cycles, so two issuers double the issue rate; each commit tracks only
+    // its own thread's MMAs, and both walk every item to keep the key ring's
+    // stage and phase.
     if (lane == 0) {
+      const int me = warp == kWarpMma ? 0 : 1;
       constexpr uint32_t idesc = idesc_e4m3_f32(kMmaM, (int)ACCW);
       // B descriptors: the start-address field counts 16-byte units, so the
       // layer and K-step offsets are plain adds (the field cannot carry: the
@@ -371,38 +392,49 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); ok && pw.valid() && !*sAbort;) {
         const int b = pw.u[0].b;
         if (b != cur) {
-          if (!mbar_wait_bounded(B_.q_full, rows & 1, sAbort, args.err)) break;
+          if (!mbar_wait_bounded(B_.q_full, rows & 1, sAbort, args.err, args.wait_ns)) break;
           ++rows;
           cur = b;
         }
         uint64_t bd = bdesc0;
+        Ring su = ast;  // shared keys: the key stage of unit u[me]
+        if (SK && me == 1) su.advance();
         for (int l = 0; l < L && ok; ++l, bd += kLayerStep) {
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             if (j == 1 && !pw.has1) break;
+            if (j != me) {
+              if (!SK) ast.advance();
+              continue;
+            }
+            const Ring& as = SK ? su : ast;
             const uint32_t ph = j == 0 ? ph0 : ph1;
-            ok = mbar_wait_bounded(&B_.a_full[ast.stage], ast.phase, sAbort, args.err) &&
-                 mbar_wait_bounded(&B_.acc_empty[j], ph ^ 1, sAbort, args.err);
+            ok = ((SK && l > 0) || mbar_wait_bounded(&B_.a_full[as.stage], as.phase, sAbort, args.err, args.wait_ns)) &&
+                 mbar_wait_bounded(&B_.acc_empty[j], ph ^ 1, sAbort, args.err, args.wait_ns);
             if (!ok) break;
             tc_fence_after();
             const uint32_t d = tmem_base + (uint32_t)j * ACCW;
-            const uint32_t a = tmem_base + ABASE + ast.stage * kACols;
+            const uint32_t a = tmem_base + ABASE + as.stage * kACols;
             umma_f8f6f4_ts(d, a, bd, idesc, 0u);
             umma_f8f6f4_ts(d, a + 8u, bd + kKStep, idesc, 1u);
             umma_f8f6f4_ts(d, a + 16u, bd + 2 * kKStep, idesc, 1u);
             umma_f8f6f4_ts(d, a + 24u, bd + 3 * kKStep, idesc, 1u);
-            umma_commit(&B_.a_empty[ast.stage]);  // the TMEM key tile may be overwritten
+            if (!SK || l == L - 1) umma_commit(&B_.a_empty[as.stage]);  // the TMEM key tile may be overwritten
             umma_commit(&B_.acc_full[j]);
             ++item;
-            ast.advance();
+            if (!SK) ast.advance();
             if (j == 0) ph0 ^= 1u; else ph1 ^= 1u;
           }
         }
         if (!ok) break;
+        if (SK) {  // the pair's units each held one key stage
+          ast.advance();
+          if (pw.has1) ast.advance();
+        }
         pw.next();
         if (!pw.valid() || pw.u[0].b != b) umma_commit(B_.q_empty);
       }
-      if (item > 0) {  // every issued MMA and commit retired before TMEM and smem go away
+      {  // every issued MMA and commit retired before TMEM and smem go away (both issuers arrive)
         umma_commit(B_.done);
         mbar_drain(B_.done, 0, args.err);
       }
@@ -412,20 +444,30 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
     // Thread `lane` of this warp owns one chunk row of the tile: it reads the
     // row's 128 key bytes (the 33-word row stride puts the 32 lanes of a load
     // in 32 different banks) and stores them to its TMEM lane.  The four
-    // warps run independently; each arrives once per item on both barriers.
-    // Items arrive in the loader's order, so only their number matters here.
+    // warps run independently; each arrives once per key tile on both
+    // barriers.  Tiles arrive in the loader's order (pairs, then the layers
+    // copied per unit, then the pair's units), which also gives each tile's
+    // epilogue group and so its scale slot.
     const uint32_t quarter = (uint32_t)warp & 3u;
     const uint32_t row = quarter * 32u + (uint32_t)lane;
     const uint32_t lane_base = tmem_base + ((quarter * 32u) << 16);
     Ring raw(NR), ast(NA);
-    const int64_t items = count * L;
-    for (int64_t i = 0; i < items; ++i, raw.advance(), ast.advance()) {
+    uint32_t gtiles[2] = {0u, 0u};  // key tiles of each group so far
+    bool go = true;
+    for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); go && pw.valid(); pw.next())
+    for (int l = 0; l < LK && go; ++l)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      if (j == 1 && !pw.has1) break;
       int good = 1;
       if (lane == 0)
-        good = mbar_wait_bounded(&B_.raw_full[raw.stage], raw.phase, sAbort, args.err) &&
-               mbar_wait_bounded(&B_.a_empty[ast.stage], ast.phase ^ 1, sAbort, args.err);
+        good = mbar_wait_bounded(&B_.raw_full[raw.stage], raw.phase, sAbort, args.err, args.wait_ns) &&
+               mbar_wait_bounded(&B_.a_empty[ast.stage], ast.phase ^ 1, sAbort, args.err, args.wait_ns);
       good = __shfl_sync(0xffffffffu, good, 0);
-      if (!good) break;
+      if (!good) {
+        go = false;
+        break;
+      }
       const uint32_t* src =
           reinterpret_cast<const uint32_t*>(sRaw + (size_t)raw.stage * kRawBytes + row * kRecord);
       uint32_t v[32];
@@ -434,28 +476,32 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       const uint32_t scale_bits = src[32];  // the record's little-endian fp32 scale
       tc_fence_after();  // the MMA that last read this TMEM stage has retired (a_empty)
       tmem_st32_st1_wait(lane_base + ABASE + ast.stage * kACols, v,
-                         lane_base + kScaleCol + ((uint32_t)i & (kScaleSlots - 1)), scale_bits);
+                         lane_base + kScaleCol + (uint32_t)j * kGroupSlots + (gtiles[j] & (kGroupSlots - 1)),
+                         scale_bits);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&B_.raw_empty[raw.stage]);
         mbar_arrive(&B_.a_full[ast.stage]);
       }
+      ++gtiles[j];
+      raw.advance();
+      ast.advance();
     }
   } else if (warp >= kWarpEpi0) {
     // ------------------------------------------------------------ epilogue
+    grid_dependency_wait();  // the head weights are written by the packing kernel ahead
     const int group = (warp - kWarpEpi0) >> 2;
     const int quarter = warp & 3;
     const int ew = group * kQuarters + quarter;  // 0..7
     const int r = quarter * 32 + lane;           // row of the tile
     float* sWpw = sWp + ew * L * kHeads;
     const uint32_t col_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)group * ACCW;
-    const uint32_t scale_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + kScaleCol;
-    uint32_t ph = 0, gbase = 0;  // gbase: index of the pair's first item in the CTA's item order
+    const uint32_t scale_base =
+        tmem_base + ((uint32_t)(quarter * 32) << 16) + kScaleCol + (uint32_t)group * kGroupSlots;
+    uint32_t ph = 0, gtiles = 0;  // gtiles: this group's key tiles so far (its scale slots)
     int cur = -1;
     for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); pw.valid(); pw.next()) {
-      const uint32_t per = pw.has1 ? 2u : 1u, gb = gbase;  // items per layer in this pair
-      gbase += per * (uint32_t)L;
       if (group == 1 && !pw.has1) continue;
       const Unit U = group == 0 ? pw.u[0] : pw.u[1];
       if (U.b != cur) {  // this warp's private copy of the row's head weights
@@ -471,14 +517,15 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       float ens = 0.f;
       bool ok = true;
       for (int l = 0; l < L; ++l, ph ^= 1u) {
-        ok = mbar_wait_bounded(&B_.acc_full[group], ph, sAbort, args.err);
+        ok = mbar_wait_bounded(&B_.acc_full[group], ph, sAbort, args.err, args.wait_ns);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t item = gb + (uint32_t)l * per + (uint32_t)group;
+        // the scale slot of the key tile this item read (one tile per unit with shared keys)
+        const uint32_t slot = (gtiles + (SK ? 0u : (uint32_t)l)) & (kGroupSlots - 1);
         const float* w = sWpw + l * kHeads;
         HeadCols<P> c;
         uint32_t s_bits;
-        c.load_with(col_base, scale_base + (item & (kScaleSlots - 1)), &s_bits);
+        c.load_with(col_base, scale_base + slot, &s_bits);
         const float s = valid ? __uint_as_float(s_bits) : 0.f;  // rows past the tail hold stale bytes
         const bool nonneg = __all_sync(0xffffffffu, !(s < 0.f));
         if constexpr (DUMP) {
@@ -503,9 +550,10 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
         float score = 1.0f / (1.0f + __expf(-logit));
         if (!valid) score = 0.f;
         if (args.scores && in_row) args.scores[((size_t)l * args.B + U.b) * args.N + n] = score;
-        ens = (args.mode == FM_ENSEMBLE_MAX) ? (l == 0 ? score : fmaxf(ens, score)) : ens + score;
+        ens = (args.mode == FM_ENSEMBLE_MAX) ? (l == 0 ? score : fmax_nan(ens, score)) : ens + score;
       }
       if (!ok) break;
+      gtiles += SK ? 1u : (uint32_t)L;
       if (args.mode != FM_ENSEMBLE_MAX) ens = ens / (float)L;
       if (!valid) ens = 0.f;
       if (in_row) {
@@ -537,16 +585,15 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
   }
 }
 
-template <int P, bool DUMP>
+template <int P, bool DUMP, bool SK>
 fm_status launch_score_p(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t st) {
-  static int configured_dev = -1;
+  static PerDeviceOnce smem_set;
   int max_smem = 0;
   if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, ctx->device) !=
       cudaSuccess)
     return check_launch();
   // deepest key ring that fits: every stage is keys in flight
   int NR = 16;
-  if (const char* e = getenv("FM_RAW_STAGES")) NR = atoi(e) < 2 ? 2 : atoi(e);
   constexpr int NA = (int)a_stages<P>();
   Layout lay = make_layout(a.L, P, NR, NA);
   while (lay.total > (uint32_t)max_smem && NR > 2) {
@@ -554,28 +601,31 @@ fm_status launch_score_p(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t st) {
     lay = make_layout(a.L, P, NR, NA);
   }
   if (lay.total > (uint32_t)max_smem) return FM_ERR_UNSUPPORTED;
-  if (configured_dev != ctx->device) {
-    if (cudaFuncSetAttribute(score_kernel<P, DUMP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             max_smem) != cudaSuccess)
-      return check_launch();
-    configured_dev = ctx->device;
-  }
+  if (fm_status s = smem_limit_once(smem_set, ctx->device, score_kernel<P, DUMP, SK>, max_smem)) return s;
   const int64_t units = (int64_t)a.B * ((a.N + kTile - 1) / kTile);  // upper bound
   int grid = ctx->num_sms;
   if (units < grid) grid = (int)(units > 0 ? units : 1);
-  score_kernel<P, DUMP><<<grid, kThreads, lay.total, st>>>(a, NR);
+  // the packing kernel ahead of this one writes only the query image and the
+  // head weights, which the query loader and the epilogue wait for; the key
+  // stream starts while it runs
+  const cudaError_t e = launch_overlapped(score_kernel<P, DUMP, SK>, dim3(grid), dim3(kThreads), lay.total, st, a, NR);
   note_launch();
-  return check_launch();
+  return e == cudaSuccess ? check_launch() : record_cuda_error(e);
 }
 
 }  // namespace
 
 fm_status launch_score(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t st) {
   if (a.dbg_out)
-    return ctx->cfg.q_pieces == 3 ? launch_score_p<3, true>(ctx, a, st)
-                                  : launch_score_p<2, true>(ctx, a, st);
-  return ctx->cfg.q_pieces == 3 ? launch_score_p<3, false>(ctx, a, st)
-                                : launch_score_p<2, false>(ctx, a, st);
+    return ctx->cfg.q_pieces == 3 ? launch_score_p<3, true, false>(ctx, a, st)
+                                  : launch_score_p<2, true, false>(ctx, a, st);
+  bool shared = a.L > 1;
+  for (int l = 1; l < a.L; ++l) shared = shared && a.comp_k[l] == a.comp_k[0];
+  if (shared)
+    return ctx->cfg.q_pieces == 3 ? launch_score_p<3, false, true>(ctx, a, st)
+                                  : launch_score_p<2, false, true>(ctx, a, st);
+  return ctx->cfg.q_pieces == 3 ? launch_score_p<3, false, false>(ctx, a, st)
+                                : launch_score_p<2, false, false>(ctx, a, st);
 }
 
 }  // namespace fm

@@ -140,7 +140,7 @@ __global__ void ensemble_kernel(const float* __restrict__ scores, int L, int64_t
        i += (int64_t)gridDim.x * blockDim.x) {
     float e = scores[i];
     if (mode == FM_ENSEMBLE_MAX) {
-      for (int l = 1; l < L; ++l) e = fmaxf(e, scores[(int64_t)l * BN + i]);
+      for (int l = 1; l < L; ++l) e = fmax_nan(e, scores[(int64_t)l * BN + i]);
     } else {
       for (int l = 1; l < L; ++l) e = e + scores[(int64_t)l * BN + i];
       e = e / (float)L;
@@ -659,6 +659,7 @@ fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, in
                       void* ws, size_t ws_size, cudaStream_t st) {
   const int nblk = (int)(((int64_t)N + kChunk - 1) / kChunk);
   if (ws_size < ws_bytes(B, nblk)) return FM_ERR_INVALID_ARG;
+  if (topk_use_cluster(N)) return launch_topk_cluster(ens, n_valid, B, N, k, keep, st);
   Workspace w = carve(ws, B, nblk);
   const int C = cand_cap(N);
   const bool fast = ws_size >= fast_ws_bytes(B, nblk, C) && 2 * (int64_t)k + 1024 <= C;
@@ -666,15 +667,12 @@ fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, in
   note_launch();
   dim3 grid(nblk, B);
   if (fast) {
-    static int configured_dev = -1;
+    static PerDeviceOnce smem_set;
     int dev = 0;
     cudaGetDevice(&dev);
-    if (configured_dev != dev) {
-      if (cudaFuncSetAttribute(topk_fastsel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)(2 * sizeof(uint32_t) * kCandMax)) != cudaSuccess)
-        return check_launch();
-      configured_dev = dev;
-    }
+    if (fm_status s = smem_limit_once(smem_set, dev, topk_fastsel_kernel,
+                                      (int)(2 * sizeof(uint32_t) * kCandMax)))
+      return s;
     const FastWs f = carve_fast(ws, B, nblk, C);
     topk_sample_kernel<<<B, kBlkThreads, sizeof(uint32_t) * kSample, st>>>(w, f, ens, N);
     topk_collect_kernel<<<grid, kThreads, 0, st>>>(w, f, C, ens, N, keep);

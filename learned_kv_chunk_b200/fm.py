@@ -47,6 +47,21 @@ class fm_level2_desc(ctypes.Structure):
                 ("out_count", ctypes.c_void_p)]
 
 
+class fm_host_batch(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("hidden", ctypes.c_void_p),
+                ("positions", ctypes.c_void_p), ("comp_k", ctypes.c_void_p * 4),
+                ("row_stride_bytes", ctypes.c_int64), ("n_valid", ctypes.c_void_p), ("mode", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("thr", ctypes.c_float), ("keep_topk", ctypes.c_void_p),
+                ("keep_thr", ctypes.c_void_p)]
+
+
+class fm_device_staging(ctypes.Structure):
+    _fields_ = [("comp_k", ctypes.c_void_p * 4), ("hidden", ctypes.c_void_p), ("positions", ctypes.c_void_p),
+                ("n_valid", ctypes.c_void_p), ("q", ctypes.c_void_p), ("fused_w", ctypes.c_void_p),
+                ("ens", ctypes.c_void_p), ("keep_topk", ctypes.c_void_p), ("keep_thr", ctypes.c_void_p),
+                ("topk_ws", ctypes.c_void_p), ("topk_ws_bytes", ctypes.c_size_t)]
+
+
 class FMError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -75,6 +90,7 @@ def _load():
         "fm_topk_workspace_bytes_fast": (S, [I, I]),
         "fm_select_topk": (I, [P, P, I, I, I, P, P, S, P]),
         "fm_select_threshold": (I, [P, P, I, I, F, P, P]),
+        "fm_retrieve_host": (I, [P, ctypes.POINTER(fm_host_batch), ctypes.POINTER(fm_device_staging), P]),
         "fm_select_topk_static": (I, [P, P, I, I, I, P, P]),
         "fm_compact_workspace_bytes": (S, [I, I]),
         "fm_compact_mask": (I, [P, I, I, I, P, P, P, S, P]),
@@ -95,6 +111,9 @@ def _load():
         "fm_strerror": (ctypes.c_char_p, [I]),
         "fm_last_cuda_error": (I, []),
         "fm_launch_count": (ctypes.c_uint64, []),
+        "fm_debug_fail_alloc": (None, [I]),
+        "fm_debug_live_allocations": (I64, []),
+        "fm_debug_stall_next_score": (I, [P, ctypes.c_uint64]),
         "fm_debug_tile_dots": (I, [P, P, I64, I, I, P, P, I, I, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -608,35 +627,63 @@ class Retriever:
         return out, e
 
     def retrieve_from_host(self, hidden, positions, comp_k, n_valid=None, mode="max", top_k=None,
-                           threshold=None, N=None, device_buffers: Optional[dict] = None):
-        """The whole path for inputs that live in (pinned) host memory: copies
-        them to device buffers, runs retrieve() and copies the keep masks back.
-        Returns (keep_topk, keep_thr) as host tensors (either may be None)."""
+                           threshold=None, N=None, device_buffers: Optional[dict] = None, sync=True):
+        """The whole path for inputs in (pinned) host memory through the C call
+        fm_retrieve_host: host inputs copied to device staging buffers, query
+        prep, scoring, top-K, masks copied back.  Returns (keep_topk, keep_thr)
+        as host uint8 tensors (either may be None).  `device_buffers` (a dict)
+        keeps the staging buffers and the host masks between calls."""
         dev = torch.device("cuda", self.device)
         buf = device_buffers if device_buffers is not None else {}
-        def stage(name, t):
+        B, N_pad, rec = comp_k[0].shape
+        N = N_pad if N is None else N
+        for t in list(comp_k) + [hidden, positions] + ([n_valid] if n_valid is not None else []):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError("fm_retrieve_host takes contiguous host tensors")
+
+        def dbuf(name, shape, dtype):
             d = buf.get(name)
-            if d is None or d.shape != t.shape or d.dtype != t.dtype:
-                d = buf[name] = torch.empty(t.shape, dtype=t.dtype, device=dev)
-            d.copy_(t, non_blocking=True)
+            if d is None or tuple(d.shape) != tuple(shape) or d.dtype != dtype:
+                d = buf[name] = torch.empty(shape, dtype=dtype, device=dev)
             return d
-        h = stage("hidden", hidden)
-        p = stage("positions", positions)
-        keys = [stage(f"keys{l}", t) for l, t in enumerate(comp_k)]
-        nv = stage("n_valid", n_valid) if n_valid is not None else None
-        ens, keep_topk, keep_thr = self.retrieve(h, keys, p, nv, mode, top_k, threshold, N)
-        out = []
-        for name, t in (("out_topk", keep_topk), ("out_thr", keep_thr)):
-            if t is None:
-                out.append(None)
-                continue
-            o = buf.get(name)
-            if o is None or o.shape != t.shape:
-                o = buf[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-            o.copy_(t, non_blocking=True)
-            out.append(o)
-        torch.cuda.current_stream().synchronize()
-        return out[0], out[1]
+
+        def hbuf(name, shape):
+            h = buf.get(name)
+            if h is None or tuple(h.shape) != tuple(shape):
+                h = buf[name] = torch.empty(shape, dtype=torch.uint8, pin_memory=True)
+            return h
+
+        st = fm_device_staging()
+        for l, t in enumerate(comp_k):
+            st.comp_k[l] = dbuf(f"keys{l}", t.shape, torch.uint8).data_ptr()
+        st.hidden = dbuf("hidden", hidden.shape, torch.float32).data_ptr()
+        st.positions = dbuf("positions", positions.shape, torch.int64).data_ptr()
+        st.n_valid = dbuf("n_valid", (B,), torch.int32).data_ptr()
+        st.q = dbuf("q", (B, self.L, 64, 128), torch.float32).data_ptr()
+        st.fused_w = dbuf("fused_w", (B, self.L, 64), torch.float32).data_ptr()
+        st.ens = dbuf("ens", (B, N), torch.float32).data_ptr()
+        st.keep_topk = dbuf("keep_topk", (B, N), torch.uint8).data_ptr()
+        st.keep_thr = dbuf("keep_thr", (B, N), torch.uint8).data_ptr()
+        ws = dbuf("topk_ws", (fm_topk_workspace_bytes_fast(B, N),), torch.uint8)
+        st.topk_ws, st.topk_ws_bytes = ws.data_ptr(), ws.numel()
+        hb = fm_host_batch()
+        hb.B, hb.N = B, N
+        hb.hidden, hb.positions = hidden.data_ptr(), positions.data_ptr()
+        for l, t in enumerate(comp_k):
+            hb.comp_k[l] = t.data_ptr()
+        hb.row_stride_bytes = N_pad * rec
+        hb.n_valid = n_valid.data_ptr() if n_valid is not None else None
+        hb.mode = MODES[mode]
+        hb.top_k = int(top_k) if top_k is not None else 0
+        hb.thr = 0.0 if threshold is None else float(threshold)
+        out_topk = hbuf("out_topk", (B, N)) if top_k is not None else None
+        out_thr = hbuf("out_thr", (B, N)) if threshold is not None else None
+        hb.keep_topk = out_topk.data_ptr() if out_topk is not None else None
+        hb.keep_thr = out_thr.data_ptr() if out_thr is not None else None
+        _check(_lib.fm_retrieve_host(self._h, ctypes.byref(hb), ctypes.byref(st), _stream()), "fm_retrieve_host")
+        if sync:
+            self.fm_sync_status()
+        return out_topk, out_thr
 
     # the pages' calls, composed (README "Usage")
     def retrieve(self, hidden, comp_k, positions, n_valid=None, mode="max", top_k=None,

@@ -245,13 +245,13 @@ def test_shared_keys_across_layers(retr, weights):
 
 
 def test_topk_candidate_path_and_its_fallbacks():
-    """Rows of 262144 scores, K = 4096, a workspace large enough for the
-    candidate path: ordinary scores (the path finishes the row), large scores
-    placed only where the threshold sample looks (too few candidates: the row
-    falls back to the histogram passes), all scores equal (too many
-    candidates), and a K-th value tied across the cut (ties need chunk order):
-    every mask must equal the selection rule."""
-    B, N, K = 4, 262144, 4096
+    """Rows of 300000 scores (past the one-kernel cluster form), K = 4096, a
+    workspace large enough for the candidate path: ordinary scores (the path
+    finishes the row), large scores placed only where the threshold sample
+    looks (too few candidates: the row falls back to the histogram passes),
+    all scores equal (too many candidates), and a K-th value tied across the
+    cut (ties need chunk order): every mask must equal the selection rule."""
+    B, N, K = 4, 300000, 4096
     g = torch.Generator().manual_seed(12)
     ens = torch.rand(B, N, generator=g) * 0.5
     sampled = (torch.arange(8192, dtype=torch.int64) * N) // 8192
@@ -267,3 +267,82 @@ def test_topk_candidate_path_and_its_fallbacks():
     ws_min = torch.zeros(fm.fm_topk_workspace_bytes(B, N), device=DEV, dtype=torch.uint8)
     keep_min = fm.fm_select_topk(ens.to(DEV), K, nv.to(DEV), workspace=ws_min)
     assert torch.equal(keep.cpu(), keep_min.cpu())
+
+
+def test_retrieve_host_call_matches_the_device_calls(retr, weights):
+    """fm_retrieve_host (host buffers in, host masks out, through the C ABI)
+    gives the masks of the device calls it composes, bit for bit."""
+    case = H.make_case(3, 2000, [2000, 1500, 333], seed=22, weights=weights)
+    hk = [k.pin_memory() for k in case.comp_k]
+    hh, hp, hn = case.hidden.pin_memory(), case.positions.pin_memory(), case.n_valid.pin_memory()
+    bufs = {}
+    for _ in range(2):  # the second call reuses the staging buffers
+        kt, kh = retr.retrieve_from_host(hh, hp, hk, hn, "mean", 100, 0.5, case.N, bufs)
+        ens, keep_topk, keep_thr = retr.retrieve(case.hidden.to(DEV), _dev(case.comp_k), case.positions.to(DEV),
+                                                 case.n_valid.to(DEV), "mean", 100, 0.5, case.N)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(kt.numpy(), keep_topk.cpu().numpy().astype(np.uint8))
+        np.testing.assert_array_equal(kh.numpy(), keep_thr.cpu().numpy().astype(np.uint8))
+        H.check_topk_near_oracle(kt.numpy().astype(bool), O.ensemble(H.oracle_scores(case), "mean"),
+                                 case.n_valid.numpy(), 100)
+
+
+@pytest.mark.parametrize("N", [1, 100, 4096, 16383, 16384, 16385, 65536, 131073, 262144])
+def test_topk_rule_across_row_lengths(N):
+    """Rows up to 16384 chunks (the one-kernel form) and past it (the
+    candidate path): ordinary scores, a K-th value tied across the cut, all
+    scores equal, ragged and empty rows, K past the row's length."""
+    g = torch.Generator().manual_seed(N)
+    B = 5
+    ens = torch.rand(B, N, generator=g)
+    ens[1] = torch.randint(0, 5, (N,), generator=g).float() / 5.0   # heavy ties
+    ens[2] = 0.25
+    nv = torch.tensor([N, N, N, max(0, N - 37), 0], dtype=torch.int32)
+    for k in sorted({1, 3, min(N, 512), max(1, N // 3), N + 5}):
+        keep = fm.fm_select_topk(ens.to(DEV), k, nv.to(DEV))
+        torch.cuda.synchronize()
+        H.check_topk_against_rule(keep.cpu().numpy(), ens.numpy(), nv.numpy(), k)
+
+
+@pytest.mark.parametrize("B", [2, 12])
+def test_query_prep_rank_2048(B):
+    """A Q_LORA_RANK of 2048 (the pages leave the rank open): the RMSNorm
+    block spans more than 2048 elements, on the GEMV path (B <= 8) and the
+    tensor-core path."""
+    weights = G.make_weights(4646, 3, rank=2048)
+    g = np.random.default_rng(47 + B)
+    hidden = g.standard_normal((B, G.HIDDEN)).astype(np.float32)
+    pos = g.integers(0, 1 << 20, size=B).astype(np.int64)
+    r = fm.Retriever(weights, device=0, max_batch=16, q_lora_rank=2048)
+    try:
+        q, w = r.fm_query_prep(torch.from_numpy(hidden).to(DEV), torch.from_numpy(pos).to(DEV))
+        torch.cuda.synchronize()
+        r.fm_sync_status()
+        qo, wo = H.oracle_queries(H.np_layers(weights), torch.from_numpy(hidden), torch.from_numpy(pos))
+        err = np.linalg.norm(q.cpu().numpy() - qo, axis=-1) / np.linalg.norm(qo, axis=-1)
+        assert err.max() < 2e-5, err.max()
+        np.testing.assert_allclose(w.cpu().numpy(), wo, rtol=1e-4, atol=1e-6)
+    finally:
+        r.close()
+
+
+@pytest.mark.parametrize("shared", [False, True], ids=["three_key_tensors", "shared_keys"])
+def test_rows_of_one_tile_between_longer_rows(retr, weights, shared):
+    """Rows of a single 128-chunk tile give pairs with one unit, so the second
+    epilogue group idles while the first runs on: each group's scale ring
+    must stay in step with its own tiles.  With shared keys every layer's
+    pointer is the one tensor (one key tile per unit for all layers)."""
+    nv = [1000, 100, 50, 128, 1, 129, 700, 3, 90, 400]
+    case = H.make_case(len(nv), 1000, nv, seed=23, weights=weights)
+    if shared:
+        case.comp_k = [case.comp_k[0]] * 3
+    keys = _dev(case.comp_k) if not shared else [case.comp_k[0].to(DEV)] * 3
+    q, w = _run_query(retr, case)
+    n_valid = case.n_valid.to(DEV)
+    s = retr.fm_score(keys, q, w, n_valid=n_valid, N=case.N).cpu().numpy()
+    ens, _, _ = retr.fm_score_fused(keys, q, w, mode="max", n_valid=n_valid, N=case.N)
+    torch.cuda.synchronize()
+    retr.fm_sync_status()
+    want = H.oracle_scores(case)
+    assert np.abs(s - want).max() <= H.SCORE_TOL
+    assert np.abs(ens.cpu().numpy() - O.ensemble(want, "max")).max() <= H.SCORE_TOL
