@@ -355,6 +355,15 @@ fm_status fm_gather_records(const void* src, int64_t src_row_stride_bytes, int n
                             const int32_t* idx, const int32_t* count, int B, int max_sel, void* dst,
                             int64_t dst_row_stride_bytes, cudaStream_t stream);
 
+/* fm_compact_mask followed by fm_gather_records of the listed entries, in one
+ * call: same arguments, same results (idx, count, and dst's slots
+ * j < min(count[b], max_sel)).  The kernel that writes a block's part of the
+ * index list also copies those records, so the list is not read back and the
+ * gather's launch is saved.  ws: fm_compact_workspace_bytes(B, N) bytes. */
+fm_status fm_recall_records(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx, int32_t* count,
+                            void* ws, size_t ws_bytes, const void* src, int64_t src_row_stride_bytes, int n_src,
+                            int64_t rec_bytes, void* dst, int64_t dst_row_stride_bytes, cudaStream_t stream);
+
 /* ---------------------------------------------------------------- Level 2
  * The model card's "How it works", Level 2: at every decode step a top-512
  * confined to the resident set, run inside a CUDA graph.  DS-V4's own Level-2

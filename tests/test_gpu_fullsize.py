@@ -79,3 +79,35 @@ def test_full_size_workload(wl):
         H.check_topk_near_oracle(k_gpu[b:b + 1], e_row, nv[b:b + 1], wl.top_k)
     finally:
         r.close()
+
+
+def test_full_size_shared_keys():
+    """The 64-row workload with one key tensor for every layer (the README
+    Usage signature taken literally, the shared-keys form of the pass): many
+    units per CTA, so the per-unit key stages and scale slots wrap many
+    times.  Sampled chunks against the oracle, the mask against the rule."""
+    wl = G.WORKLOADS[4]
+    inp = G.make_query_inputs(wl)
+    layers_np = H.np_layers(inp.weights)
+    q_o, w_o = H.oracle_queries(layers_np, inp.hidden, inp.positions)
+    key = G.make_keys(wl.seed(G.SEED_KEYS), [int(x) for x in inp.n_valid], wl.N, 1,
+                      H.plant_dirs(q_o)[:1], device=DEV)[0]
+    r = fm.Retriever(inp.weights, device=0, max_batch=wl.B)
+    try:
+        q, w = r.fm_query_prep(inp.hidden.to(DEV), inp.positions.to(DEV))
+        nv = inp.n_valid.to(DEV)
+        ens, _, scores = r.fm_score_fused([key] * 3, q, w, mode=wl.mode, n_valid=nv, N=wl.N, want_layers=True)
+        keep = fm.fm_select_topk(ens, wl.top_k, nv)
+        torch.cuda.synchronize()
+        r.fm_sync_status()
+        e_gpu = ens.cpu().numpy()
+        H.check_topk_against_rule(keep.cpu().numpy(), e_gpu, inp.n_valid.numpy(), wl.top_k)
+        rng = np.random.default_rng(404)
+        for b in (0, 17, 63):
+            idx = np.unique(np.concatenate([rng.integers(0, wl.N, 1500), [0, wl.N - 1]]))
+            host = key[b, idx].cpu().numpy()
+            s_o = np.stack([O.score_chunks(host, q_o[b, l], w_o[b, l]) for l in range(3)])
+            assert np.abs(scores[:, b, idx].cpu().numpy() - s_o).max() <= H.SCORE_TOL
+            assert np.abs(e_gpu[b, idx] - O.ensemble(s_o, wl.mode)).max() <= H.SCORE_TOL
+    finally:
+        r.close()
