@@ -397,10 +397,7 @@ def run_recall(args):
     def compact():
         fm.fm_compact_mask(keep, K, idx=idx, count=count, workspace=ws)
 
-    def step_dev():  # compaction and gather in one call (fm_recall_records)
-        fm.fm_recall_records(keep, K, src_dev, idx=idx, count=count, dst=dst, workspace=ws)
-
-    def step_dev_separate():
+    def step_dev():
         compact()
         fm.fm_gather_records(src_dev, idx, count, dst)
 
@@ -415,7 +412,6 @@ def run_recall(args):
     launches0 = fm.fm_launch_count()
     with sampler:
         t_step = _timed_flushed(step_dev, args.steps, flush_buf, stream)
-        t_separate = _timed_flushed(step_dev_separate, args.steps, flush_buf, stream)
         t_compact = _timed_flushed(compact, args.steps, flush_buf, stream)
         t_host = _timed_flushed(gather_host, max(3, args.steps // 10), flush_buf, stream)
     launches = fm.fm_launch_count() - launches0
@@ -442,10 +438,9 @@ def run_recall(args):
                       "l2": "flushed between steps (256 MB write)"},
            "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
                         "frac": round(ach / hbm_peak, 4), "traffic": None, "peak_kind": peak_kind,
-                        "kernel": "fm_recall_records: mask count + ordered index write with the gather (2 kernels)",
+                        "kernel": "compaction (2 kernels) + gather, one step",
                         "alg_bytes_per_step": alg_dev},
            "compact_ms": round(t_compact, 4),
-           "separate_calls_ms": round(t_separate, 4),
            "host_source": {"value": sel / (t_host / 1e3), "unit": "records/s", "gather_ms": round(t_host, 4),
                            "achieved_gbs": round(host_gbs, 2),
                            "h2d_copy_gbs": round(h2d_gbs, 2),

@@ -78,9 +78,12 @@ typedef struct fm_config {
   float rms_eps;          /* 1e-6 */
   int max_batch;          /* largest B any call on this context will pass */
   int q_pieces;           /* e4m3 pieces per query element in the tensor-core
-                             product: 2 (default; query split error ~2^-8
-                             relative, scores within ~5e-4 on the shipped
-                             workloads) or 3 (~2^-12, ~1e-5; about 15% slower) */
+                             product: 2 (default; the residual piece stored
+                             unscaled so the tensor core sums both into one
+                             accumulator; query split error ~2^-8 relative,
+                             scores within ~5e-4 on the shipped workloads) or
+                             3 (~2^-12, ~1e-5; one accumulator per piece,
+                             slower) */
 } fm_config;
 
 /* One layer's weights, fp32, row-major [out, in], no biases (README
@@ -355,15 +358,6 @@ fm_status fm_gather_records(const void* src, int64_t src_row_stride_bytes, int n
                             const int32_t* idx, const int32_t* count, int B, int max_sel, void* dst,
                             int64_t dst_row_stride_bytes, cudaStream_t stream);
 
-/* fm_compact_mask followed by fm_gather_records of the listed entries, in one
- * call: same arguments, same results (idx, count, and dst's slots
- * j < min(count[b], max_sel)).  The kernel that writes a block's part of the
- * index list also copies those records, so the list is not read back and the
- * gather's launch is saved.  ws: fm_compact_workspace_bytes(B, N) bytes. */
-fm_status fm_recall_records(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx, int32_t* count,
-                            void* ws, size_t ws_bytes, const void* src, int64_t src_row_stride_bytes, int n_src,
-                            int64_t rec_bytes, void* dst, int64_t dst_row_stride_bytes, cudaStream_t stream);
-
 /* ---------------------------------------------------------------- Level 2
  * The model card's "How it works", Level 2: at every decode step a top-512
  * confined to the resident set, run inside a CUDA graph.  DS-V4's own Level-2
@@ -482,10 +476,13 @@ fm_status fm_debug_stall_next_score(fm_ctx* ctx, uint64_t wait_limit_ns);
 
 /* Diagnostic: the raw tensor-core dot products of one 128-chunk tile of layer
  * `layer`, row b, tile t (chunks t*128 .. t*128+127), before the per-chunk
- * scale, the per-head power-of-two scale and the epilogue, for p < q_pieces:
+ * scale, the per-head power-of-two scale and the epilogue.  With q_pieces = 3:
  *   out[r, p*64 + h] = sum_d e4m3(comp_k[layer][b, t*128 + r, d]) * piece_p(q[b,layer,h])[d]
- * where the query pieces satisfy
- *   q[b,layer,h,d] ~= 2^-pow2_exp[h] * sum_p 16^-p * piece_p[d].
+ * for p < 3, the pieces satisfying q[b,layer,h,d] ~= 2^-pow2_exp[h] * sum_p 16^-p * piece_p[d].
+ * With q_pieces = 2 the tensor core adds the two pieces in one accumulator:
+ *   out[r, h] = sum_d e4m3(comp_k[layer][b, t*128 + r, d]) * (piece_0 + piece_1)(q[b,layer,h])[d]
+ * with q[b,layer,h,d] ~= 2^-pow2_exp[h] * (piece_0[d] + piece_1[d]) (piece 1 the
+ * unscaled e4m3 residual); out[r, 64:] is left untouched.
  * out [128, 192] fp32 device (the entries above written, the rest untouched),
  * pow2_exp [64] int32 device (written).  Rows of the tile past N
  * hold unspecified values.  Used by the

@@ -485,6 +485,20 @@ __device__ __forceinline__ void tmem_ld32x2_wait(uint32_t t0, uint32_t t1, uint3
       : "memory");
 }
 
+
+// One 32-column load plus one single column (ts, result in *s), one wait.
+__device__ __forceinline__ void tmem_ld32_x1_wait(uint32_t t0, uint32_t ts, uint32_t* a, uint32_t* s) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%32}, [%34];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : FM_TMEM_REGS32(a), "=r"(*s)
+      : "r"(t0), "r"(ts)
+      : "memory");
+}
+
 // Three 32-column loads and one wait.
 // Two 32-column loads plus one single column (ts, result in *s), one wait.
 __device__ __forceinline__ void tmem_ld32x2_x1_wait(uint32_t t0, uint32_t t1, uint32_t ts, uint32_t* a,

@@ -813,7 +813,9 @@ __global__ void __launch_bounds__(kThreads) qpack_kernel(const float* __restrict
     for (int i = 0; i < 4; ++i) {
       const uint32_t c = to_e4m3(x[i]);
       word |= c << (8 * i);
-      x[i] = (x[i] - e4m3_value(c)) * 16.0f;  // exact: the residual of a 4-bit rounding
+      // exact: the residual of a 4-bit rounding; two pieces are summed as they
+      // are by the tensor core, three carry the residuals scaled by 16
+      x[i] = P == 2 ? (x[i] - e4m3_value(c)) : (x[i] - e4m3_value(c)) * 16.0f;
     }
     const int row = p * kHeads + h;
     *reinterpret_cast<uint32_t*>(img + sw128_offset(row, lane * 4)) = word;

@@ -149,7 +149,9 @@ __global__ void __launch_bounds__(kCThreads) compact_write_kernel(const uint8_t*
 }
 
 // One warp per record, RU records in flight per warp, each lane moving UPL
-// units of VEC bytes per record per round.
+// units of VEC bytes per record per round; a record's index and its row's
+// count are loaded side by side, so a round waits on one load before the
+// record's own.
 template <int VEC>
 struct Unit;
 template <>
@@ -166,7 +168,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__
                                                      int64_t total, uint8_t* __restrict__ dst,
                                                      int64_t dst_stride) {
   using U = typename Unit<VEC>::T;
-  constexpr int RU = 4, UPL = 2;
+  constexpr int RU = 8, UPL = 2;
   const int lane = threadIdx.x & 31;
   const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -181,8 +183,9 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__
       const int64_t r = r0 + q;
       if (r < total) {
         const int b = (int)(r / max_sel), j = (int)(r - (int64_t)b * max_sel);
-        const int cnt = min(count[b], max_sel);
-        const int n = j < cnt ? idx[r] : -1;
+        const int cnt = min(__ldg(count + b), max_sel);
+        const int id = __ldg(idx + r);  // in bounds whatever the count: loaded beside it, not after it
+        const int n = j < cnt ? id : -1;
         if (n >= 0 && n < n_src) {
           s[q] = reinterpret_cast<const U*>(src + b * src_stride + (int64_t)n * rec);
           d[q] = reinterpret_cast<U*>(dst + b * dst_stride + (int64_t)j * rec);
@@ -206,133 +209,6 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__
           if (d[q] && u < units) d[q][u] = v[q][i];
         }
     }
-  }
-}
-
-// Compaction and gather in one pass over the mask (after the count pass):
-// the ordered index write of compact_write_kernel, then the block copies the
-// records of the chunks it kept, from a shared-memory list of their indices
-// (kRecallList at a time), one warp per record with RU records in flight.
-// Saves the gather's launch and its dependent reads of the index list.
-constexpr int kRecallList = 4096;
-
-template <int VEC>
-__global__ void __launch_bounds__(kCThreads) compact_gather_kernel(
-    const uint8_t* __restrict__ keep, int N, int nblk, const int* __restrict__ blkcnt, int max_sel,
-    int32_t* __restrict__ idx, int32_t* __restrict__ count, const uint8_t* __restrict__ src, int64_t src_stride,
-    int n_src, int64_t rec, uint8_t* __restrict__ dst, int64_t dst_stride) {
-  using U = typename Unit<VEC>::T;
-  constexpr int RU = 4, UPL = 2;
-  __shared__ int s_warp[kCThreads / 32];
-  __shared__ int s_scan[kCThreads / 32];
-  __shared__ int s_prefix, s_total;
-  __shared__ int s_list[kRecallList];
-  const int b = blockIdx.y;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (warp == 0) {
-    int p = 0;
-    for (int j = lane; j < (int)blockIdx.x; j += 32) p += blkcnt[(size_t)b * nblk + j];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-    if (lane == 0) s_prefix = p;
-  }
-  const uint8_t* row = keep + (int64_t)b * N;
-  const int64_t n0 = (int64_t)blockIdx.x * kCChunk + (int64_t)threadIdx.x * kCBytes;
-  uint32_t w[8];
-  const int c = load_mask(row, n0, N, row_vec_ok(keep, N), w);
-  int incl = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int v = lane < kCThreads / 32 ? s_warp[lane] : 0;
-    int sc = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, sc, o);
-      if (lane >= o) sc += u;
-    }
-    if (lane < kCThreads / 32) s_scan[lane] = sc - v;
-    if (lane == kCThreads / 32 - 1) s_total = sc;
-  }
-  __syncthreads();
-  const int local0 = s_scan[warp] + (incl - c);  // this thread's first kept entry, block-local
-  const int prefix = s_prefix, total = s_total;
-  int32_t* out = idx + (size_t)b * max_sel;
-  if (c) {
-    int pos = prefix + local0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if ((w[i] >> (8 * k)) & 0xffu) {
-          if (pos < max_sel) out[pos] = (int32_t)(n0 + 4 * i + k);
-          ++pos;
-        }
-  }
-  if (blockIdx.x == gridDim.x - 1) {
-    const int row_total = prefix + total;
-    if (threadIdx.x == 0) count[b] = row_total;
-    for (int j = row_total + threadIdx.x; j < max_sel; j += kCThreads) out[j] = -1;
-  }
-  // the records of the listed entries (slots below max_sel), kRecallList at a time
-  const int listed = min(total, max(0, max_sel - prefix));
-  const int64_t units = rec / VEC;
-  const uint8_t* srow = src + b * src_stride;
-  uint8_t* drow = dst + b * dst_stride;
-  for (int r0 = 0; r0 < listed; r0 += kRecallList) {
-    const int cnt = min(kRecallList, listed - r0);
-    if (c) {
-      int e = local0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if ((w[i] >> (8 * k)) & 0xffu) {
-            if (e >= r0 && e < r0 + cnt) s_list[e - r0] = (int)(n0 + 4 * i + k);
-            ++e;
-          }
-    }
-    __syncthreads();
-    for (int e0 = warp * RU; e0 < cnt; e0 += (kCThreads / 32) * RU) {
-      const U* sp[RU];
-      U* dp[RU];
-#pragma unroll
-      for (int q = 0; q < RU; ++q) {
-        sp[q] = nullptr;
-        dp[q] = nullptr;
-        const int e = e0 + q;
-        if (e < cnt) {
-          const int n = s_list[e];
-          if (n < n_src) {
-            sp[q] = reinterpret_cast<const U*>(srow + (int64_t)n * rec);
-            dp[q] = reinterpret_cast<U*>(drow + (int64_t)(prefix + r0 + e) * rec);
-          }
-        }
-      }
-      for (int64_t u0 = 0; u0 < units; u0 += 32 * UPL) {
-        U v[RU][UPL];
-#pragma unroll
-        for (int q = 0; q < RU; ++q)
-#pragma unroll
-          for (int i = 0; i < UPL; ++i) {
-            const int64_t u = u0 + i * 32 + lane;
-            if (sp[q] && u < units) v[q][i] = sp[q][u];
-          }
-#pragma unroll
-        for (int q = 0; q < RU; ++q)
-#pragma unroll
-          for (int i = 0; i < UPL; ++i) {
-            const int64_t u = u0 + i * 32 + lane;
-            if (dp[q] && u < units) dp[q][u] = v[q][i];
-          }
-      }
-    }
-    __syncthreads();
   }
 }
 
@@ -368,37 +244,6 @@ fm_status launch_compact(const uint8_t* keep, int B, int N, int max_sel, int32_t
   return check_launch();
 }
 
-fm_status launch_compact_gather(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx, int32_t* count,
-                                void* ws, const void* src, int64_t src_row_stride_bytes, int n_src,
-                                int64_t rec_bytes, void* dst, int64_t dst_row_stride_bytes, cudaStream_t stream) {
-  const int nblk = compact_blocks(N);
-  int* blkcnt = static_cast<int*>(ws);
-  dim3 grid(nblk, B);
-  const uint8_t* s = static_cast<const uint8_t*>(src);
-  uint8_t* d = static_cast<uint8_t*>(dst);
-  auto all_aligned = [&](uintptr_t a) {
-    return (reinterpret_cast<uintptr_t>(s) % a) == 0 && (reinterpret_cast<uintptr_t>(d) % a) == 0 &&
-           rec_bytes % (int64_t)a == 0 && src_row_stride_bytes % (int64_t)a == 0 &&
-           dst_row_stride_bytes % (int64_t)a == 0;
-  };
-  compact_count_kernel<<<grid, kCThreads, 0, stream>>>(keep, N, nblk, blkcnt);
-  if (all_aligned(16))
-    compact_gather_kernel<16><<<grid, kCThreads, 0, stream>>>(keep, N, nblk, blkcnt, max_sel, idx, count, s,
-                                                              src_row_stride_bytes, n_src, rec_bytes, d,
-                                                              dst_row_stride_bytes);
-  else if (all_aligned(4))
-    compact_gather_kernel<4><<<grid, kCThreads, 0, stream>>>(keep, N, nblk, blkcnt, max_sel, idx, count, s,
-                                                             src_row_stride_bytes, n_src, rec_bytes, d,
-                                                             dst_row_stride_bytes);
-  else
-    compact_gather_kernel<1><<<grid, kCThreads, 0, stream>>>(keep, N, nblk, blkcnt, max_sel, idx, count, s,
-                                                             src_row_stride_bytes, n_src, rec_bytes, d,
-                                                             dst_row_stride_bytes);
-  note_launch();
-  note_launch();
-  return check_launch();
-}
-
 fm_status launch_gather(const void* src, int64_t src_row_stride_bytes, int n_src, int64_t rec_bytes,
                         const int32_t* idx, const int32_t* count, int B, int max_sel, void* dst,
                         int64_t dst_row_stride_bytes, cudaStream_t stream) {
@@ -413,7 +258,7 @@ fm_status launch_gather(const void* src, int64_t src_row_stride_bytes, int n_src
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t want = (total + 4 * 8 - 1) / (4 * 8);  // 8 warps of 256 threads, 4 records each
+  const int64_t want = (total + 8 * 8 - 1) / (8 * 8);  // 8 warps of 256 threads, 8 records each
   const int grid = (int)(want < (int64_t)sms * 8 ? (want > 0 ? want : 1) : (int64_t)sms * 8);
   if (all_aligned(16))
     gather_kernel<16><<<grid, 256, 0, stream>>>(s, src_row_stride_bytes, n_src, rec_bytes, idx, count,
@@ -465,21 +310,3 @@ extern "C" fm_status fm_gather_records(const void* src, int64_t src_row_stride_b
                        dst_row_stride_bytes, stream);
 }
 
-extern "C" fm_status fm_recall_records(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx,
-                                       int32_t* count, void* ws, size_t ws_bytes, const void* src,
-                                       int64_t src_row_stride_bytes, int n_src, int64_t rec_bytes, void* dst,
-                                       int64_t dst_row_stride_bytes, cudaStream_t stream) {
-  if (!keep || !idx || !count || !ws || !src || !dst || B < 1 || N < 1 || max_sel < 1 || B > 65535 || n_src < 1 ||
-      rec_bytes < 1)
-    return FM_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(count) & 3u) ||
-      (reinterpret_cast<uintptr_t>(ws) & 15u))
-    return FM_ERR_ALIGNMENT;
-  if (ws_bytes < compact_workspace_bytes(B, N)) return FM_ERR_INVALID_ARG;
-  if (src_row_stride_bytes < (int64_t)n_src * rec_bytes || dst_row_stride_bytes < (int64_t)max_sel * rec_bytes)
-    return FM_ERR_INVALID_ARG;
-  const void* s = device_address(src);
-  if (!s || !device_address(dst)) return FM_ERR_INVALID_ARG;  // pageable host memory
-  return launch_compact_gather(keep, B, N, max_sel, idx, count, ws, s, src_row_stride_bytes, n_src, rec_bytes,
-                               dst, dst_row_stride_bytes, stream);
-}

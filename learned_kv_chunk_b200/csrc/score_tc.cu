@@ -12,11 +12,14 @@
 //    so the ensemble stays in registers and one fp32 per chunk is written;
 //  * the keys go to the tensor cores as stored: kind::f8f6f4 MMA with A = the
 //    128 e4m3 bytes of each record (K = 128 dims) and B = the query split into
-//    P e4m3 pieces (N = P * 64: piece p of head h in column p*64 + h), fp32
-//    accumulators in TMEM -- four MMAs (the K steps) per item, M = 128 chunks
-//    in the 128 TMEM lanes.  The per-chunk fp32 scale, the
-//    per-head power-of-two scale of the pieces, relu, the head-weighted sum
-//    and the sigmoid run in the epilogue;
+//    P e4m3 pieces, fp32 accumulators in TMEM, M = 128 chunks in the 128 TMEM
+//    lanes.  With two pieces the residual piece is stored unscaled and the
+//    tensor core adds both into one 64-column accumulator (eight MMAs of
+//    N = 64 per item: four K steps per piece), and each epilogue group has two
+//    accumulator stages; with three pieces each piece keeps its own 64
+//    columns (four MMAs of N = 192) and one stage per group.  The per-chunk
+//    fp32 scale, the per-head power-of-two scale of the pieces, relu, the
+//    head-weighted sum and the sigmoid run in the epilogue;
 //  * the 132-byte records are not 16-byte aligned, so a tile is fetched with
 //    one 1-D bulk copy (TMA engine) of 128 * 132 bytes into a shared-memory
 //    stage; four transform warps (one TMEM lane quarter each, one chunk row
@@ -38,8 +41,8 @@
 //  * warp roles (16 warps): 0 key loader, 1 and 3 MMA issuers (one per
 //    epilogue group), 2 TMEM owner + query loader, 4-7 transform, 8-11 and
 //    12-15 two epilogue groups (one lane
-//    quarter per warp, all 64 heads of a chunk row), each with one
-//    accumulator stage.  Units are taken in pairs from the same row,
+//    quarter per warp, all 64 heads of a chunk row), each with its
+//    accumulator stages.  Units are taken in pairs from the same row,
 //    the first for group 0 and the second for group 1, and their items are
 //    issued layer by layer alternately, (u0,l0) (u1,l0) (u0,l1) (u1,l1) ...,
 //    so each group has a whole MMA to drain its stage before it is needed
@@ -71,10 +74,19 @@ constexpr uint32_t kPieceBytes = kHeads * kHeadDim;  // one query piece of one l
 constexpr uint32_t kScaleSlots = 32;
 constexpr uint32_t kScaleCol = kTmemCols - kScaleSlots;
 constexpr uint32_t kGroupSlots = kScaleSlots / 2;
+// P = 2: the two query pieces go to one accumulator (piece 1 is stored
+// unscaled, so the tensor core sums p0 + p1), two stages per epilogue group;
+// P = 3: one accumulator block per piece, one stage per group.
 template <int P>
-constexpr uint32_t acc_cols() { return (uint32_t)P * kHeads; }
+constexpr bool fold() { return P == 2; }
 template <int P>
-constexpr uint32_t a_col_base() { return 2u * acc_cols<P>(); }
+constexpr int acc_pieces() { return fold<P>() ? 1 : P; }
+template <int P>
+constexpr uint32_t acc_stages() { return fold<P>() ? 2u : 1u; }
+template <int P>
+constexpr uint32_t acc_cols() { return (uint32_t)acc_pieces<P>() * kHeads; }
+template <int P>
+constexpr uint32_t a_col_base() { return 2u * acc_stages<P>() * acc_cols<P>(); }
 template <int P>
 constexpr uint32_t a_stages() { return (kScaleCol - a_col_base<P>()) / kACols; }  // 7 (P=2), 3 (P=3)
 // A group's scale slot is rewritten 16 of that group's key tiles later.  The
@@ -99,7 +111,7 @@ __host__ __device__ inline Layout make_layout(int L, int P, int NR, int NA) {
   s.raw_off = o;  o += (uint32_t)NR * kRawBytes;                       // 128-aligned stages
   s.wp_off = o;   o += 2u * kQuarters * (uint32_t)L * kHeads * 4;     // per epilogue warp
   o = (o + 7u) & ~7u;
-  s.bar_off = o;  o += (uint32_t)(2 * NR + 2 * NA + 4 + 3) * 8;
+  s.bar_off = o;  o += (uint32_t)(2 * NR + 2 * NA + 8 + 3) * 8;
   s.misc_off = o; o += 64;
   s.total = o + 1024;  // slack to align the base to 1024
   return s;
@@ -184,13 +196,17 @@ template <int P>
 struct HeadCols {
   uint32_t u[P][32];
   __device__ __forceinline__ void load(uint32_t col0) {
-    if constexpr (P == 3)
+    if constexpr (P == 1)
+      tmem_ld32_wait(col0, u[0]);
+    else if constexpr (P == 3)
       tmem_ld32x3_wait(col0, col0 + kHeads, col0 + 2 * kHeads, u[0], u[1], u[2]);
     else
       tmem_ld32x2_wait(col0, col0 + kHeads, u[0], u[1]);
   }
   __device__ __forceinline__ void load_with(uint32_t col0, uint32_t scol, uint32_t* sv) {
-    if constexpr (P == 3)
+    if constexpr (P == 1)
+      tmem_ld32_x1_wait(col0, scol, u[0], sv);
+    else if constexpr (P == 3)
       tmem_ld32x3_x1_wait(col0, col0 + kHeads, col0 + 2 * kHeads, scol, u[0], u[1], u[2], sv);
     else
       tmem_ld32x2_x1_wait(col0, col0 + kHeads, scol, u[0], u[1], sv);
@@ -199,7 +215,8 @@ struct HeadCols {
 };
 
 // Head sum over 32 heads for one chunk row:
-//   sum_h relu(d_h) * w'_h  with d_h = D0 + D1/16 (+ D2/256),  when s >= 0
+//   sum_h relu(d_h) * w'_h  with d_h = D0 (one accumulator for two pieces)
+//                           or D0 + D1/16 + D2/256 (three),   when s >= 0
 //   sum_h relu(s d_h) * w'_h                                  otherwise
 // where D_p are the accumulator columns of piece p and w' the head weights
 // with the pieces' power-of-two scale folded in.
@@ -212,12 +229,17 @@ __device__ __forceinline__ float head_sum32(const HeadCols<P>& c, const float* _
     uint64_t acc = f2_pack(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const uint64_t p0 = f2_pack(c.at(0, 2 * j), c.at(0, 2 * j + 1));
-      const uint64_t p1 = f2_pack(c.at(1, 2 * j), c.at(1, 2 * j + 1));
-      uint64_t d = f2_fma(p1, c16, p0);
-      if constexpr (P == 3) d = f2_fma(f2_pack(c.at(2, 2 * j), c.at(2, 2 * j + 1)), c256, d);
       float dx, dy;
-      f2_unpack(d, dx, dy);
+      if constexpr (P == 1) {
+        dx = c.at(0, 2 * j);
+        dy = c.at(0, 2 * j + 1);
+      } else {
+        const uint64_t p0 = f2_pack(c.at(0, 2 * j), c.at(0, 2 * j + 1));
+        const uint64_t p1 = f2_pack(c.at(1, 2 * j), c.at(1, 2 * j + 1));
+        uint64_t d = f2_fma(p1, c16, p0);
+        if constexpr (P == 3) d = f2_fma(f2_pack(c.at(2, 2 * j), c.at(2, 2 * j + 1)), c256, d);
+        f2_unpack(d, dx, dy);
+      }
       const float2 ww = *reinterpret_cast<const float2*>(w + 2 * j);
       const uint64_t rr = f2_pack(fmax_nan(dx, 0.f), fmax_nan(dy, 0.f));
       acc = f2_fma(rr, f2_pack(ww.x, ww.y), acc);  // one chain: fewer registers, same issue count
@@ -228,7 +250,8 @@ __device__ __forceinline__ float head_sum32(const HeadCols<P>& c, const float* _
   }
   float acc = 0.f;
   for (int i = 0; i < 32; ++i) {
-    float d = fmaf(c.at(1, i), kInv16, c.at(0, i));
+    float d = c.at(0, i);
+    if constexpr (P >= 2) d = fmaf(c.at(1, i), kInv16, d);
     if constexpr (P == 3) d = fmaf(c.at(2, i), kInv256, d);
     acc = fmaf(fmax_nan(d * s, 0.f), w[i], acc);
   }
@@ -259,8 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
   Bars B_;
   B_.raw_full = bar;                B_.raw_empty = B_.raw_full + NR;
   B_.a_full = B_.raw_empty + NR;    B_.a_empty = B_.a_full + NA;
-  B_.acc_full = B_.a_empty + NA;    B_.acc_empty = B_.acc_full + 2;
-  B_.q_full = B_.acc_empty + 2;
+  B_.acc_full = B_.a_empty + NA;    B_.acc_empty = B_.acc_full + 4;
+  B_.q_full = B_.acc_empty + 4;
   B_.q_empty = B_.q_full + 1;       B_.done = B_.q_empty + 1;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + lay.misc_off);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + lay.misc_off + 4);
@@ -276,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       mbar_init(&B_.a_full[i], kQuarters);     // key tile stored in TMEM (one arrival per warp)
       mbar_init(&B_.a_empty[i], 1);            // the MMA that read it retired
     }
-    for (int g = 0; g < 2; ++g) { mbar_init(&B_.acc_full[g], 1); mbar_init(&B_.acc_empty[g], kQuarters); }
+    for (int g = 0; g < 4; ++g) { mbar_init(&B_.acc_full[g], 1); mbar_init(&B_.acc_empty[g], kQuarters); }
     mbar_init(B_.q_full, 1);
     mbar_init(B_.q_empty, 2);                // both MMA issuers' commits
     mbar_init(B_.done, 2);
@@ -379,13 +402,13 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
     // stage and phase.
     if (lane == 0) {
       const int me = warp == kWarpMma ? 0 : 1;
-      constexpr uint32_t idesc = idesc_e4m3_f32(kMmaM, (int)ACCW);
+      constexpr uint32_t idesc = idesc_e4m3_f32(kMmaM, (int)ACCW);  // N = 64 with the pieces folded
       // B descriptors: the start-address field counts 16-byte units, so the
       // layer and K-step offsets are plain adds (the field cannot carry: the
       // query image lies in the first 256 KB of shared memory)
       const uint64_t bdesc0 = sdesc_kmajor_sw128(smem_u32(sQ));
       constexpr uint64_t kLayerStep = kQLayerBytes >> 4, kKStep = 32 >> 4;
-      uint32_t item = 0, rows = 0, ph0 = 0, ph1 = 0;
+      uint32_t item = 0, rows = 0, phs = 0, gcnt = 0;  // phs: phase bit per accumulator stage
       Ring ast(NA);
       int cur = -1;
       bool ok = true;
@@ -408,22 +431,32 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
               continue;
             }
             const Ring& as = SK ? su : ast;
-            const uint32_t ph = j == 0 ? ph0 : ph1;
+            const uint32_t st = acc_stages<P>() == 2 ? (gcnt & 1u) : 0u;
+            const uint32_t slot_i = (uint32_t)j * acc_stages<P>() + st;
+            const uint32_t ph = (phs >> st) & 1u;
             ok = ((SK && l > 0) || mbar_wait_bounded(&B_.a_full[as.stage], as.phase, sAbort, args.err, args.wait_ns)) &&
-                 mbar_wait_bounded(&B_.acc_empty[j], ph ^ 1, sAbort, args.err, args.wait_ns);
+                 mbar_wait_bounded(&B_.acc_empty[slot_i], ph ^ 1, sAbort, args.err, args.wait_ns);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t d = tmem_base + (uint32_t)j * ACCW;
+            const uint32_t d = tmem_base + slot_i * ACCW;
             const uint32_t a = tmem_base + ABASE + as.stage * kACols;
             umma_f8f6f4_ts(d, a, bd, idesc, 0u);
             umma_f8f6f4_ts(d, a + 8u, bd + kKStep, idesc, 1u);
             umma_f8f6f4_ts(d, a + 16u, bd + 2 * kKStep, idesc, 1u);
             umma_f8f6f4_ts(d, a + 24u, bd + 3 * kKStep, idesc, 1u);
+            if constexpr (fold<P>()) {  // piece 1 (rows 64..127 of the layer's image) into the same accumulator
+              const uint64_t bd1 = bd + (kPieceBytes >> 4);
+              umma_f8f6f4_ts(d, a, bd1, idesc, 1u);
+              umma_f8f6f4_ts(d, a + 8u, bd1 + kKStep, idesc, 1u);
+              umma_f8f6f4_ts(d, a + 16u, bd1 + 2 * kKStep, idesc, 1u);
+              umma_f8f6f4_ts(d, a + 24u, bd1 + 3 * kKStep, idesc, 1u);
+            }
             if (!SK || l == L - 1) umma_commit(&B_.a_empty[as.stage]);  // the TMEM key tile may be overwritten
-            umma_commit(&B_.acc_full[j]);
+            umma_commit(&B_.acc_full[slot_i]);
             ++item;
             if (!SK) ast.advance();
-            if (j == 0) ph0 ^= 1u; else ph1 ^= 1u;
+            phs ^= 1u << st;
+            ++gcnt;
           }
         }
         if (!ok) break;
@@ -496,10 +529,10 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
     const int ew = group * kQuarters + quarter;  // 0..7
     const int r = quarter * 32 + lane;           // row of the tile
     float* sWpw = sWp + ew * L * kHeads;
-    const uint32_t col_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)group * ACCW;
+    const uint32_t col_base0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)group * acc_stages<P>() * ACCW;
     const uint32_t scale_base =
         tmem_base + ((uint32_t)(quarter * 32) << 16) + kScaleCol + (uint32_t)group * kGroupSlots;
-    uint32_t ph = 0, gtiles = 0;  // gtiles: this group's key tiles so far (its scale slots)
+    uint32_t phs = 0, gtiles = 0, gitems = 0;  // gtiles: this group's key tiles so far (its scale slots)
     int cur = -1;
     for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); pw.valid(); pw.next()) {
       if (group == 1 && !pw.has1) continue;
@@ -516,36 +549,40 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       const bool in_row = n < args.N;
       float ens = 0.f;
       bool ok = true;
-      for (int l = 0; l < L; ++l, ph ^= 1u) {
-        ok = mbar_wait_bounded(&B_.acc_full[group], ph, sAbort, args.err, args.wait_ns);
+      for (int l = 0; l < L; ++l, ++gitems) {
+        const uint32_t st = acc_stages<P>() == 2 ? (gitems & 1u) : 0u;
+        const uint32_t slot_i = (uint32_t)group * acc_stages<P>() + st;
+        const uint32_t col_base = col_base0 + st * ACCW;
+        ok = mbar_wait_bounded(&B_.acc_full[slot_i], (phs >> st) & 1u, sAbort, args.err, args.wait_ns);
+        phs ^= 1u << st;
         if (!ok) break;
         tc_fence_after();
         // the scale slot of the key tile this item read (one tile per unit with shared keys)
         const uint32_t slot = (gtiles + (SK ? 0u : (uint32_t)l)) & (kGroupSlots - 1);
         const float* w = sWpw + l * kHeads;
-        HeadCols<P> c;
+        HeadCols<acc_pieces<P>()> c;
         uint32_t s_bits;
         c.load_with(col_base, scale_base + slot, &s_bits);
         const float s = valid ? __uint_as_float(s_bits) : 0.f;  // rows past the tail hold stale bytes
         const bool nonneg = __all_sync(0xffffffffu, !(s < 0.f));
         if constexpr (DUMP) {
           if (U.b == args.dbg_b && U.t == args.dbg_t && l == args.dbg_layer)
-            for (int p = 0; p < P; ++p)
+            for (int p = 0; p < acc_pieces<P>(); ++p)
               for (int i = 0; i < 32; ++i) args.dbg_out[(size_t)r * 192 + p * kHeads + i] = c.at(p, i);
         }
-        float part = head_sum32<P>(c, w, s, nonneg);
+        float part = head_sum32<acc_pieces<P>()>(c, w, s, nonneg);
         c.load(col_base + 32);
         // the accumulator stage is free once this warp holds all its columns
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B_.acc_empty[group]);
+        if (lane == 0) mbar_arrive(&B_.acc_empty[slot_i]);
         if constexpr (DUMP) {
           if (U.b == args.dbg_b && U.t == args.dbg_t && l == args.dbg_layer)
-            for (int p = 0; p < P; ++p)
+            for (int p = 0; p < acc_pieces<P>(); ++p)
               for (int i = 0; i < 32; ++i)
                 args.dbg_out[(size_t)r * 192 + p * kHeads + 32 + i] = c.at(p, i);
         }
-        part += head_sum32<P>(c, w + 32, s, nonneg);
+        part += head_sum32<acc_pieces<P>()>(c, w + 32, s, nonneg);
         const float logit = nonneg ? part * s : part;
         float score = 1.0f / (1.0f + __expf(-logit));
         if (!valid) score = 0.f;

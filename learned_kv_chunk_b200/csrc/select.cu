@@ -613,14 +613,38 @@ __global__ void __launch_bounds__(kBlkThreads) topk_fastsel_kernel(Workspace w, 
   int eq = 0;
   for (int i = t; i < cnt; i += kBlkThreads) eq += keys[i] == T ? 1 : 0;
   int eq_total;
-  block_exclusive_scan(eq, s_warp, &eq_total);
-  if (eq_total != need) {  // the K-th value is tied with values not kept: rank them by chunk order
+  const int eq_before = block_exclusive_scan(eq, s_warp, &eq_total);
+  if (eq_total == need) {  // every candidate equal to the K-th is kept
+    for (int i = t; i < cnt; i += kBlkThreads)
+      if (keys[i] >= T) out[idx[i]] = 1;
+    if (t == 0) st->mode = kModeDone;
+    return;
+  }
+  // The K-th value is tied with candidates it does not keep: the tied
+  // candidates are ranked by chunk index among themselves (every chunk with
+  // that score is a candidate, since the score is at least tau), in the
+  // histogram's shared memory when they fit, else over the whole row.
+  constexpr int kTieMax = 2048;
+  if (eq_total > kTieMax) {
     row_select_in_block(ens + (int64_t)b * N, st->nv, N, K, out, sc);
     if (t == 0) st->mode = kModeDone;
     return;
   }
+  int* tie = reinterpret_cast<int*>(s_hist);  // the selection is done with the histogram
+  {
+    int pos = eq_before;
+    for (int i = t; i < cnt; i += kBlkThreads)
+      if (keys[i] == T) tie[pos++] = idx[i];
+  }
+  __syncthreads();
   for (int i = t; i < cnt; i += kBlkThreads)
-    if (keys[i] >= T) out[idx[i]] = 1;
+    if (keys[i] > T) out[idx[i]] = 1;
+  for (int e = t; e < eq_total; e += kBlkThreads) {
+    const int me = tie[e];
+    int rank = 0;
+    for (int f = 0; f < eq_total; ++f) rank += tie[f] < me ? 1 : 0;
+    if (rank < need) out[me] = 1;
+  }
   if (t == 0) st->mode = kModeDone;
 }
 

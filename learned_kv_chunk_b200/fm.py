@@ -95,7 +95,6 @@ def _load():
         "fm_compact_workspace_bytes": (S, [I, I]),
         "fm_compact_mask": (I, [P, I, I, I, P, P, P, S, P]),
         "fm_gather_records": (I, [P, I64, I, I64, P, P, I, I, P, I64, P]),
-        "fm_recall_records": (I, [P, I, I, I, P, P, P, S, P, I64, I, I64, P, I64, P]),
         "fm_level2_create": (I, [P, ctypes.POINTER(fm_level2_desc), P, ctypes.POINTER(P)]),
         "fm_level2_launch": (I, [P, P]),
         "fm_level2_copy_scores": (I, [P, P, P]),
@@ -283,34 +282,6 @@ def fm_gather_records(src: torch.Tensor, idx: torch.Tensor, count: torch.Tensor,
     _check(_lib.fm_gather_records(_ptr(src), n_src * rec, n_src, rec, _ptr(idx), _ptr(count), B, max_sel,
                                   _ptr(dst), dst.stride(0), _stream(stream)), "fm_gather_records")
     return dst
-
-
-def fm_recall_records(keep: torch.Tensor, max_sel: int, src: torch.Tensor, idx: Optional[torch.Tensor] = None,
-                      count: Optional[torch.Tensor] = None, dst: Optional[torch.Tensor] = None,
-                      workspace: Optional[torch.Tensor] = None, stream=None):
-    """fm_compact_mask and fm_gather_records in one call: returns (idx, count,
-    dst) as those two calls would."""
-    if keep.dtype not in (torch.bool, torch.uint8) or not keep.is_cuda or not keep.is_contiguous():
-        raise ValueError("keep must be a contiguous bool or uint8 CUDA tensor")
-    if src.dtype != torch.uint8 or src.dim() != 3 or not src.is_contiguous():
-        raise ValueError("src must be a contiguous uint8 tensor [B, n_src, rec]")
-    if not src.is_cuda and not src.is_pinned():
-        raise ValueError("src must be on the device or in pinned host memory")
-    B, N = keep.shape
-    _, n_src, rec = src.shape
-    dev = keep.device
-    idx = idx if idx is not None else torch.empty(B, max_sel, device=dev, dtype=torch.int32)
-    count = count if count is not None else torch.empty(B, device=dev, dtype=torch.int32)
-    dst = dst if dst is not None else torch.zeros(B, max_sel, rec, device=dev, dtype=torch.uint8)
-    _need(idx, torch.int32, "idx")
-    _need(count, torch.int32, "count")
-    _need(dst, torch.uint8, "dst")
-    nbytes = int(_lib.fm_compact_workspace_bytes(B, N))
-    ws = workspace if workspace is not None else torch.empty(nbytes, device=dev, dtype=torch.uint8)
-    _check(_lib.fm_recall_records(_ptr(keep), B, N, int(max_sel), _ptr(idx), _ptr(count), _ptr(ws), ws.numel(),
-                                  _ptr(src), n_src * rec, n_src, rec, _ptr(dst), dst.stride(0), _stream(stream)),
-           "fm_recall_records")
-    return idx, count, dst
 
 
 class Level2Step:

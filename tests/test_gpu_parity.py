@@ -70,13 +70,18 @@ def test_tile_dot_products_layout(retr, weights):
         kv = O.e4m3_decode(codes).astype(np.float64)             # [128, 128]
         exact = kv @ qh[b, l].T                                    # [128, 64]
         assert np.all(out[:, P * 64:] == 0.0)  # columns past the pieces are untouched
+        # two pieces share one accumulator (the tensor core adds p0 + p1, p1
+        # stored unscaled): columns 64.. stay untouched; three pieces keep one
+        # block each, p_k scaled by 16^k
         rec = np.zeros((128, 64))
         for p in range(P):
             rec += out[:, p * 64:(p + 1) * 64] * 16.0 ** (-p)
         rec *= 2.0 ** (-e[None, :].astype(np.float64))
         # split error: 2^-4P relative per query element, plus the e4m3
-        # subnormal floor of the last piece; doubled for fp32 accumulation
-        floor = 2.0 ** (-10 - 4 * (P - 1)) * 2.0 ** (-e.astype(np.float64))
+        # subnormal floor of the last piece (2^-10 of the head's scale when it
+        # is stored unscaled, 2^-18 with three scaled pieces); doubled for
+        # fp32 accumulation
+        floor = (2.0 ** -10 if P == 2 else 2.0 ** -18) * 2.0 ** (-e.astype(np.float64))
         bound = (np.abs(kv) @ np.abs(qh[b, l]).T * 2.0 ** (-4 * P)
                  + np.abs(kv).sum(1, keepdims=True) * floor[None, :]) * 2 + 1e-6
         assert np.all(np.abs(rec - exact) <= bound), np.abs(rec - exact).max()

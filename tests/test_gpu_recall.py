@@ -89,26 +89,3 @@ def test_topk_mask_to_resident_keys_full_size():
         want = OR.gather_records(keys[b:b + 1].cpu().numpy(), want_idx, want_count,
                                  np.zeros((1, K, 132), np.uint8))
         np.testing.assert_array_equal(dst[b].cpu().numpy(), want[0])
-
-
-@pytest.mark.parametrize("rec", [132, 1024, 131])
-@pytest.mark.parametrize("where", ["device", "pinned"])
-@pytest.mark.parametrize("N,max_sel", [(3 * 16384 + 77, 600), (2 * 16384 + 32, 20000), (5, 3)])
-def test_recall_in_one_call_matches_oracle(rec, where, N, max_sel):
-    """fm_recall_records: the index list, the count and the gathered records
-    of the oracle's compaction and gather, bit for bit -- masks from empty to
-    dense (more kept chunks than one block lists at a time), lists cut by
-    max_sel, the three copy widths, device and pinned host sources."""
-    B = 6
-    g = torch.Generator().manual_seed(rec + N)
-    src = torch.randint(0, 256, (B, N, rec), generator=g, dtype=torch.uint8)
-    keep = _masks(B, N, rec + N)
-    src_in = src.to(DEV) if where == "device" else src.pin_memory()
-    dst = torch.full((B, max_sel, rec), 0xA5, dtype=torch.uint8, device=DEV)
-    idx, count, _ = fm.fm_recall_records(keep.to(DEV), max_sel, src_in, dst=dst)
-    torch.cuda.synchronize()
-    want_idx, want_count = OR.compact_mask(keep.numpy(), max_sel)
-    np.testing.assert_array_equal(count.cpu().numpy(), want_count)
-    np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
-    want = OR.gather_records(src.numpy(), want_idx, want_count, np.full((B, max_sel, rec), 0xA5, np.uint8))
-    np.testing.assert_array_equal(dst.cpu().numpy(), want)
