@@ -130,8 +130,8 @@ struct ScoreArgs {
   float thr;
   int mode;                // FM_ENSEMBLE_*
   int* err;
-  uint64_t wait_ns;        // bound of every wait (kWaitLimitNs unless a test shortens it)
-  int withhold_query;      // test hook: the query operand is never loaded, so its wait runs out
+  uint64_t wait_ns = kWaitLimitNs;  // bound of every wait (shortened only by the test hook)
+  int withhold_query = 0;  // test hook: the query operand is never loaded, so its wait runs out
   // diagnostic dump of one tile's raw accumulators
   float* dbg_out;          // [128, 192] or null
   int dbg_layer, dbg_b, dbg_t;

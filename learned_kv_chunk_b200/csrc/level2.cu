@@ -125,6 +125,7 @@ fm_status record_step(fm_level2* s, cudaStream_t st) {
   a.ens = s->ens;
   a.mode = d.mode;
   a.err = c->d_err;
+  a.wait_ns = kWaitLimitNs;
   e = launch_score(c, a, st);
   if (e != FM_OK) return e;
   if (d.R <= kSelMaxR) {  // one CTA per row does selection, compaction and id mapping

@@ -624,6 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
 
 template <int P, bool DUMP, bool SK>
 fm_status launch_score_p(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t st) {
+  if (a.wait_ns == 0) return FM_ERR_INVALID_ARG;  // every wait needs a bound that lets work finish
   static PerDeviceOnce smem_set;
   int max_smem = 0;
   if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, ctx->device) !=

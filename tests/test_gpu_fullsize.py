@@ -1,7 +1,8 @@
 """Full-size workloads in the launch configuration bench.py times: the fused
 scoring pass (ensemble written, per-layer scores not written) followed by the
-top-K select, checked on sampled chunks against the oracle and, for whole
-rows, through the oracle's selection rule."""
+top-K select, checked on sampled chunks against the oracle, one whole row
+element by element against the oracle's scores, and every row's mask
+through the oracle's selection rule."""
 import numpy as np
 import pytest
 import torch
@@ -74,8 +75,12 @@ def test_full_size_workload(wl):
         n = int(nv[b])
         full = np.stack([O.score_chunks(case.comp_k[l][b, :n].cpu().numpy(), case.q_o[b, l],
                                         case.w_o[b, l]) for l in range(3)])
+        # every chunk of the row, per layer and ensembled, element by element
+        d_layers = np.abs(scores[:, b, :n].cpu().numpy().astype(np.float64) - full).max()
+        assert d_layers <= H.SCORE_TOL, d_layers
         e_row = np.zeros((1, wl.N))
         e_row[0, :n] = O.ensemble(full, wl.mode)
+        assert np.abs(e_gpu[b, :n] - e_row[0, :n]).max() <= H.SCORE_TOL
         H.check_topk_near_oracle(k_gpu[b:b + 1], e_row, nv[b:b + 1], wl.top_k)
     finally:
         r.close()

@@ -67,6 +67,7 @@ def test_level2_graph_matches_oracle_and_eager(B):
             step.positions.copy_(positions.to(DEV))
             step.launch()
             torch.cuda.synchronize()
+            r.fm_sync_status()  # no bounded wait ran out inside the graph
             ens = step.scores().cpu().numpy()
             ids = step.out_ids.cpu().numpy()
             cnt = count.cpu().numpy()
@@ -138,6 +139,44 @@ def test_level2_ties_take_the_lowest_slots():
         np.testing.assert_array_equal(out[2, :60], idh[2, :60])
         assert (out[2, 60:] == -1).all()
         np.testing.assert_array_equal(step.out_count.cpu().numpy(), [k, k, 60])
+        step.close()
+    finally:
+        r.close()
+
+
+def test_level2_at_bench_size():
+    """The bench's Level-2 shape (64 rows x 4096 resident chunks, top-512):
+    every CTA of the scoring pass takes many units and rows change inside its
+    range.  Several graph launches without an error recorded, scores of a few
+    rows against the oracle, the top-k rule on the graph's own scores."""
+    B, R, k, N1 = 64, 4096, 512, 262144
+    weights = G.make_weights(5000, 3)
+    layers_np = H.np_layers(weights)
+    r = fm.Retriever(weights, device=0, max_batch=B, q_pieces=2)
+    try:
+        g = torch.Generator().manual_seed(5001)
+        ids = torch.stack([torch.randperm(N1, generator=g)[:R].sort().values for _ in range(B)]).to(torch.int32)
+        res_keys = G.make_keys(5002, [R] * B, R, 3, None, device=DEV)
+        count = torch.full((B,), R, dtype=torch.int32, device=DEV)
+        step = fm.Level2Step(r, res_keys, ids.to(DEV), count, k=k, mode="max")
+        hidden = G.make_hidden(5003, B)
+        positions = torch.full((B,), 4 * N1, dtype=torch.int64)
+        step.hidden.copy_(hidden.to(DEV))
+        step.positions.copy_(positions.to(DEV))
+        for _ in range(4):
+            step.launch()
+        torch.cuda.synchronize()
+        r.fm_sync_status()
+        ens = step.scores().cpu().numpy()
+        q_o, w_o = H.oracle_queries(layers_np, hidden, positions)
+        for b in (0, 33, 63):
+            per = [O.score_chunks(res_keys[l][b].cpu().numpy(), q_o[b, l], w_o[b, l]) for l in range(3)]
+            assert np.abs(ens[b] - O.ensemble(np.stack(per), "max")).max() <= H.SCORE_TOL
+        keep = O.select_topk(ens, np.full(B, R), k)
+        idh = ids.numpy()
+        out = step.out_ids.cpu().numpy()
+        for b in range(B):
+            np.testing.assert_array_equal(out[b], idh[b, np.flatnonzero(keep[b])])
         step.close()
     finally:
         r.close()
