@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--shared-keys", action="store_true",
                     help="one compressed_k tensor scored by all three layers' queries (the README "
                          "Usage signature taken literally); reports against the fp8 tensor peak")
+    ap.add_argument("--decode-rows", type=int, default=64,
+                    help="--path decode: rows of the 262144-chunk workload (64 is the bench line; fewer "
+                         "give a small case for profiling)")
     ap.add_argument("--path", default="retrieve", choices=["retrieve", "recall", "level2", "decode"],
                     help="retrieve: the scoring path (default); recall: keep mask -> index lists -> "
                          "gather of the kept chunks' records into a resident buffer; level2: the "
@@ -95,6 +98,15 @@ def fp8_tensor_peak():
             return 2.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 x 2 (nominal fp8/bf16 ratio)"
     except Exception:
         return 2.0 * 1590.0, "fallback bf16 x 2"
+
+
+def bf16_tensor_peak():
+    """Dense bf16 tensor peak (TFLOP/s): the measured cuBLAS burst figure."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 def peaks():
@@ -273,7 +285,7 @@ def run_ours(args, wl, rank, world, local_rank):
         else:
             elapsed_ms = 0.0
             for _ in range(args.steps):
-                flush_buf.fill_(1.0)
+                flush_l2(flush_buf)
                 t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 t0.record(stream)
                 step(timed=True)
@@ -357,11 +369,19 @@ def run_ours(args, wl, rank, world, local_rank):
 
 
 # ------------------------------------------------------------ recall path
+def flush_l2(flush_buf):
+    """Flushes L2: writes a buffer of at least twice its size, then reads it back, so the
+    timed work starts with a cold L2 that holds no dirty lines (the write-back
+    of the flush's own lines is not charged to the timed kernels)."""
+    flush_buf.fill_(1.0)
+    flush_buf.sum()
+
+
 def _timed_flushed(fn, steps, flush_buf, stream):
     """Mean CUDA-event time (ms) of fn() over `steps` calls, L2 flushed before each."""
     total = 0.0
     for _ in range(steps):
-        flush_buf.fill_(1.0)
+        flush_l2(flush_buf)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()
@@ -415,6 +435,11 @@ def run_recall(args):
         t_compact = _timed_flushed(compact, args.steps, flush_buf, stream)
         t_host = _timed_flushed(gather_host, max(3, args.steps // 10), flush_buf, stream)
     launches = fm.fm_launch_count() - launches0
+    # the same gather by torch's own indexing kernel (records as 33 int32 words),
+    # for the rate a library gather reaches on this access pattern
+    flat = (idx.to(torch.int64) + torch.arange(B, device=dev, dtype=torch.int64)[:, None] * N).view(-1)
+    words = src_dev.view(B * N, rec).view(torch.int32)
+    t_torch = _timed_flushed(lambda: torch.index_select(words, 0, flat), args.steps, flush_buf, stream)
     # the bus: one pinned host -> device copy of 256 MB with the copy engine, same run
     hbuf = torch.empty(1 << 28, dtype=torch.uint8).pin_memory()
     dbuf = torch.empty(1 << 28, dtype=torch.uint8, device=dev)
@@ -435,12 +460,14 @@ def run_recall(args):
            "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic (seeded)",
            "config": {"workload": "recall_B64_N262144_top4096_rec132", "rows": B, "chunks_per_row": N,
                       "kept_per_row": K, "record_bytes": rec, "source": "device memory",
-                      "l2": "flushed between steps (256 MB write)"},
+                      "l2": "flushed between steps (256 MB written, then read back)"},
            "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
                         "frac": round(ach / hbm_peak, 4), "traffic": None, "peak_kind": peak_kind,
                         "kernel": "compaction (2 kernels) + gather, one step",
                         "alg_bytes_per_step": alg_dev},
            "compact_ms": round(t_compact, 4),
+           "gather_ms": round(t_step - t_compact, 4),
+           "torch_index_select_ms": round(t_torch, 4),
            "host_source": {"value": sel / (t_host / 1e3), "unit": "records/s", "gather_ms": round(t_host, 4),
                            "achieved_gbs": round(host_gbs, 2),
                            "h2d_copy_gbs": round(h2d_gbs, 2),
@@ -523,7 +550,7 @@ def run_level2(args):
             "vs_baseline": None, "dtype": "e4m3", "data": "synthetic (seeded generator, random-init weights)",
             "config": {"workload": "level2_B64_R4096_top512", "rows": B, "resident_per_row": R, "top_k": k,
                        "layers": L, "ensemble": "max", "query_prep_in_step": True,
-                       "l2": "flushed between steps (256 MB write)"},
+                       "l2": "flushed between steps (256 MB written, then read back)"},
             "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(ach / hbm_peak, 4), "traffic": None, "peak_kind": peak_kind,
                          "kernel": "the whole step (one graph: query prep, scoring, top-k, compaction, id map)",
@@ -543,6 +570,9 @@ def run_decode(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     wl = G.WORKLOADS[4]
+    if args.decode_rows != wl.B:
+        import dataclasses
+        wl = dataclasses.replace(wl, B=int(args.decode_rows))
     inp = G.make_query_inputs(wl)
     B, N, L, K = wl.B, wl.N, G.N_LAYERS, wl.top_k
     r = fm.Retriever(inp.weights, device=0, max_batch=B, q_pieces=args.q_pieces)
@@ -575,31 +605,34 @@ def run_decode(args):
         flush_buf = torch.empty(max(2 * l2, 1 << 28) // 4, device=dev, dtype=torch.float32)
         ws = torch.empty(int(fm.lib().fm_decode_attention_workspace_bytes(B, K)), device=dev, dtype=torch.uint8)
         out = torch.empty(B, 32, 128, device=dev)
-        t_attn = _timed_flushed(lambda: fm.fm_decode_attention(dec.hidden.view(B, 32, 128), dec.mem, dec.idx,
-                                                                dec.count, out=out, workspace=ws),
-                                20, flush_buf, stream)
+        t_attn = _timed_flushed(dec.attend, 20, flush_buf, stream)
     launches = fm.fm_launch_count() - launches0
     r.fm_sync_status()
     kept = int(dec.count.clamp(max=K).sum())
     flops = kept * 32 * 128 * 4  # q.x and p.x: one multiply-add each per (chunk, head, dim)
-    alu_peak = 148 * 128 * 2 * 1965e6 / 1e12  # fp32 lanes x 2 FLOP x max SM clock
-    ach = flops / (t_attn / 1e3) / 1e12
+    # the kept records once (the resident buffer), the query in, the output out
+    attn_bytes = kept * G.RECORD_BYTES + 2 * B * 32 * 128 * 4
+    hbm_peak, peak_kind = peaks()
+    ach = attn_bytes / (t_attn / 1e3) / 1e9
+    tc_frac = flops / (t_attn / 1e3) / 1e12 / bf16_tensor_peak()
     r.close()
     return {"metric": "toy sparse decode tokens/sec (retrieval every 64 steps, attention over kept chunks)",
             "value": B * interval / (t_cycle / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": cycles * interval,
             "warmup": max(3, args.warmup), "ms_per_step": t_cycle / interval, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32 (attention), e4m3 (retrieval)",
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 pieces, f32 accumulate (attention), e4m3 (retrieval)",
             "data": "synthetic (seeded generator, random-init weights)",
-            "config": {"workload": "decode_B64_N262144_top4096_interval64", "rows": B, "chunks_per_row": N,
+            "config": {"workload": f"decode_B{B}_N262144_top4096_interval64", "rows": B, "chunks_per_row": N,
                        "kept_per_row": K, "retrieval_interval": interval, "attention_heads": 32,
                        "l2": "cycle inputs larger than L2 (6.64 GB of keys per retrieval); attention timed "
                              "alone after a 256 MB L2 flush"},
             "cycle_ms": round(t_cycle, 4),
-            "roofline": {"bound": "alu", "achieved": round(ach, 2), "peak": round(alu_peak, 1), "unit": "TFLOP/s",
-                         "frac": round(ach / alu_peak, 4), "traffic": None,
-                         "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz",
-                         "kernel": "sparse attention over the kept chunks (partial + combine)",
-                         "kernel_ms": round(t_attn, 4), "alg_flops_per_launch": flops},
+            "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(ach / hbm_peak, 4), "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "sparse attention over the resident kept records (segments on tcgen05 + "
+                                   "combine), L2 flushed before each launch",
+                         "kernel_ms": round(t_attn, 4), "alg_bytes_per_launch": attn_bytes,
+                         "alg_flops_per_launch": flops,
+                         "tensor_frac_of_bf16_peak": round(tc_frac, 4)},
             "gpu_launches": launches, "clocks": sampler.summary()}
 
 
@@ -704,7 +737,7 @@ def config_of(wl, gpus, flush=None, key_bytes=None, shared_keys=False):
          "ensemble": wl.mode, "top_k": wl.top_k, "threshold": wl.threshold,
          "query_prep_in_step": True, "parallelism": f"rows sharded over {gpus} GPU(s), no collective"}
     if flush is not None:
-        c["l2"] = ("flushed between steps (256 MB write)" if flush
+        c["l2"] = ("flushed between steps (256 MB written, then read back)" if flush
                    else f"inputs larger than L2 ({key_bytes / 1e9:.2f} GB of keys per step)")
     return c
 

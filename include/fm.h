@@ -423,7 +423,9 @@ size_t fm_decode_attention_workspace_bytes(int B, int max_sel);
 /* The sparse attention, reading only the kept chunks: idx/count as written by
  * fm_compact_mask for the keep mask (the first min(count[b], max_sel) entries
  * of idx[b] are the kept chunk indices; an index outside [0, n_mem) counts as
- * masked).  q [B, 32, 128] fp32 device, 16-byte aligned; mem: the chunk
+ * masked).  idx NULL: the resident form, in which row b of mem holds the kept
+ * records themselves in increasing chunk order (fm_gather_records with the
+ * same idx/count), and record j < min(count[b], max_sel, n_mem) is used.  q [B, 32, 128] fp32 device, 16-byte aligned; mem: the chunk
  * records [B, n_mem, 132] uint8 device, row b at mem + b*row_stride_bytes
  * (4-byte aligned, row_stride_bytes >= n_mem*132, a multiple of 4);
  * out [B, 32, 128] fp32 device (written); ws: the workspace, 16-byte aligned. */

@@ -426,6 +426,7 @@ fm_status fm_sync_status(fm_ctx* c, cudaStream_t stream) {
     cudaMemset(c->d_err, 0, sizeof(int));
     return FM_ERR_DEVICE;
   }
+  if (take_attention_error() != kDevErrNone) return FM_ERR_DEVICE;
   return FM_OK;
 }
 

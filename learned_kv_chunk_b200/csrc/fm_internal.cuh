@@ -175,6 +175,10 @@ fm_status launch_topk_shard_mask(const float* ens, int B, int N, const int32_t* 
                                  uint8_t* keep, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 // ------------------------------------------------------------ PTX wrappers
+// Reads and clears the error word of the decode attention's segment kernel
+// on the current device (kDevErrNone when no wait ran out).
+int take_attention_error();
+
 #if defined(__CUDACC__)
 
 // Launches `kernel` so that it may start while the kernel ahead of it in

@@ -12,12 +12,15 @@
 //               over the bus by the SMs, or device memory) into slot j of a
 //               resident buffer on the GPU.
 //
-// Compaction is two passes over the mask (1 byte per chunk): per-block counts,
-// then an ordered write in which each block starts at the sum of the counts
-// of the blocks before it.  No block waits on another.  The gather is a copy
+// Compaction is one launch with a cluster of up to 4 CTAs per row: each CTA
+// counts the kept entries of its part of the mask, the cluster exchanges the
+// counts through distributed shared memory, and each CTA writes its indices
+// at the offset the CTAs before it leave.  The gather is a copy
 // with one warp per record and several records in flight per warp: the
 // selected records are scattered, so the copy engines (one call per
 // contiguous run) are not used.
+#include <cooperative_groups.h>
+
 #include "fm_internal.cuh"
 
 namespace fm {
@@ -27,9 +30,7 @@ constexpr int kCThreads = 512;
 constexpr int kCBytes = 32;                      // mask bytes per thread
 constexpr int kCChunk = kCThreads * kCBytes;     // mask bytes per block
 
-size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-
-int compact_blocks(int N) { return (int)(((int64_t)N + kCChunk - 1) / kCChunk); }
+__host__ __device__ inline int compact_blocks(int N) { return (int)(((int64_t)N + kCChunk - 1) / kCChunk); }
 
 // The 32 mask bytes of this thread as eight words (bytes past N read as 0),
 // and how many of them are nonzero.
@@ -62,89 +63,105 @@ __device__ __forceinline__ bool row_vec_ok(const uint8_t* keep, int N) {
   return (N & 15) == 0 && (reinterpret_cast<uintptr_t>(keep) & 15u) == 0;
 }
 
-__device__ __forceinline__ int block_sum(int v, int* s_warp) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((threadIdx.x & 31) == 0) s_warp[threadIdx.x >> 5] = v;
-  __syncthreads();
-  int t = 0;
-#pragma unroll
-  for (int i = 0; i < kCThreads / 32; ++i) t += s_warp[i];
-  return t;
-}
-
-__global__ void __launch_bounds__(kCThreads) compact_count_kernel(const uint8_t* __restrict__ keep, int N,
-                                                                  int nblk, int* __restrict__ blkcnt) {
-  __shared__ int s_warp[kCThreads / 32];
-  const int b = blockIdx.y;
-  const uint8_t* row = keep + (int64_t)b * N;
-  uint32_t w[8];
-  const int c = load_mask(row, (int64_t)blockIdx.x * kCChunk + (int64_t)threadIdx.x * kCBytes, N,
-                          row_vec_ok(keep, N), w);
-  const int t = block_sum(c, s_warp);
-  if (threadIdx.x == 0) blkcnt[(size_t)b * nblk + blockIdx.x] = t;
-}
-
-__global__ void __launch_bounds__(kCThreads) compact_write_kernel(const uint8_t* __restrict__ keep, int N,
-                                                                  int nblk, const int* __restrict__ blkcnt,
-                                                                  int max_sel, int32_t* __restrict__ idx,
-                                                                  int32_t* __restrict__ count) {
-  __shared__ int s_warp[kCThreads / 32];
-  __shared__ int s_scan[kCThreads / 32];
-  __shared__ int s_prefix;
-  const int b = blockIdx.y;
+// Exclusive scan of one int per thread over the block (thread order); also
+// returns the block's total.  Two __syncthreads; s_warp has kCThreads/32 ints.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  // kept entries of the blocks before this one (warp 0, strided)
-  if (warp == 0) {
-    int p = 0;
-    for (int j = lane; j < (int)blockIdx.x; j += 32) p += blkcnt[(size_t)b * nblk + j];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-    if (lane == 0) s_prefix = p;
-  }
-  const uint8_t* row = keep + (int64_t)b * N;
-  const int64_t n0 = (int64_t)blockIdx.x * kCChunk + (int64_t)threadIdx.x * kCBytes;
-  uint32_t w[8];
-  const int c = load_mask(row, n0, N, row_vec_ok(keep, N), w);
-  // exclusive scan of the per-thread counts in thread (= chunk) order
-  int incl = c;
+  int incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
   }
   if (lane == 31) s_warp[warp] = incl;
   __syncthreads();
-  if (warp == 0) {
-    const int v = lane < kCThreads / 32 ? s_warp[lane] : 0;
-    int s = v;
+  int before = 0;
+  total = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += u;
-    }
-    if (lane < kCThreads / 32) s_scan[lane] = s - v;  // exclusive over warps
+  for (int i = 0; i < kCThreads / 32; ++i) {
+    const int x = s_warp[i];
+    before += i < warp ? x : 0;
+    total += x;
   }
-  __syncthreads();
-  int pos = s_prefix + s_scan[warp] + (incl - c);
+  __syncthreads();  // s_warp may be rewritten by the next scan
+  return before + incl - v;
+}
+
+// One cluster of C <= 4 CTAs per row (blockIdx.y; 4 measured faster than 2
+// or 8 on 64 rows of 262144); CTA r of the cluster takes the
+// mask chunks [r*nch/C, (r+1)*nch/C) of kCChunk bytes.  Pass 1 counts its
+// kept entries; the CTAs exchange their totals through distributed shared
+// memory, so every CTA knows how many kept entries of the row come before
+// its part; pass 2 writes its indices in order (the first two chunks from
+// registers, later ones re-read, from L2).  The cluster's last CTA writes
+// the count and the -1 tail.  One read of the mask from DRAM, one launch.
+__global__ void __launch_bounds__(kCThreads) compact_cluster_kernel(const uint8_t* __restrict__ keep, int N,
+                                                                    int max_sel, int32_t* __restrict__ idx,
+                                                                    int32_t* __restrict__ count) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  __shared__ int s_warp[kCThreads / 32];
+  __shared__ int s_total;
+  const int b = blockIdx.y;
+  const int C = (int)cl.num_blocks();
+  const int rank = (int)cl.block_rank();
+  const int nch = compact_blocks(N);
+  const int j0 = (int)((int64_t)nch * rank / C), j1 = (int)((int64_t)nch * (rank + 1) / C);
+  const uint8_t* row = keep + (int64_t)b * N;
+  const bool vec = row_vec_ok(keep, N);
+  const int64_t tb = (int64_t)threadIdx.x * kCBytes;
+  // the first two chunks stay in registers for pass 2
+  uint32_t w0[8] = {}, w1[8] = {};
+  int c0 = 0, c1 = 0, mine = 0;
+  if (j0 < j1) c0 = load_mask(row, (int64_t)j0 * kCChunk + tb, N, vec, w0);
+  if (j0 + 1 < j1) c1 = load_mask(row, (int64_t)(j0 + 1) * kCChunk + tb, N, vec, w1);
+  mine = c0 + c1;
+  for (int j = j0 + 2; j < j1; ++j) {
+    uint32_t t[8];
+    mine += load_mask(row, (int64_t)j * kCChunk + tb, N, vec, t);
+  }
+  int cta_total;
+  (void)block_exclusive_scan(mine, s_warp, cta_total);
+  if (threadIdx.x == 0) s_total = cta_total;
+  cl.sync();
+  int before = 0, row_total = 0;
+  for (int r = 0; r < C; ++r) {
+    const int x = *cl.map_shared_rank(&s_total, r);
+    before += r < rank ? x : 0;
+    row_total += x;
+  }
+  cl.sync();  // no CTA leaves while another reads its total
   int32_t* out = idx + (size_t)b * max_sel;
-  if (c) {
+  int base = before;
+  // writes one chunk's kept indices in order from `base`; returns the chunk's total
+  auto write_chunk = [&](int j, const uint32_t (&t)[8], int cj) {
+    const int64_t n0 = (int64_t)j * kCChunk + tb;
+    int chunk_total;
+    int pos = base + block_exclusive_scan(cj, s_warp, chunk_total);
+    if (cj) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 8; ++i) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if ((w[i] >> (8 * k)) & 0xffu) {
-          if (pos < max_sel) out[pos] = (int32_t)(n0 + 4 * i + k);
-          ++pos;
+        for (int k = 0; k < 4; ++k) {
+          if ((t[i] >> (8 * k)) & 0xffu) {
+            if (pos < max_sel) out[pos] = (int32_t)(n0 + 4 * i + k);
+            ++pos;
+          }
         }
       }
     }
+    base += chunk_total;
+  };
+  if (j0 < j1 && base < max_sel) write_chunk(j0, w0, c0);
+  if (j0 + 1 < j1 && base < max_sel) write_chunk(j0 + 1, w1, c1);
+  for (int j = j0 + 2; j < j1 && base < max_sel; ++j) {
+    uint32_t t[8];
+    const int cj = load_mask(row, (int64_t)j * kCChunk + tb, N, vec, t);
+    write_chunk(j, t, cj);
   }
-  if (blockIdx.x == gridDim.x - 1) {
-    // the last block knows the row's total: the count, and -1 past it
-    const int total = s_prefix + s_scan[kCThreads / 32 - 1] + s_warp[kCThreads / 32 - 1];
-    if (threadIdx.x == 0) count[b] = total;
-    for (int j = total + threadIdx.x; j < max_sel; j += kCThreads) out[j] = -1;
+  if (rank == C - 1) {
+    if (threadIdx.x == 0) count[b] = row_total;
+    for (int j = row_total + (int)threadIdx.x; j < max_sel; j += kCThreads) out[j] = -1;
   }
 }
 
@@ -230,18 +247,34 @@ const void* device_address(const void* p) {
 
 namespace fm {
 
-size_t compact_workspace_bytes(int B, int N) { return align256(sizeof(int) * (size_t)B * compact_blocks(N)); }
+// The cluster kernel needs no workspace; the entry point keeps its argument.
+size_t compact_workspace_bytes(int B, int N) {
+  (void)B;
+  (void)N;
+  return 256;
+}
+
+int compact_cluster_size(int N) { return compact_blocks(N) < 4 ? compact_blocks(N) : 4; }
 
 fm_status launch_compact(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx, int32_t* count,
                          void* ws, cudaStream_t stream) {
-  const int nblk = compact_blocks(N);
-  int* blkcnt = static_cast<int*>(ws);
-  dim3 grid(nblk, B);
-  compact_count_kernel<<<grid, kCThreads, 0, stream>>>(keep, N, nblk, blkcnt);
-  compact_write_kernel<<<grid, kCThreads, 0, stream>>>(keep, N, nblk, blkcnt, max_sel, idx, count);
+  (void)ws;
+  if (B > 65535) return FM_ERR_UNSUPPORTED;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)compact_cluster_size(N);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(attr[0].val.clusterDim.x, (unsigned)B);
+  cfg.blockDim = dim3(kCThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, compact_cluster_kernel, keep, N, max_sel, idx, count);
   note_launch();
-  note_launch();
-  return check_launch();
+  return e == cudaSuccess ? check_launch() : record_cuda_error(e);
 }
 
 fm_status launch_gather(const void* src, int64_t src_row_stride_bytes, int n_src, int64_t rec_bytes,

@@ -78,8 +78,9 @@ __host__ __device__ inline size_t ws_bytes(int B, int nblk) {
 }
 
 // ------------------------------------------------- the candidate fast path
-// Exact top-K with one full pass over the scores.  A CTA per row takes an
-// evenly spread sample of up to kSample scores and sets the threshold tau to
+// Exact top-K with one full pass over the scores.  A CTA per row takes a
+// sample of up to kSample scores (256 runs of 32 consecutive ones, evenly
+// spread over the row) and sets the threshold tau to
 // the sample's key of rank 2K * S / n + 16 (about the 2K-th largest score of
 // the row).  One pass over the row then writes the mask's zeros and appends
 // every valid score >= tau, with its index, to the row's candidate list.  If
@@ -449,13 +450,18 @@ __global__ void __launch_bounds__(kBlkThreads) topk_sample_kernel(Workspace w, F
   const int nv = st->nv, K = st->remaining;
   const int S = nv < kSample ? nv : kSample;
   const float* row = ens + (size_t)b * N;
-  {  // all of a thread's strided loads in flight at once
+  {  // all of a thread's loads in flight at once
+    // S = kSample: 256 runs of 32 consecutive scores spread evenly over the
+    // row (each run one 128-byte line: a warp reads a run per load); else
+    // the whole row
     constexpr int kPer = kSample / kBlkThreads;
+    static_assert(kSample == 256 * 32 && kBlkThreads % 32 == 0, "sample runs");
+    const int64_t run_step = S == kSample ? nv / 256 : 32;
     float v[kPer];
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
       const int j = t + q * kBlkThreads;
-      v[q] = j < S ? __ldg(row + (int64_t)j * nv / S) : 0.f;
+      v[q] = j < S ? __ldg(row + (int64_t)(j >> 5) * run_step + (j & 31)) : 0.f;
     }
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {

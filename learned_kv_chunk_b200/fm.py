@@ -345,20 +345,23 @@ class Level2Step:
             pass
 
 
-def fm_decode_attention(q: torch.Tensor, mem: torch.Tensor, idx: torch.Tensor, count: torch.Tensor,
+def fm_decode_attention(q: torch.Tensor, mem: torch.Tensor, idx: Optional[torch.Tensor], count: torch.Tensor,
                         out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                         stream=None) -> torch.Tensor:
     """The toy decoder's sparse attention over the kept chunks: q [B, 32, 128]
     fp32 (the hidden state [B, 4096] viewed as 32 heads), mem [B, N, 132]
-    uint8 chunk records, idx/count from fm_compact_mask.  Returns o [B, 32, 128]."""
+    uint8 chunk records, idx/count from fm_compact_mask; with idx None, mem
+    is the resident buffer [B, max_sel, 132] of the kept records in order
+    (fm_gather_records).  Returns o [B, 32, 128]."""
     _need(q, torch.float32, "q")
     _need(mem, torch.uint8, "mem")
-    _need(idx, torch.int32, "idx")
+    if idx is not None:
+        _need(idx, torch.int32, "idx")
     _need(count, torch.int32, "count")
     B, n_mem, rec = mem.shape
     if rec != 132:
         raise ValueError("mem must be [B, N, 132] uint8")
-    max_sel = idx.shape[1]
+    max_sel = idx.shape[1] if idx is not None else n_mem
     out = out if out is not None else torch.empty(B, 32, 128, device=q.device, dtype=torch.float32)
     nbytes = int(_lib.fm_decode_attention_workspace_bytes(B, max_sel))
     ws = workspace if workspace is not None else torch.empty(nbytes, device=q.device, dtype=torch.uint8)
@@ -404,6 +407,10 @@ class ToySparseDecoder:
         self.max_sel = int(top_k) if top_k is not None else self.N
         self.idx = torch.empty(self.B, self.max_sel, device=dev, dtype=torch.int32)
         self.count = torch.empty(self.B, device=dev, dtype=torch.int32)
+        # top-K: the kept records are gathered once per retrieval into a
+        # resident buffer that every step's attention reads in order
+        self.resident = (torch.empty(self.B, self.max_sel, 132, device=dev, dtype=torch.uint8)
+                         if top_k is not None else None)
         self.attn = torch.empty(self.B, 32, 128, device=dev, dtype=torch.float32)
         self._cws = torch.empty(int(_lib.fm_compact_workspace_bytes(self.B, self.N)), device=dev,
                                 dtype=torch.uint8)
@@ -420,13 +427,22 @@ class ToySparseDecoder:
         self.ens = ens
         self.keep = keep_topk if self.top_k is not None else keep_thr
         fm_compact_mask(self.keep, self.max_sel, idx=self.idx, count=self.count, workspace=self._cws)
+        if self.resident is not None:
+            fm_gather_records(self.mem, self.idx, self.count, self.resident)
+
+    def attend(self):
+        """The sparse attention of the current hidden state over the kept chunks."""
+        if self.resident is not None:
+            return fm_decode_attention(self.hidden.view(self.B, 32, 128), self.resident, None, self.count,
+                                       out=self.attn, workspace=self._aws)
+        return fm_decode_attention(self.hidden.view(self.B, 32, 128), self.mem, self.idx, self.count,
+                                   out=self.attn, workspace=self._aws)
 
     def step(self):
         """One decode step; returns the new hidden state [B, 4096]."""
         if self.t % self.interval == 0:
             self.retrieve()
-        fm_decode_attention(self.hidden.view(self.B, 32, 128), self.mem, self.idx, self.count, out=self.attn,
-                            workspace=self._aws)
+        self.attend()
         fm_toy_decoder_update(self.hidden, self.attn.view(self.B, -1), out=self.hidden)
         self.t += 1
         return self.hidden

@@ -1,5 +1,6 @@
 """The toy sparse decode on the GPU against the oracle: the sparse attention
-over the kept chunks (several 128-chunk segments, ragged tails, empty rows,
+over the kept chunks, through the index list and from a resident buffer of
+the kept records (several 128-chunk segments, ragged tails, empty rows,
 out-of-range indices), the state update, and the decode loop teacher-forced
 step by step (each step's GPU output against the oracle's step from the GPU's
 own input state and keep mask; retrievals at t % 64 == 0 against the top-K
@@ -30,8 +31,9 @@ def _check_attention(o_gpu, o_ref):
     assert err.max() <= ATTN_TOL, err.max()
 
 
+@pytest.mark.parametrize("resident", [False, True], ids=["index_list", "resident"])
 @pytest.mark.parametrize("max_sel", [1, 128, 300, 1000])
-def test_sparse_attention_matches_masked_oracle(max_sel):
+def test_sparse_attention_matches_masked_oracle(max_sel, resident):
     B, N = 5, 3000
     keys = G.make_keys(61, [N, 2500, 900, N, 10], N, 1, None)[0]
     rng = np.random.default_rng(max_sel)
@@ -41,7 +43,11 @@ def test_sparse_attention_matches_masked_oracle(max_sel):
     keep[4, 10:] = False
     q = torch.from_numpy(rng.standard_normal((B, 32, 128)).astype(np.float32))
     idx, count = fm.fm_compact_mask(torch.from_numpy(keep).to(DEV), max_sel)
-    o = fm.fm_decode_attention(q.to(DEV), keys.to(DEV), idx, count).cpu().numpy()
+    if resident:  # the kept records gathered in order; the attention reads them without the list
+        res = fm.fm_gather_records(keys.to(DEV), idx, count)
+        o = fm.fm_decode_attention(q.to(DEV), res, None, count).cpu().numpy()
+    else:
+        o = fm.fm_decode_attention(q.to(DEV), keys.to(DEV), idx, count).cpu().numpy()
     # the oracle attends over exactly the chunks the index list holds (the first max_sel kept)
     used = np.zeros_like(keep)
     idx_h, cnt_h = idx.cpu().numpy(), count.cpu().numpy()
