@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--workload", default="4",
                     help="index of the synthetic workload (0-4), or 'all': one JSON line per workload")
     ap.add_argument("--q-pieces", type=int, default=2)
+    ap.add_argument("--cta-pairs", type=int, default=0, choices=[0, 1],
+                    help="scoring pass on CTA pairs (tcgen05 cta_group::2); 0 is the default form")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -214,7 +216,8 @@ def run_ours(args, wl, rank, world, local_rank):
     torch.cuda.set_device(dev)
     inp = G.make_query_inputs(wl)
     B, N, L = wl.B, wl.N, G.N_LAYERS
-    r = fm.Retriever(inp.weights, device=local_rank, max_batch=max(64, B), q_pieces=args.q_pieces)
+    r = fm.Retriever(inp.weights, device=local_rank, max_batch=max(64, B), q_pieces=args.q_pieces,
+                     cta_pairs=args.cta_pairs)
     hidden = inp.hidden.to(dev)
     positions = inp.positions.to(dev)
     n_valid = inp.n_valid.to(dev)
@@ -732,10 +735,12 @@ def run_reference(args, wl):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def config_of(wl, gpus, flush=None, key_bytes=None, shared_keys=False):
+def config_of(wl, gpus, flush=None, key_bytes=None, shared_keys=False, cta_pairs=0):
     c = {"workload": wl.name + ("_shared_keys" if shared_keys else ""), "global_batch": wl.B * gpus, "chunks_per_row": wl.N, "layers": 3,
          "ensemble": wl.mode, "top_k": wl.top_k, "threshold": wl.threshold,
          "query_prep_in_step": True, "parallelism": f"rows sharded over {gpus} GPU(s), no collective"}
+    if cta_pairs:
+        c["scoring_form"] = "CTA pairs (tcgen05 cta_group::2)"
     if flush is not None:
         c["l2"] = ("flushed between steps (256 MB written, then read back)" if flush
                    else f"inputs larger than L2 ({key_bytes / 1e9:.2f} GB of keys per step)")
@@ -786,7 +791,7 @@ def result_line(args, wl, world, res):
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "e4m3",
            "data": "synthetic (seeded generator, random-init weights)",
-           "config": config_of(wl, world, res["flush"], res["key_bytes"], args.shared_keys),
+           "config": config_of(wl, world, res["flush"], res["key_bytes"], args.shared_keys, args.cta_pairs),
            "roofline": res["roofline"], "stages_ms": res["stages_ms"], "e2e": res["e2e"],
            "gpu_launches": res["launches"],
            "clocks": res["clocks"], "cpu_baseline": res["cpu"]}

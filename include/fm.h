@@ -62,7 +62,7 @@ enum { FM_ENSEMBLE_MAX = 0, FM_ENSEMBLE_MEAN = 1 };
  * give Q_LORA_RANK and N_HEADS is missing from the pages, so they are inputs
  * (1024 and 64 in every shipped workload).  Supported: hidden % 128 == 0,
  * q_lora_rank % 128 == 0, n_heads == 64, head_dim == 128, rope_dim == 64,
- * 1 <= n_layers <= 4, 1 <= max_batch <= 4096, q_pieces in {2, 3}. */
+ * 1 <= n_layers <= 4, 1 <= max_batch <= 4096, q_pieces in {2, 3}, cta_pairs in {0, 1}. */
 typedef struct fm_config {
   int hidden;             /* 4096 */
   int q_lora_rank;        /* 1024 */
@@ -84,6 +84,13 @@ typedef struct fm_config {
                              scores within ~5e-4 on the shipped workloads) or
                              3 (~2^-12, ~1e-5; one accumulator per piece,
                              slower) */
+  int cta_pairs;          /* scoring pass with q_pieces 2 and one key tensor
+                             per layer: 0 (default) one CTA per SM issues its
+                             own MMAs; 1 pairs of CTAs share each MMA
+                             (tcgen05 cta_group::2, M = 256 chunks), which
+                             halves the MMA instructions per SM but couples
+                             the two SMs' key streams; same results.  Other
+                             forms ignore it. */
 } fm_config;
 
 /* One layer's weights, fp32, row-major [out, in], no biases (README
@@ -101,7 +108,7 @@ typedef struct fm_ctx fm_ctx;
 
 /* Fills *cfg with the shipped constants (hidden 4096, rank 1024, 64 heads,
  * head_dim 128, 3 layers, YaRN 160000/16/65536/32/1, eps 1e-6, max_batch 64,
- * q_pieces 2). */
+ * q_pieces 2, cta_pairs 0). */
 void fm_config_default(fm_config* cfg);
 
 /* Creates a context on `device`: uploads the weights (cfg->n_layers entries of

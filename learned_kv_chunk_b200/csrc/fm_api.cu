@@ -57,6 +57,7 @@ fm_status check_config(const fm_config* c) {
   if (c->n_heads != kHeads || c->head_dim != kHeadDim || c->rope_dim != kRopeDim)
     return FM_ERR_UNSUPPORTED;
   if (c->q_pieces != 2 && c->q_pieces != 3) return FM_ERR_INVALID_ARG;
+  if (c->cta_pairs != 0 && c->cta_pairs != 1) return FM_ERR_INVALID_ARG;
   if (!(c->rope_base > 1.0) || !(c->rope_factor >= 1.0) || !(c->rope_orig_max_pos > 0) ||
       !(c->rope_beta_fast > 0) || !(c->rope_beta_slow > 0) || !(c->rms_eps >= 0.f))
     return FM_ERR_INVALID_ARG;
@@ -128,6 +129,7 @@ void fm_config_default(fm_config* c) {
   c->rms_eps = 1e-6f;
   c->max_batch = 64;
   c->q_pieces = 2;
+  c->cta_pairs = 0;
 }
 
 fm_status fm_create(const fm_config* cfg, const fm_layer_weights* w, int device, fm_ctx** out) {

@@ -104,14 +104,15 @@ struct Layout {
   uint32_t q_off, raw_off, wp_off, bar_off, misc_off, total;
 };
 
-__host__ __device__ inline Layout make_layout(int L, int P, int NR, int NA) {
+// qheads: query rows per piece held by this CTA (64, or 32 for a CTA pair)
+__host__ __device__ inline Layout make_layout(int L, int P, int NR, int NA, int qheads = kHeads) {
   Layout s;
   uint32_t o = 0;
-  s.q_off = o;    o += (uint32_t)L * P * kPieceBytes;                  // multiple of 1024
+  s.q_off = o;    o += (uint32_t)L * P * (uint32_t)qheads * kHeadDim;  // multiple of 1024
   s.raw_off = o;  o += (uint32_t)NR * kRawBytes;                       // 128-aligned stages
   s.wp_off = o;   o += 2u * kQuarters * (uint32_t)L * kHeads * 4;     // per epilogue warp
   o = (o + 7u) & ~7u;
-  s.bar_off = o;  o += (uint32_t)(2 * NR + 2 * NA + 8 + 3) * 8;
+  s.bar_off = o;  o += (uint32_t)(2 * NR + 2 * NA + 8 + 4) * 8;
   s.misc_off = o; o += 64;
   s.total = o + 1024;  // slack to align the base to 1024
   return s;
@@ -119,8 +120,98 @@ __host__ __device__ inline Layout make_layout(int L, int P, int NR, int NA) {
 
 struct Bars {
   uint64_t *raw_full, *raw_empty, *a_full, *a_empty, *acc_full, *acc_empty, *q_full, *q_empty,
-      *done;
+      *done, *q_peer;
 };
+
+// ------------------------------------------------------------ CTA pairs
+// The pair form (cta_group::2): two CTAs of a cluster share each MMA, M = 256
+// chunks (128 in each CTA's TMEM), so one instruction does the work of two.
+// The leader (cluster rank 0) issues every MMA and commit; each CTA copies
+// and stores its own key tile and holds half of the query (32 heads per
+// piece); the MMA reads both halves.  The peer's transform and epilogue
+// warps signal the leader's barriers across the cluster; the commits arrive
+// on the barrier of the same offset in both CTAs.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Shared-memory address of `p` in the CTA of cluster rank `rank`.
+__device__ __forceinline__ uint32_t cluster_smem(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// Arrive on a barrier of either CTA of the pair.  Default (CTA-scope release)
+// semantics: a cluster-scope release waits for every earlier write of the
+// thread (the epilogue's score stores) to become visible to the cluster,
+// which cost each transform and epilogue step over a thousand cycles; what
+// the arrival publishes is ordered by the tcgen05 fences around it (the
+// TMEM stores before it, the MMA after the leader's wait).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void umma_f8f6f4_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                    uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrives on `bar` (same offset) in both CTAs of the pair once every MMA this
+// thread issued before has completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  const uint16_t mask = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// mbarrier wait with cluster-scope acquire (for barriers the peer arrives on)
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                          int* err, uint64_t limit_ns) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        atomicExch(err, kDevErrTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
 
 // Position in a ring of n stages: the stage index and the parity of the
 // stage's mbarrier phase for the current pass.  Advanced once per item, so no
@@ -133,10 +224,11 @@ struct Ring {
   }
 };
 
-// Walks this CTA's contiguous range of valid (row, tile) units.
+// Walks this CTA's contiguous range of valid (row, unit) units; a unit is
+// one 128-chunk tile, or for a CTA pair two (the tile of each CTA).
 struct UnitWalk {
   const int32_t* n_valid;
-  int N, B;
+  int N, B, span;  // span: chunks per unit
   int b, t, nv, tiles;
   int64_t left;
   __device__ int nvalid_of(int row) const {
@@ -145,7 +237,7 @@ struct UnitWalk {
   }
   __device__ void start(int b0, int t0, int64_t count) {
     b = b0; t = t0; left = count;
-    if (left > 0) { nv = nvalid_of(b); tiles = (nv + kTile - 1) / kTile; }
+    if (left > 0) { nv = nvalid_of(b); tiles = (nv + span - 1) / span; }
   }
   __device__ bool valid() const { return left > 0; }
   __device__ void next() {
@@ -153,7 +245,7 @@ struct UnitWalk {
     if (left <= 0) return;
     if (++t >= tiles) {
       t = 0;
-      do { ++b; nv = nvalid_of(b); tiles = (nv + kTile - 1) / kTile; } while (tiles == 0);
+      do { ++b; nv = nvalid_of(b); tiles = (nv + span - 1) / span; } while (tiles == 0);
     }
   }
 };
@@ -181,8 +273,8 @@ struct PairWalk {
       w.next();
     }
   }
-  __device__ void start(const int32_t* n_valid, int N, int B, int b0, int t0, int64_t count) {
-    w.n_valid = n_valid; w.N = N; w.B = B;
+  __device__ void start(const int32_t* n_valid, int N, int B, int b0, int t0, int64_t count, int span) {
+    w.n_valid = n_valid; w.N = N; w.B = B; w.span = span;
     w.start(b0, t0, count);
     fill();
   }
@@ -262,18 +354,23 @@ __device__ __forceinline__ float head_sum32(const HeadCols<P>& c, const float* _
 // unit's tile is copied and stored into TMEM once and every layer's MMAs read
 // it; the key ring, the TMEM key stages and the scale slots then go per unit
 // instead of per (unit, layer).
-template <int P, bool DUMP, bool SK>
+template <int P, bool DUMP, bool SK, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int NR) {
   extern __shared__ uint8_t smem_raw[];
   constexpr uint32_t ACCW = acc_cols<P>();
   constexpr uint32_t ABASE = a_col_base<P>();
   constexpr uint32_t NA = a_stages<P>();
-  const Layout lay = make_layout(args.L, P, NR, NA);
+  constexpr int kSpan = PAIR ? 2 * kTile : kTile;             // chunks per unit
+  constexpr uint32_t kQHeads = PAIR ? kHeads / 2 : kHeads;     // query rows per piece in this CTA
+  constexpr uint32_t kQPiece = kQHeads * kHeadDim;             // bytes of one piece in shared memory
+  constexpr uint32_t kArrivals = PAIR ? 2 * kQuarters : kQuarters;  // warps arriving on a_full, acc_empty
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const Layout lay = make_layout(args.L, P, NR, NA, (int)kQHeads);
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int L = args.L;
   const int LK = SK ? 1 : L;  // key tiles copied per unit
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr uint32_t kQLayerBytes = (uint32_t)P * kPieceBytes;
+  constexpr uint32_t kQLayerBytes = (uint32_t)P * kQPiece;  // one layer's query in shared memory
 
   uint8_t* sQ = smem + lay.q_off;
   uint8_t* sRaw = smem + lay.raw_off;
@@ -285,6 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
   B_.acc_full = B_.a_empty + NA;    B_.acc_empty = B_.acc_full + 4;
   B_.q_full = B_.acc_empty + 4;
   B_.q_empty = B_.q_full + 1;       B_.done = B_.q_empty + 1;
+  B_.q_peer = B_.done + 1;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + lay.misc_off);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + lay.misc_off + 4);
   int* sRange = reinterpret_cast<int*>(smem + lay.misc_off + 8);  // b0, t0, count lo, count hi
@@ -296,32 +394,35 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       mbar_init(&B_.raw_empty[i], kQuarters);  // read by all transform warps
     }
     for (uint32_t i = 0; i < NA; ++i) {
-      mbar_init(&B_.a_full[i], kQuarters);     // key tile stored in TMEM (one arrival per warp)
+      mbar_init(&B_.a_full[i], kArrivals);     // key tile stored in TMEM (one arrival per warp)
       mbar_init(&B_.a_empty[i], 1);            // the MMA that read it retired
     }
-    for (int g = 0; g < 4; ++g) { mbar_init(&B_.acc_full[g], 1); mbar_init(&B_.acc_empty[g], kQuarters); }
+    for (int g = 0; g < 4; ++g) { mbar_init(&B_.acc_full[g], 1); mbar_init(&B_.acc_empty[g], kArrivals); }
     mbar_init(B_.q_full, 1);
     mbar_init(B_.q_empty, 2);                // both MMA issuers' commits
     mbar_init(B_.done, 2);
+    mbar_init(B_.q_peer, 1);                 // pair: the peer's query half landed
     *sAbort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kWarpMma && lane == 0) {
-    // this CTA's share of the valid units: rows contribute ceil(n_b / 128) tiles
+    // this CTA's (or pair's) share of the valid units: rows contribute
+    // ceil(n_b / span) units
     int64_t total = 0;
     for (int b = 0; b < args.B; ++b) {
       int v = args.n_valid ? __ldg(args.n_valid + b) : args.N;
       v = max(0, min(v, args.N));
-      total += (v + kTile - 1) / kTile;
+      total += (v + kSpan - 1) / kSpan;
     }
-    const int64_t u0 = total * blockIdx.x / gridDim.x;
-    const int64_t u1 = total * (blockIdx.x + 1) / gridDim.x;
+    const int64_t slot = PAIR ? blockIdx.x >> 1 : blockIdx.x, slots = PAIR ? gridDim.x >> 1 : gridDim.x;
+    const int64_t u0 = total * slot / slots;
+    const int64_t u1 = total * (slot + 1) / slots;
     int64_t acc = 0;
     int b0 = 0, t0 = 0;
     for (int b = 0; b < args.B; ++b) {
       int v = args.n_valid ? __ldg(args.n_valid + b) : args.N;
       v = max(0, min(v, args.N));
-      const int tiles = (v + kTile - 1) / kTile;
+      const int tiles = (v + kSpan - 1) / kSpan;
       if (acc + tiles > u0) { b0 = b; t0 = (int)(u0 - acc); break; }
       acc += tiles;
     }
@@ -329,11 +430,17 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
     sRange[2] = (int)((u1 - u0) & 0xffffffff); sRange[3] = (int)((u1 - u0) >> 32);
   }
   if (warp == kWarpQ) {
-    tmem_alloc(sTmem, kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(sTmem, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(sTmem, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrival
   tc_fence_after();
   const uint32_t tmem_base = *sTmem;
   const int b_start = sRange[0], t_start = sRange[1];
@@ -346,20 +453,26 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       uint32_t item = 0;
       Ring raw(NR);
       bool ok = true;
-      for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); ok && pw.valid() && !*sAbort;
+      for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count, kSpan); ok && pw.valid() && !*sAbort;
            pw.next()) {
         for (int l = 0; l < LK && ok; ++l) {
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             if (j == 1 && !pw.has1) break;
             const Unit U = j == 0 ? pw.u[0] : pw.u[1];
-            const int nrem = min(kTile, U.nv - U.t * kTile);
-            const uint32_t bytes = (uint32_t)((nrem + 3) & ~3) * kRecord;
+            const int tt = PAIR ? 2 * U.t + (int)rank : U.t;  // this CTA's tile of the unit
+            const int nrem = min(kTile, U.nv - tt * kTile);
             ok = mbar_wait_bounded(&B_.raw_empty[raw.stage], raw.phase ^ 1, sAbort, args.err, args.wait_ns);
             if (!ok) break;
-            mbar_arrive_expect_tx(&B_.raw_full[raw.stage], bytes);
-            const uint8_t* src = args.comp_k[l] + (int64_t)U.b * args.row_stride + (int64_t)U.t * kRawBytes;
-            bulk_g2s(sRaw + (size_t)raw.stage * kRawBytes, src, bytes, &B_.raw_full[raw.stage]);
+            if (PAIR && nrem <= 0) {
+              // the pair's odd last tile: this CTA has none, its stage passes through unread
+              mbar_arrive(&B_.raw_full[raw.stage]);
+            } else {
+              const uint32_t bytes = (uint32_t)((nrem + 3) & ~3) * kRecord;
+              mbar_arrive_expect_tx(&B_.raw_full[raw.stage], bytes);
+              const uint8_t* src = args.comp_k[l] + (int64_t)U.b * args.row_stride + (int64_t)tt * kRawBytes;
+              bulk_g2s(sRaw + (size_t)raw.stage * kRawBytes, src, bytes, &B_.raw_full[raw.stage]);
+            }
             ++item;
             raw.advance();
           }
@@ -379,19 +492,30 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       grid_dependency_wait();  // the query image is written by the packing kernel ahead
       int cur = -1;
       uint32_t loads = 0;
-      for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); pw.valid() && !*sAbort; pw.next()) {
+      for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count, kSpan); pw.valid() && !*sAbort; pw.next()) {
         const int b = pw.u[0].b;
         if (b == cur) continue;
         if (loads > 0 && !mbar_wait_bounded(B_.q_empty, (loads - 1) & 1, sAbort, args.err, args.wait_ns)) break;
         mbar_arrive_expect_tx(B_.q_full, (uint32_t)L * kQLayerBytes);
+        // piece p of layer l: this CTA's heads (all 64, or 32 rank .. of a pair)
         for (int l = 0; l < L; ++l)
-          bulk_g2s(sQ + (size_t)l * kQLayerBytes, args.qpack + ((size_t)b * L + l) * kQLayerBytes,
-                   kQLayerBytes, B_.q_full);
+          for (int pc = 0; pc < P; ++pc)
+            bulk_g2s(sQ + (size_t)l * kQLayerBytes + (size_t)pc * kQPiece,
+                     args.qpack + (((size_t)b * L + l) * P + pc) * kPieceBytes + (size_t)rank * kQPiece, kQPiece,
+                     B_.q_full);
+        if (PAIR && rank == 1) {  // tell the leader, which issues the MMAs, that this half landed
+          if (!mbar_wait_bounded(B_.q_full, loads & 1, sAbort, args.err, args.wait_ns)) break;
+          mbar_arrive_remote(cluster_smem(B_.q_peer, 0));
+        }
         cur = b;
         ++loads;
       }
       if (loads > 0) mbar_drain(B_.q_full, (loads - 1) & 1, args.err);
     }
+  } else if ((warp == kWarpMma || warp == kWarpMma2) && PAIR && rank != 0) {
+    // pair peer: the leader issues; wait for every MMA that uses this CTA's
+    // TMEM and shared memory to retire before they go away
+    if (lane == 0) mbar_drain(B_.done, 0, args.err);
   } else if (warp == kWarpMma || warp == kWarpMma2) {
     // --------------------------------------------------------- MMA issuers
     // Two issuing threads on two schedulers, one per epilogue group: thread
@@ -402,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
     // stage and phase.
     if (lane == 0) {
       const int me = warp == kWarpMma ? 0 : 1;
-      constexpr uint32_t idesc = idesc_e4m3_f32(kMmaM, (int)ACCW);  // N = 64 with the pieces folded
+      constexpr uint32_t idesc = idesc_e4m3_f32(PAIR ? 2 * kMmaM : kMmaM, (int)ACCW);  // N = 64 with the pieces folded
       // B descriptors: the start-address field counts 16-byte units, so the
       // layer and K-step offsets are plain adds (the field cannot carry: the
       // query image lies in the first 256 KB of shared memory)
@@ -412,10 +536,11 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       Ring ast(NA);
       int cur = -1;
       bool ok = true;
-      for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); ok && pw.valid() && !*sAbort;) {
+      for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count, kSpan); ok && pw.valid() && !*sAbort;) {
         const int b = pw.u[0].b;
         if (b != cur) {
           if (!mbar_wait_bounded(B_.q_full, rows & 1, sAbort, args.err, args.wait_ns)) break;
+          if (PAIR && !mbar_wait_cluster_bounded(B_.q_peer, rows & 1, sAbort, args.err, args.wait_ns)) break;
           ++rows;
           cur = b;
         }
@@ -434,25 +559,38 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
             const uint32_t st = acc_stages<P>() == 2 ? (gcnt & 1u) : 0u;
             const uint32_t slot_i = (uint32_t)j * acc_stages<P>() + st;
             const uint32_t ph = (phs >> st) & 1u;
-            ok = ((SK && l > 0) || mbar_wait_bounded(&B_.a_full[as.stage], as.phase, sAbort, args.err, args.wait_ns)) &&
-                 mbar_wait_bounded(&B_.acc_empty[slot_i], ph ^ 1, sAbort, args.err, args.wait_ns);
+            if constexpr (PAIR)
+              ok = mbar_wait_cluster_bounded(&B_.a_full[as.stage], as.phase, sAbort, args.err, args.wait_ns) &&
+                   mbar_wait_cluster_bounded(&B_.acc_empty[slot_i], ph ^ 1, sAbort, args.err, args.wait_ns);
+            else
+              ok = ((SK && l > 0) ||
+                    mbar_wait_bounded(&B_.a_full[as.stage], as.phase, sAbort, args.err, args.wait_ns)) &&
+                   mbar_wait_bounded(&B_.acc_empty[slot_i], ph ^ 1, sAbort, args.err, args.wait_ns);
             if (!ok) break;
             tc_fence_after();
             const uint32_t d = tmem_base + slot_i * ACCW;
             const uint32_t a = tmem_base + ABASE + as.stage * kACols;
-            umma_f8f6f4_ts(d, a, bd, idesc, 0u);
-            umma_f8f6f4_ts(d, a + 8u, bd + kKStep, idesc, 1u);
-            umma_f8f6f4_ts(d, a + 16u, bd + 2 * kKStep, idesc, 1u);
-            umma_f8f6f4_ts(d, a + 24u, bd + 3 * kKStep, idesc, 1u);
-            if constexpr (fold<P>()) {  // piece 1 (rows 64..127 of the layer's image) into the same accumulator
-              const uint64_t bd1 = bd + (kPieceBytes >> 4);
-              umma_f8f6f4_ts(d, a, bd1, idesc, 1u);
-              umma_f8f6f4_ts(d, a + 8u, bd1 + kKStep, idesc, 1u);
-              umma_f8f6f4_ts(d, a + 16u, bd1 + 2 * kKStep, idesc, 1u);
-              umma_f8f6f4_ts(d, a + 24u, bd1 + 3 * kKStep, idesc, 1u);
+            const auto mma = [&](uint32_t aa, uint64_t bb, uint32_t acc) {
+              if constexpr (PAIR) umma_f8f6f4_ts_pair(d, aa, bb, idesc, acc);
+              else umma_f8f6f4_ts(d, aa, bb, idesc, acc);
+            };
+            const auto commit = [&](uint64_t* bar) {
+              if constexpr (PAIR) umma_commit_pair(bar);
+              else umma_commit(bar);
+            };
+            mma(a, bd, 0u);
+            mma(a + 8u, bd + kKStep, 1u);
+            mma(a + 16u, bd + 2 * kKStep, 1u);
+            mma(a + 24u, bd + 3 * kKStep, 1u);
+            if constexpr (fold<P>()) {  // piece 1 of the layer's image into the same accumulator
+              const uint64_t bd1 = bd + (kQPiece >> 4);
+              mma(a, bd1, 1u);
+              mma(a + 8u, bd1 + kKStep, 1u);
+              mma(a + 16u, bd1 + 2 * kKStep, 1u);
+              mma(a + 24u, bd1 + 3 * kKStep, 1u);
             }
-            if (!SK || l == L - 1) umma_commit(&B_.a_empty[as.stage]);  // the TMEM key tile may be overwritten
-            umma_commit(&B_.acc_full[slot_i]);
+            if (!SK || l == L - 1) commit(&B_.a_empty[as.stage]);  // the TMEM key tile may be overwritten
+            commit(&B_.acc_full[slot_i]);
             ++item;
             if (!SK) ast.advance();
             phs ^= 1u << st;
@@ -465,10 +603,14 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
           if (pw.has1) ast.advance();
         }
         pw.next();
-        if (!pw.valid() || pw.u[0].b != b) umma_commit(B_.q_empty);
+        if (!pw.valid() || pw.u[0].b != b) {
+          if constexpr (PAIR) umma_commit_pair(B_.q_empty);
+          else umma_commit(B_.q_empty);
+        }
       }
       {  // every issued MMA and commit retired before TMEM and smem go away (both issuers arrive)
-        umma_commit(B_.done);
+        if constexpr (PAIR) umma_commit_pair(B_.done);
+        else umma_commit(B_.done);
         mbar_drain(B_.done, 0, args.err);
       }
     }
@@ -487,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
     Ring raw(NR), ast(NA);
     uint32_t gtiles[2] = {0u, 0u};  // key tiles of each group so far
     bool go = true;
-    for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); go && pw.valid(); pw.next())
+    for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count, kSpan); go && pw.valid(); pw.next())
     for (int l = 0; l < LK && go; ++l)
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -515,7 +657,8 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&B_.raw_empty[raw.stage]);
-        mbar_arrive(&B_.a_full[ast.stage]);
+        if constexpr (PAIR) mbar_arrive_remote(cluster_smem(&B_.a_full[ast.stage], 0));
+        else mbar_arrive(&B_.a_full[ast.stage]);
       }
       ++gtiles[j];
       raw.advance();
@@ -534,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
         tmem_base + ((uint32_t)(quarter * 32) << 16) + kScaleCol + (uint32_t)group * kGroupSlots;
     uint32_t phs = 0, gtiles = 0, gitems = 0;  // gtiles: this group's key tiles so far (its scale slots)
     int cur = -1;
-    for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count); pw.valid(); pw.next()) {
+    for (pw.start(args.n_valid, args.N, args.B, b_start, t_start, count, kSpan); pw.valid(); pw.next()) {
       if (group == 1 && !pw.has1) continue;
       const Unit U = group == 0 ? pw.u[0] : pw.u[1];
       if (U.b != cur) {  // this warp's private copy of the row's head weights
@@ -544,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
         __syncwarp();
         cur = U.b;
       }
-      const int n = U.t * kTile + r;
+      const int n = (PAIR ? 2 * U.t + (int)rank : U.t) * kTile + r;
       const bool valid = n < U.nv;
       const bool in_row = n < args.N;
       float ens = 0.f;
@@ -575,7 +718,10 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
         // the accumulator stage is free once this warp holds all its columns
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B_.acc_empty[slot_i]);
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_remote(cluster_smem(&B_.acc_empty[slot_i], 0));
+          else mbar_arrive(&B_.acc_empty[slot_i]);
+        }
         if constexpr (DUMP) {
           if (U.b == args.dbg_b && U.t == args.dbg_t && l == args.dbg_layer)
             for (int p = 0; p < acc_pieces<P>(); ++p)
@@ -616,13 +762,15 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(ScoreArgs args, int 
   // ------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // neither CTA leaves while the other may still signal it
   if (warp == kWarpQ) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
-template <int P, bool DUMP, bool SK>
+template <int P, bool DUMP, bool SK, bool PAIR>
 fm_status launch_score_p(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t st) {
   if (a.wait_ns == 0) return FM_ERR_INVALID_ARG;  // every wait needs a bound that lets work finish
   static PerDeviceOnce smem_set;
@@ -633,20 +781,75 @@ fm_status launch_score_p(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t st) {
   // deepest key ring that fits: every stage is keys in flight
   int NR = 16;
   constexpr int NA = (int)a_stages<P>();
-  Layout lay = make_layout(a.L, P, NR, NA);
+  constexpr int kQHeads = PAIR ? kHeads / 2 : kHeads;
+  Layout lay = make_layout(a.L, P, NR, NA, kQHeads);
   while (lay.total > (uint32_t)max_smem && NR > 2) {
     --NR;
-    lay = make_layout(a.L, P, NR, NA);
+    lay = make_layout(a.L, P, NR, NA, kQHeads);
   }
   if (lay.total > (uint32_t)max_smem) return FM_ERR_UNSUPPORTED;
-  if (fm_status s = smem_limit_once(smem_set, ctx->device, score_kernel<P, DUMP, SK>, max_smem)) return s;
-  const int64_t units = (int64_t)a.B * ((a.N + kTile - 1) / kTile);  // upper bound
+  if (fm_status s = smem_limit_once(smem_set, ctx->device, score_kernel<P, DUMP, SK, PAIR>, max_smem)) return s;
+  const int span = PAIR ? 2 * kTile : kTile;
+  const int64_t units = (int64_t)a.B * ((a.N + span - 1) / span);  // upper bound
   int grid = ctx->num_sms;
-  if (units < grid) grid = (int)(units > 0 ? units : 1);
+  if constexpr (PAIR) {
+    // the CTAs are persistent, so every pair must be resident at once: as
+    // many pairs as the device holds together (a GPC with an odd number of
+    // SMs leaves one SM out), found once per device
+    static PerDeviceOnce pairs_set;
+    static std::atomic<int> max_pairs[64];
+    const int dev = ctx->device;
+    if (fm_status s = pairs_set.run(dev, [&]() -> fm_status {
+          cudaLaunchAttribute ca[1];
+          ca[0].id = cudaLaunchAttributeClusterDimension;
+          ca[0].val.clusterDim.x = 2;
+          ca[0].val.clusterDim.y = 1;
+          ca[0].val.clusterDim.z = 1;
+          cudaLaunchConfig_t qc = {};
+          qc.gridDim = dim3(grid & ~1);
+          qc.blockDim = dim3(kThreads);
+          qc.dynamicSmemBytes = lay.total;
+          qc.attrs = ca;
+          qc.numAttrs = 1;
+          int n = 0;
+          const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, score_kernel<P, DUMP, SK, PAIR>, &qc);
+          if (e != cudaSuccess) return record_cuda_error(e);
+          if (dev >= 0 && dev < 64) max_pairs[dev].store(n);
+          return FM_OK;
+        }))
+      return s;
+    const int pairs = dev >= 0 && dev < 64 ? max_pairs[dev].load() : 0;
+    if (pairs < 1) return FM_ERR_UNSUPPORTED;
+    grid = 2 * (pairs < ctx->num_sms / 2 ? pairs : ctx->num_sms / 2);
+    if (units * 2 < grid) grid = (int)(units > 0 ? units * 2 : 2);
+  } else if (units < grid) {
+    grid = (int)(units > 0 ? units : 1);
+  }
   // the packing kernel ahead of this one writes only the query image and the
   // head weights, which the query loader and the epilogue wait for; the key
   // stream starts while it runs
-  const cudaError_t e = launch_overlapped(score_kernel<P, DUMP, SK>, dim3(grid), dim3(kThreads), lay.total, st, a, NR);
+  cudaError_t e;
+  if constexpr (PAIR) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return record_cuda_error(cudaGetLastError());
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = lay.total;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = cap == cudaStreamCaptureStatusNone ? 2 : 1;
+    e = cudaLaunchKernelEx(&cfg, score_kernel<P, DUMP, SK, PAIR>, a, NR);
+  } else {
+    e = launch_overlapped(score_kernel<P, DUMP, SK, PAIR>, dim3(grid), dim3(kThreads), lay.total, st, a, NR);
+  }
   note_launch();
   return e == cudaSuccess ? check_launch() : record_cuda_error(e);
 }
@@ -655,15 +858,16 @@ fm_status launch_score_p(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t st) {
 
 fm_status launch_score(fm_ctx* ctx, const ScoreArgs& a, cudaStream_t st) {
   if (a.dbg_out)
-    return ctx->cfg.q_pieces == 3 ? launch_score_p<3, true, false>(ctx, a, st)
-                                  : launch_score_p<2, true, false>(ctx, a, st);
+    return ctx->cfg.q_pieces == 3 ? launch_score_p<3, true, false, false>(ctx, a, st)
+                                  : launch_score_p<2, true, false, false>(ctx, a, st);
   bool shared = a.L > 1;
   for (int l = 1; l < a.L; ++l) shared = shared && a.comp_k[l] == a.comp_k[0];
   if (shared)
-    return ctx->cfg.q_pieces == 3 ? launch_score_p<3, false, true>(ctx, a, st)
-                                  : launch_score_p<2, false, true>(ctx, a, st);
-  return ctx->cfg.q_pieces == 3 ? launch_score_p<3, false, false>(ctx, a, st)
-                                : launch_score_p<2, false, false>(ctx, a, st);
+    return ctx->cfg.q_pieces == 3 ? launch_score_p<3, false, true, false>(ctx, a, st)
+                                  : launch_score_p<2, false, true, false>(ctx, a, st);
+  if (ctx->cfg.q_pieces == 3) return launch_score_p<3, false, false, false>(ctx, a, st);
+  return ctx->cfg.cta_pairs ? launch_score_p<2, false, false, true>(ctx, a, st)
+                            : launch_score_p<2, false, false, false>(ctx, a, st);
 }
 
 }  // namespace fm

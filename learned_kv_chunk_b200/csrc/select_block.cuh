@@ -3,9 +3,9 @@
 // or a whole candidate list's) keys in shared memory at once.
 //
 // Keys are the order-preserving 32-bit images of fp32 scores (larger float ->
-// larger key, +0 and -0 equal, NaN lowest).  Three passes (11 + 11 + 10 bits,
-// most significant first) fix the want-th largest key T and how many keys
-// equal to T it takes.  Every function here must be called by all
+// larger key, +0 and -0 equal, NaN lowest).  Histogram passes over the
+// undecided bits (most significant first) fix the want-th largest key T and
+// how many keys equal to T it takes.  Every function here must be called by all
 // kBlkThreads threads of the block (they synchronise it).
 #pragma once
 
@@ -61,47 +61,86 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
 // The want-th largest of the keys key_at(0 .. n-1) (1 <= want <= n): *T
 // receives it and *need how many of the keys equal to T are among the want
 // largest.  key_at reads a key from shared or global memory.
+//
+// The keys share every bit above the highest bit in which their maximum and
+// minimum differ, so the passes start there: each pass histograms the next
+// (up to) 11 undecided bits of the keys that match the bits decided so far
+// and picks the digit holding the want-th largest.  Once the picked digit
+// holds at most kSelFinish keys, they are gathered and ranked directly.
+constexpr int kSelFinish = 256;
+
 template <class KeyAt>
 __device__ __forceinline__ void block_kth_largest_of(KeyAt key_at, int n, uint32_t want, BlockSelScratch sc,
                                                      uint32_t* T, int* need) {
-  const int t = threadIdx.x;
-  uint32_t prefix = 0u;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  constexpr int W = kBlkThreads / 32;
+  uint32_t kmax = 0u, kmin = 0xffffffffu;
+  for (int i = t; i < n; i += kBlkThreads) {
+    const uint32_t k = key_at(i);
+    kmax = max(kmax, k);
+    kmin = min(kmin, k);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+  }
+  if (lane == 0) {
+    sc.hist[warp] = kmax;
+    sc.hist[W + warp] = kmin;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < W; ++i) {
+    kmax = max(kmax, sc.hist[i]);
+    kmin = min(kmin, sc.hist[W + i]);
+  }
+  __syncthreads();
+  if (kmax == kmin) {  // every key equal
+    *T = kmax;
+    *need = (int)want;
+    return;
+  }
+  int lo = 32 - __clz(kmax ^ kmin);  // bits [0, lo) undecided
+  uint32_t prefix = lo >= 32 ? 0u : (kmax >> lo) << lo;
+  const unsigned lane_lt = (1u << lane) - 1u;
 #pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0), nbits = pass == 2 ? 10 : 11;
-    const int nb = 1 << nbits, hi = shift + nbits;
+  while (lo > 0) {
+    const int nbits = lo < 11 ? lo : 11, shift = lo - nbits, nb = 1 << nbits;
     for (int i = t; i < nb; i += kBlkThreads) sc.hist[i] = 0u;
     __syncthreads();
-    // Keys that reach a selection crowd into a few digits (scores near the
-    // cut share their leading bits), so lanes holding the same digit add to
-    // the histogram with one atomic.
-    const unsigned lane_lt = (1u << (t & 31)) - 1u;
+    // lanes holding the same digit add to the histogram with one atomic
     for (int i0 = 0; i0 < n; i0 += kBlkThreads) {
       const int i = i0 + t;
       const uint32_t key = i < n ? key_at(i) : 0u;
-      const bool act = i < n && (hi >= 32 || (key >> hi) == (prefix >> hi));
+      const bool act = i < n && (lo >= 32 || (key >> lo) == (prefix >> lo));
       const unsigned active = __ballot_sync(0xffffffffu, act);
       if (act) {
-        const uint32_t bin = (key >> shift) & (nb - 1);
+        const uint32_t bin = (key >> shift) & (uint32_t)(nb - 1);
         const unsigned peers = __match_any_sync(active, bin);
         if ((peers & lane_lt) == 0) atomicAdd(&sc.hist[bin], (uint32_t)__popc(peers));
       }
     }
     __syncthreads();
     // thread t owns bins [t*per, (t+1)*per) in descending digit order
-    const int per = nb / kBlkThreads;
+    const int per = (nb + kBlkThreads - 1) / kBlkThreads;
     uint32_t mine = 0;
-    for (int j = 0; j < per; ++j) mine += sc.hist[nb - 1 - (t * per + j)];
+    for (int j = 0; j < per; ++j) {
+      const int d = nb - 1 - (t * per + j);
+      if (d >= 0) mine += sc.hist[d];
+    }
     int tot;
     const uint32_t before = (uint32_t)block_exclusive_scan((int)mine, sc.warp, &tot);
     if (before < want && before + mine >= want) {
       uint32_t acc = before;
       for (int j = 0; j < per; ++j) {
         const int d = nb - 1 - (t * per + j);
+        if (d < 0) break;
         const uint32_t c = sc.hist[d];
         if (acc + c >= want) {
           sc.pick[0] = prefix | ((uint32_t)d << shift);
           sc.pick[1] = want - acc;
+          sc.warp[W] = (int)c;  // keys in the picked digit
           break;
         }
         acc += c;
@@ -110,7 +149,38 @@ __device__ __forceinline__ void block_kth_largest_of(KeyAt key_at, int n, uint32
     __syncthreads();
     prefix = sc.pick[0];
     want = sc.pick[1];
+    const int cnt = sc.warp[W];
+    lo = shift;
     __syncthreads();
+    if (lo > 0 && cnt <= kSelFinish) {
+      // gather the picked digit's keys and rank them directly
+      uint32_t* list = sc.hist;
+      uint32_t* fill = sc.hist + kSelFinish;
+      if (t == 0) *fill = 0u;
+      __syncthreads();
+      for (int i = t; i < n; i += kBlkThreads) {
+        const uint32_t key = key_at(i);
+        if ((key >> lo) == (prefix >> lo)) list[atomicAdd(fill, 1u)] = key;
+      }
+      __syncthreads();
+      for (int e = t; e < cnt; e += kBlkThreads) {
+        const uint32_t k = list[e];
+        uint32_t gt = 0, eq = 0;
+        for (int f = 0; f < cnt; ++f) {
+          gt += list[f] > k ? 1u : 0u;
+          eq += list[f] == k ? 1u : 0u;
+        }
+        if (gt < want && want <= gt + eq) {  // every key equal to k writes the same values
+          sc.pick[0] = k;
+          sc.pick[1] = want - gt;
+        }
+      }
+      __syncthreads();
+      prefix = sc.pick[0];
+      want = sc.pick[1];
+      __syncthreads();
+      break;
+    }
   }
   *T = prefix;
   *need = (int)want;

@@ -31,7 +31,7 @@ class fm_config(ctypes.Structure):
                 ("rope_base", ctypes.c_double), ("rope_factor", ctypes.c_double),
                 ("rope_orig_max_pos", ctypes.c_double), ("rope_beta_fast", ctypes.c_double),
                 ("rope_beta_slow", ctypes.c_double), ("rms_eps", ctypes.c_float),
-                ("max_batch", ctypes.c_int), ("q_pieces", ctypes.c_int)]
+                ("max_batch", ctypes.c_int), ("q_pieces", ctypes.c_int), ("cta_pairs", ctypes.c_int)]
 
 
 class fm_layer_weights(ctypes.Structure):

@@ -63,6 +63,7 @@ def test_config_defaults(lib):
     assert (c.rope_beta_fast, c.rope_beta_slow) == (32.0, 1.0)
     assert abs(c.rms_eps - 1e-6) < 1e-12
     assert c.q_pieces in (2, 3) and c.max_batch >= 1
+    assert c.cta_pairs == 0
 
 
 def test_topk_workspace_sizing(lib):

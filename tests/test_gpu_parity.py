@@ -23,9 +23,10 @@ def weights():
     return G.make_weights(4242, 3)
 
 
-@pytest.fixture(scope="module", params=[3, 2], ids=["pieces3", "pieces2"])
+@pytest.fixture(scope="module", params=[(3, 0), (2, 0), (2, 1)], ids=["pieces3", "pieces2", "pieces2_cta_pairs"])
 def retr(request, weights):
-    r = fm.Retriever(weights, device=0, max_batch=64, q_pieces=request.param)
+    pieces, pairs = request.param
+    r = fm.Retriever(weights, device=0, max_batch=64, q_pieces=pieces, cta_pairs=pairs)
     yield r
     r.close()
 
