@@ -327,12 +327,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
+    // The unit's tile coordinates advance incrementally: divisions run once
+    // per tile, not per unit (a dependent chain of integer divisions cost
+    // this single thread ~0.6 us per unit, longer than the copies took).
     uint32_t stage = 0, phase = 0, issued = 0;
+    int t = (int)(u0 / sk.KB), kb = (int)(u0 - (int64_t)t * sk.KB);
+    int m0 = 0, n0 = 0, layer = 0;
+    const auto tile_coords = [&]() {
+      m0 = (t % sk.mtiles) * kTcBM;
+      n0 = (t / sk.mtiles) * BN;
+      layer = a.rows_per_layer ? m0 / a.rows_per_layer : 0;
+    };
+    tile_coords();
     for (int64_t u = u0; u < u1; ++u) {
       if (!mbar_wait_bounded(&empty[stage], phase ^ 1, sAbort, a.err)) break;
-      const int t = (int)(u / sk.KB), kb = (int)(u - (int64_t)t * sk.KB);
-      const int m0 = (t % sk.mtiles) * kTcBM, n0 = (t / sk.mtiles) * BN;
-      const int layer = a.rows_per_layer ? m0 / a.rows_per_layer : 0;
       const int k = kb * kTcBK;
       uint8_t* st = smem + (size_t)stage * kStage;
       mbar_arrive_expect_tx(&full[stage], kStage);
@@ -341,6 +349,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tma_load_3d(st + kTcWTile + kXTile, &x_lo, k, layer, n0, &full[stage]);
       ++issued;
       if (++stage == (uint32_t)S) { stage = 0; phase ^= 1u; }
+      if (++kb == sk.KB) {
+        kb = 0;
+        ++t;
+        tile_coords();
+      }
     }
     // every copy issued lands before the CTA can exit
     const uint32_t inflight = issued < (uint32_t)S ? issued : (uint32_t)S;

@@ -193,13 +193,18 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__
   for (int64_t r0 = gw * RU; r0 < total; r0 += nw * RU) {
     const U* s[RU];
     U* d[RU];
+    // (row, slot) of record r0, then stepped: one division per round
+    int b = (int)(r0 / max_sel), j = (int)(r0 - (int64_t)b * max_sel);
 #pragma unroll
-    for (int q = 0; q < RU; ++q) {
+    for (int q = 0; q < RU; ++q, ++j) {
       s[q] = nullptr;
       d[q] = nullptr;
+      if (j == max_sel) {
+        j = 0;
+        ++b;
+      }
       const int64_t r = r0 + q;
       if (r < total) {
-        const int b = (int)(r / max_sel), j = (int)(r - (int64_t)b * max_sel);
         const int cnt = min(__ldg(count + b), max_sel);
         const int id = __ldg(idx + r);  // in bounds whatever the count: loaded beside it, not after it
         const int n = j < cnt ? id : -1;
