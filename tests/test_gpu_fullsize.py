@@ -21,9 +21,9 @@ from learned_kv_chunk_b200 import fm  # noqa: E402
 DEV = torch.device("cuda", 0)
 
 
-def _run(wl):
+def _run(wl, cta_pairs=0):
     case = H.workload_case(wl, key_device=DEV)
-    r = fm.Retriever(case.weights, device=0, max_batch=max(64, wl.B))
+    r = fm.Retriever(case.weights, device=0, max_batch=max(64, wl.B), cta_pairs=cta_pairs)
     try:
         q, w = r.fm_query_prep(case.hidden.to(DEV), case.positions.to(DEV))
         nv = case.n_valid.to(DEV)
@@ -38,9 +38,12 @@ def _run(wl):
         raise
 
 
-@pytest.mark.parametrize("wl", G.WORKLOADS[1:], ids=[w.name for w in G.WORKLOADS[1:]])
-def test_full_size_workload(wl):
-    case, r, q, w, ens, keep, keep_thr = _run(wl)
+@pytest.mark.parametrize("wl,cta_pairs", [(w, 0) for w in G.WORKLOADS[1:]] + [(G.WORKLOADS[3], 1)],
+                         ids=[w.name for w in G.WORKLOADS[1:]] + [G.WORKLOADS[3].name + "_cta_pairs"])
+def test_full_size_workload(wl, cta_pairs):
+    """cta_pairs: the scoring pass on CTA pairs, on the ragged rows whose odd
+    tile counts leave the pair's second CTA without a tile at a row's end."""
+    case, r, q, w, ens, keep, keep_thr = _run(wl, cta_pairs)
     try:
         nv = case.n_valid.numpy()
         e_gpu = ens.cpu().numpy()
