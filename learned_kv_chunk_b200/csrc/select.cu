@@ -489,12 +489,21 @@ __global__ void __launch_bounds__(kThreads) topk_collect_kernel(Workspace w, Fas
                                                                 const float* __restrict__ ens, int N,
                                                                 uint8_t* __restrict__ keep) {
   const int b = blockIdx.y;
+  const int64_t base = (int64_t)blockIdx.x * kChunk;
+  const float* row = ens + (int64_t)b * N;
+  // the scores are loaded before the row's state and threshold are read, so
+  // the two latencies overlap (loads past the row's valid length are masked
+  // below; every index here is inside the row)
+  uint32_t key[kPerThread];  // the scores' bits, then their order keys
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
+    key[i] = n < N ? __float_as_uint(__ldg(row + n)) : 0u;
+  }
   const RowState* st = w.state + b;
   const int mode = st->mode;
   if (mode != kModeFast && mode != kModeAll && mode != kModeEmpty) return;
   const int nv = st->nv;
-  const int64_t base = (int64_t)blockIdx.x * kChunk;
-  const float* row = ens + (int64_t)b * N;
   uint8_t* out = keep + (int64_t)b * N;
   if ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(keep) & 3u) == 0) {
 #pragma unroll
@@ -516,12 +525,11 @@ __global__ void __launch_bounds__(kThreads) topk_collect_kernel(Workspace w, Fas
   }
   if (mode != kModeFast) return;  // uniform across the block
   const uint32_t tau = f.tau[b];
-  uint32_t key[kPerThread];
   uint32_t is_cand = 0;  // bit i: element i of this thread is a candidate
 #pragma unroll
   for (int i = 0; i < kPerThread; ++i) {
     const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
-    key[i] = order_key(n < nv ? __ldg(row + n) : 0.f);
+    key[i] = order_key(n < nv ? __uint_as_float(key[i]) : 0.f);
     if (n < nv && key[i] >= tau) is_cand |= 1u << i;
   }
   // one atomic per block: the block's candidates go to one range of the list
@@ -608,9 +616,28 @@ __global__ void __launch_bounds__(kBlkThreads) topk_fastsel_kernel(Workspace w, 
   }
   uint32_t* keys = s_dyn;
   int* idx = reinterpret_cast<int*>(s_dyn + C);
-  for (int i = t; i < cnt; i += kBlkThreads) {
-    keys[i] = f.ckey[(size_t)b * C + i];
-    idx[i] = f.cidx[(size_t)b * C + i];
+  {  // eight loads of each list per thread in flight at a time, not one
+    const uint32_t* ck = f.ckey + (size_t)b * C;
+    const int* ci = f.cidx + (size_t)b * C;
+    constexpr int kU = 8;
+    for (int i0 = t; i0 < cnt; i0 += kU * kBlkThreads) {
+      uint32_t kk[kU];
+      int ii[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = i0 + u * kBlkThreads;
+        kk[u] = i < cnt ? __ldg(ck + i) : 0u;
+        ii[u] = i < cnt ? __ldg(ci + i) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = i0 + u * kBlkThreads;
+        if (i < cnt) {
+          keys[i] = kk[u];
+          idx[i] = ii[u];
+        }
+      }
+    }
   }
   __syncthreads();
   uint32_t T;
