@@ -437,17 +437,28 @@ __global__ void __launch_bounds__(kThreads) topk_mask_kernel(Workspace w, const 
   }
 }
 
-// Fast path, per row: the sample and the threshold tau; zeroes the list.
+// Fast path, per row: the row state (what topk_init_kernel writes for the
+// other forms; the fast path uses no histogram), then the sample and the
+// threshold tau; zeroes the list.
 __global__ void __launch_bounds__(kBlkThreads) topk_sample_kernel(Workspace w, FastWs f,
-                                                                  const float* __restrict__ ens, int N) {
+                                                                  const float* __restrict__ ens, int N,
+                                                                  const int32_t* __restrict__ n_valid, int k) {
   extern __shared__ uint32_t s_key[];  // [kSample]
   __shared__ uint32_t s_hist[2048];
   __shared__ int s_warp[kBlkThreads / 32 + 1];
   __shared__ uint32_t s_pick[2];
   const int b = blockIdx.x, t = threadIdx.x;
-  const RowState* st = w.state + b;
-  if (st->mode != kModeFast) return;  // uniform across the block
-  const int nv = st->nv, K = st->remaining;
+  const int nv = row_nvalid(n_valid, b, N), K = min(k, nv);
+  const int mode = nv == 0 ? kModeEmpty : (k >= nv ? kModeAll : kModeFast);
+  if (t == 0) {
+    RowState s = {};
+    s.nv = nv;
+    s.mode = mode;
+    s.prefix = 0u;
+    s.remaining = K;
+    w.state[b] = s;
+  }
+  if (mode != kModeFast) return;  // uniform across the block
   const int S = nv < kSample ? nv : kSample;
   const float* row = ens + (size_t)b * N;
   {  // all of a thread's loads in flight at once
@@ -599,14 +610,14 @@ __global__ void __launch_bounds__(kBlkThreads) topk_fastsel_kernel(Workspace w, 
   __shared__ uint32_t s_pick[2];
   const int b = blockIdx.x, t = threadIdx.x;
   RowState* st = w.state + b;
-  const int mode = st->mode;
+  // the row's mode, count and K are read together (one latency, not two)
+  const int mode = st->mode, cnt = f.cnt[b], K = st->remaining;
   __syncthreads();  // every thread has read the mode before thread 0 may change it
   if (mode == kModeAll || mode == kModeEmpty) {  // the collect pass wrote their masks
     if (t == 0) st->mode = kModeDone;
     return;
   }
   if (mode != kModeFast) return;
-  const int cnt = f.cnt[b], K = st->remaining;
   const BlockSelScratch sc{s_hist, s_warp, s_pick};
   uint8_t* out = keep + (int64_t)b * N;
   if (cnt < K || cnt > C) {  // too few candidates (tau too high) or too many to hold
@@ -720,8 +731,6 @@ fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, in
   Workspace w = carve(ws, B, nblk);
   const int C = cand_cap(N);
   const bool fast = ws_size >= fast_ws_bytes(B, nblk, C) && 2 * (int64_t)k + 1024 <= C;
-  topk_init_kernel<<<B, 256, 0, st>>>(w, n_valid, N, k, fast ? 1 : 0);
-  note_launch();
   dim3 grid(nblk, B);
   if (fast) {
     static PerDeviceOnce smem_set;
@@ -731,12 +740,14 @@ fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, in
                                       (int)(2 * sizeof(uint32_t) * kCandMax)))
       return s;
     const FastWs f = carve_fast(ws, B, nblk, C);
-    topk_sample_kernel<<<B, kBlkThreads, sizeof(uint32_t) * kSample, st>>>(w, f, ens, N);
+    topk_sample_kernel<<<B, kBlkThreads, sizeof(uint32_t) * kSample, st>>>(w, f, ens, N, n_valid, k);
     topk_collect_kernel<<<grid, kThreads, 0, st>>>(w, f, C, ens, N, keep);
     topk_fastsel_kernel<<<B, kBlkThreads, 2 * sizeof(uint32_t) * (size_t)C, st>>>(w, f, ens, C, N, keep);
     for (int i = 0; i < 3; ++i) note_launch();
     return check_launch();  // every row is finished by the candidate path or its in-block fallback
   }
+  topk_init_kernel<<<B, 256, 0, st>>>(w, n_valid, N, k, 0);
+  note_launch();
   topk_hist_kernel<0, true><<<grid, kThreads, 0, st>>>(w, ens, N, nullptr);
   topk_hist_kernel<1, true><<<grid, kThreads, 0, st>>>(w, ens, N, nullptr);
   topk_hist_kernel<2, true><<<grid, kThreads, 0, st>>>(w, ens, N, nullptr);
