@@ -301,26 +301,8 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes,
-                                              uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
-      "[%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
 
-// Prefetch [src, src + bytes) from global memory into L2 (bulk, no shared
-// memory involved).  src and bytes must be multiples of 16.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
 
 // Makes this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor-core operand reads).
@@ -328,9 +310,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -377,21 +356,6 @@ __device__ __forceinline__ void umma_f8f6f4_ts(uint32_t d_tmem, uint32_t a_tmem,
       : "memory");
 }
 
-// 32 lanes x 32 consecutive 32-bit columns from registers into TMEM at taddr
-// (thread i writes lane base+i), then waits until the store has completed.
-__device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const uint32_t* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
-      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
-      "r"(v[29]), "r"(v[30]), "r"(v[31])
-      : "memory");
-}
 
 // As tmem_st32_wait, plus one more 32-bit column per lane at taddr1 (the same
 // wait covers both stores).
@@ -411,17 +375,6 @@ __device__ __forceinline__ void tmem_st32_st1_wait(uint32_t taddr, const uint32_
       : "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, tf32 inputs (fp32 containers,
-// the low 13 mantissa bits ignored), fp32 accumulate.
-__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 
 // Tiled TMA loads (no multicast) of a box at the given element coordinates,
 // completing on `bar`.  The innermost coordinate times the element size is a
@@ -553,40 +506,6 @@ __device__ __forceinline__ void tmem_ld32x3_wait(uint32_t t0, uint32_t t1, uint3
       "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95}, [%98];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
       : FM_TMEM_REGS32(a), FM_TMEM_REGS32(b), FM_TMEM_REGS32(c)
-      : "r"(t0), "r"(t1), "r"(t2)
-      : "memory");
-}
-
-// 16-column variants: P loads of 32 lanes x 16 fp32 columns, then one wait.
-#define FM_TMEM_REGS16(p)                                                                  \
-  "=r"(p[0]), "=r"(p[1]), "=r"(p[2]), "=r"(p[3]), "=r"(p[4]), "=r"(p[5]), "=r"(p[6]),    \
-      "=r"(p[7]), "=r"(p[8]), "=r"(p[9]), "=r"(p[10]), "=r"(p[11]), "=r"(p[12]),         \
-      "=r"(p[13]), "=r"(p[14]), "=r"(p[15])
-
-__device__ __forceinline__ void tmem_ld16x2_wait(uint32_t t0, uint32_t t1, uint32_t* a,
-                                                 uint32_t* b) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%32];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%33];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : FM_TMEM_REGS16(a), FM_TMEM_REGS16(b)
-      : "r"(t0), "r"(t1)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld16x3_wait(uint32_t t0, uint32_t t1, uint32_t t2,
-                                                 uint32_t* a, uint32_t* b, uint32_t* c) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%48];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%49];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47}, [%50];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : FM_TMEM_REGS16(a), FM_TMEM_REGS16(b), FM_TMEM_REGS16(c)
       : "r"(t0), "r"(t1), "r"(t2)
       : "memory");
 }
