@@ -350,7 +350,8 @@ size_t fm_compact_workspace_bytes(int B, int N);
 fm_status fm_compact_mask(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx, int32_t* count,
                           void* ws, size_t ws_bytes, cudaStream_t stream);
 
-/* Gathers the selected chunks' records into a resident buffer:
+/* Gathers the selected chunks' records into a resident buffer (the model
+ * card's "How it works": the resident set recalled to the GPU):
  * for every row b and j < min(count[b], max_sel) with 0 <= idx[b, j] < n_src,
  *   dst[b*dst_row_stride + j*rec_bytes, +rec_bytes) =
  *   src[b*src_row_stride + idx[b, j]*rec_bytes, +rec_bytes).
@@ -359,7 +360,10 @@ fm_status fm_compact_mask(const uint8_t* keep, int B, int N, int max_sel, int32_
  * (cudaHostAlloc / torch pin_memory; read over the bus by the kernel);
  * pageable host memory is rejected with FM_ERR_INVALID_ARG.  dst: device
  * memory.  idx, count as written by fm_compact_mask (device).  Any record
- * size; 16-byte copies when both pointers, the strides and rec_bytes are
+ * size.  From device memory, records of 64 B or more whose pointers, strides
+ * and size are multiples of 4 move by bulk copies staged in shared memory
+ * (each copy covers the 16-byte granules of its record); otherwise 16-byte
+ * loads and stores when both pointers, the strides and rec_bytes are
  * multiples of 16, 4-byte ones when of 4, else byte copies. */
 fm_status fm_gather_records(const void* src, int64_t src_row_stride_bytes, int n_src, int64_t rec_bytes,
                             const int32_t* idx, const int32_t* count, int B, int max_sel, void* dst,
@@ -447,8 +451,10 @@ fm_status fm_toy_decoder_update(const float* hidden, const float* attn_out, int 
                                 float* hidden_out, cudaStream_t stream);
 
 /* Synchronises `stream` and returns FM_ERR_DEVICE if a kernel launched on this
- * context recorded an error since the last call (the record is cleared),
- * FM_ERR_CUDA if the stream reports a CUDA error, FM_OK otherwise. */
+ * context recorded an error since the last call (the record is cleared), or
+ * if one of the context-free kernels of the current device did (decode
+ * attention, compaction, gather: a bounded wait that ran out), FM_ERR_CUDA
+ * if the stream reports a CUDA error, FM_OK otherwise. */
 fm_status fm_sync_status(fm_ctx* ctx, cudaStream_t stream);
 
 /* Static text for a status code. */

@@ -428,7 +428,9 @@ fm_status fm_sync_status(fm_ctx* c, cudaStream_t stream) {
     cudaMemset(c->d_err, 0, sizeof(int));
     return FM_ERR_DEVICE;
   }
-  if (take_attention_error() != kDevErrNone) return FM_ERR_DEVICE;
+  const bool attn = take_attention_error() != kDevErrNone;
+  const bool recall = take_recall_error() != kDevErrNone;
+  if (attn || recall) return FM_ERR_DEVICE;
   return FM_OK;
 }
 

@@ -159,10 +159,10 @@ size_t compact_workspace_bytes(int B, int N);
 fm_status launch_compact(const uint8_t* keep, int B, int N, int max_sel, int32_t* idx, int32_t* count,
                          void* ws, cudaStream_t stream);
 // src and dst: addresses a kernel can dereference (device memory, or the
-// device address of pinned host memory).
-fm_status launch_gather(const void* src, int64_t src_row_stride_bytes, int n_src, int64_t rec_bytes,
-                        const int32_t* idx, const int32_t* count, int B, int max_sel, void* dst,
-                        int64_t dst_row_stride_bytes, cudaStream_t stream);
+// device address of pinned host memory); src_on_device: src is device memory.
+fm_status launch_gather(const void* src, bool src_on_device, int64_t src_row_stride_bytes, int n_src,
+                        int64_t rec_bytes, const int32_t* idx, const int32_t* count, int B, int max_sel,
+                        void* dst, int64_t dst_row_stride_bytes, cudaStream_t stream);
 fm_status launch_topk_shard_begin(const int32_t* n_valid, int B, int N, int k, int32_t* hist, void* ws,
                                   size_t ws_bytes, cudaStream_t stream);
 fm_status launch_topk_shard_hist(const float* ens, int B, int N, int pass, int32_t* hist, void* ws,
@@ -178,6 +178,8 @@ fm_status launch_topk_shard_mask(const float* ens, int B, int N, const int32_t* 
 // Reads and clears the error word of the decode attention's segment kernel
 // on the current device (kDevErrNone when no wait ran out).
 int take_attention_error();
+// The same for the recall kernels' bulk-copy waits (compaction and gather).
+int take_recall_error();
 
 #if defined(__CUDACC__)
 

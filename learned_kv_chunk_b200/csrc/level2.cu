@@ -140,7 +140,7 @@ fm_status record_step(fm_level2* s, cudaStream_t st) {
   if (e != FM_OK) return e;
   if (cudaMemsetAsync(d.out_ids, 0xff, sizeof(int32_t) * (size_t)d.B * d.k, st) != cudaSuccess)
     return check_launch();
-  e = launch_gather(d.resident_ids, (int64_t)d.R * 4, d.R, 4, s->slots, s->slot_count, d.B, d.k, d.out_ids,
+  e = launch_gather(d.resident_ids, true, (int64_t)d.R * 4, d.R, 4, s->slots, s->slot_count, d.B, d.k, d.out_ids,
                     (int64_t)d.k * 4, st);
   if (e != FM_OK) return e;
   if (d.out_count &&

@@ -1,8 +1,11 @@
 """Parity of the recall kernels (keep mask -> index list -> resident buffer)
 with the CPU oracle, bit for bit: several compaction blocks per row with a
 ragged tail, masks from empty to full, lists longer and shorter than max_sel,
-records of 132 B (4-byte copies), 1024 B (16-byte copies) and 131 B (byte
-copies), from device memory and from pinned host memory."""
+rows that start on 16 bytes (the mask landed in shared memory by bulk
+copies) and rows that do not or are too long for it (register form);
+records of 132 B and 1024 B (bulk copies from device memory, also at
+sources and strides off the 16-byte grid; 4- and 16-byte loads from pinned
+host memory) and 131 B (byte copies)."""
 import numpy as np
 import pytest
 import torch
@@ -25,7 +28,7 @@ def _masks(B, N, seed):
     return (torch.rand(B, N, generator=g) < dens[:, None]).to(torch.uint8)
 
 
-@pytest.mark.parametrize("N", [3 * 16384 + 77, 2 * 16384 + 32, 5, 16384])
+@pytest.mark.parametrize("N", [3 * 16384 + 77, 2 * 16384 + 32, 2 * 16384 + 48, 5, 16384, 17 * 16384 + 16])
 @pytest.mark.parametrize("max_sel", [1, 100, 4096, 70000])
 def test_compact_matches_oracle(N, max_sel):
     keep = _masks(6, N, N + max_sel)
@@ -57,6 +60,31 @@ def test_gather_matches_oracle(rec, where):
     torch.cuda.synchronize()
     want = OR.gather_records(src.numpy(), idx.cpu().numpy(), count.cpu().numpy(),
                              np.full((B, max_sel, rec), 0xA5, np.uint8))
+    np.testing.assert_array_equal(dst.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("src_off,pad", [(4, 0), (8, 4), (12, 12)])
+def test_gather_off_grid_sources(src_off, pad):
+    """Records that start 4, 8 or 12 bytes past a 16-byte boundary, with row
+    strides that move the start from row to row: each bulk copy covers the
+    record's 16-byte granules and the record is cut out of them."""
+    B, n_src, rec, max_sel = 5, 2100, 132, 300
+    stride = n_src * rec + pad
+    g = torch.Generator().manual_seed(src_off + 16 * pad)
+    flat = torch.randint(0, 256, (src_off + B * stride + 16,), generator=g, dtype=torch.uint8)
+    keep = _masks(B, n_src, src_off)[[2, 3, 4, 1, 0]]
+    idx, count = fm.fm_compact_mask(keep.to(DEV), max_sel)
+    flat_d = flat.to(DEV)
+    dst = torch.full((B, max_sel, rec), 0x5A, dtype=torch.uint8, device=DEV)
+    base = flat_d.data_ptr() + src_off
+    assert base % 16 == src_off
+    st = fm.lib().fm_gather_records(base, stride, n_src, rec, idx.data_ptr(), count.data_ptr(), B, max_sel,
+                                    dst.data_ptr(), max_sel * rec, None)
+    assert st == fm.FM_OK
+    torch.cuda.synchronize()
+    src = np.stack([flat.numpy()[src_off + b * stride: src_off + b * stride + n_src * rec].reshape(n_src, rec)
+                    for b in range(B)])
+    want = OR.gather_records(src, idx.cpu().numpy(), count.cpu().numpy(), np.full((B, max_sel, rec), 0x5A, np.uint8))
     np.testing.assert_array_equal(dst.cpu().numpy(), want)
 
 
