@@ -448,6 +448,7 @@ __global__ void __launch_bounds__(kBlkThreads) topk_sample_kernel(Workspace w, F
   __shared__ int s_warp[kBlkThreads / 32 + 1];
   __shared__ uint32_t s_pick[2];
   const int b = blockIdx.x, t = threadIdx.x;
+  grid_dependency_wait();  // the scores (and n_valid) come from the kernels ahead
   const int nv = row_nvalid(n_valid, b, N), K = min(k, nv);
   const int mode = nv == 0 ? kModeEmpty : (k >= nv ? kModeAll : kModeFast);
   if (t == 0) {
@@ -504,13 +505,16 @@ __global__ void __launch_bounds__(kThreads) topk_collect_kernel(Workspace w, Fas
   const float* row = ens + (int64_t)b * N;
   // the scores are loaded before the row's state and threshold are read, so
   // the two latencies overlap (loads past the row's valid length are masked
-  // below; every index here is inside the row)
+  // below; every index here is inside the row).  This grid starts once the
+  // sample kernel's CTAs have left, each after its wait on the kernels that
+  // wrote the scores, so they may be read before waiting for it.
   uint32_t key[kPerThread];  // the scores' bits, then their order keys
 #pragma unroll
   for (int i = 0; i < kPerThread; ++i) {
     const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
     key[i] = n < N ? __float_as_uint(__ldg(row + n)) : 0u;
   }
+  grid_dependency_wait();  // the row state and tau come from the sample kernel
   const RowState* st = w.state + b;
   const int mode = st->mode;
   if (mode != kModeFast && mode != kModeAll && mode != kModeEmpty) return;
@@ -609,6 +613,7 @@ __global__ void __launch_bounds__(kBlkThreads) topk_fastsel_kernel(Workspace w, 
   __shared__ int s_warp[kBlkThreads / 32 + 1];
   __shared__ uint32_t s_pick[2];
   const int b = blockIdx.x, t = threadIdx.x;
+  grid_dependency_wait();  // the list and the mask's zeros come from the collect pass
   RowState* st = w.state + b;
   // the row's mode, count and K are read together (one latency, not two)
   const int mode = st->mode, cnt = f.cnt[b], K = st->remaining;
@@ -740,10 +745,19 @@ fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, in
                                       (int)(2 * sizeof(uint32_t) * kCandMax)))
       return s;
     const FastWs f = carve_fast(ws, B, nblk, C);
-    topk_sample_kernel<<<B, kBlkThreads, sizeof(uint32_t) * kSample, st>>>(w, f, ens, N, n_valid, k);
-    topk_collect_kernel<<<grid, kThreads, 0, st>>>(w, f, C, ens, N, keep);
-    topk_fastsel_kernel<<<B, kBlkThreads, 2 * sizeof(uint32_t) * (size_t)C, st>>>(w, f, ens, C, N, keep);
+    // three launches that may each start as the one ahead drains (each waits
+    // for it where it reads what it wrote).  No kernel lets the next one in
+    // earlier: collect CTAs resident during the sample's select, loading
+    // their scores, slowed the select (ragged 32-row case: 51 us against 42)
+    cudaError_t e = launch_overlapped(topk_sample_kernel, dim3(B), dim3(kBlkThreads), sizeof(uint32_t) * kSample,
+                                      st, w, f, ens, N, n_valid, k);
+    if (e == cudaSuccess)
+      e = launch_overlapped(topk_collect_kernel, grid, dim3(kThreads), 0, st, w, f, C, ens, N, keep);
+    if (e == cudaSuccess)
+      e = launch_overlapped(topk_fastsel_kernel, dim3(B), dim3(kBlkThreads), 2 * sizeof(uint32_t) * (size_t)C, st,
+                            w, f, (const float*)ens, C, N, keep);
     for (int i = 0; i < 3; ++i) note_launch();
+    if (e != cudaSuccess) return record_cuda_error(e);
     return check_launch();  // every row is finished by the candidate path or its in-block fallback
   }
   topk_init_kernel<<<B, 256, 0, st>>>(w, n_valid, N, k, 0);
