@@ -485,16 +485,22 @@ __global__ void __launch_bounds__(kThreads) qup_finish_kernel(const float* __res
 // part[s, b, m] = sum over the s-th K slice of W[m, k] X[b, layer(m), k], for
 // B <= TB <= 8 rows of X: bound by the bytes of W, each read once.  A warp owns
 // 4 consecutive rows of W and one K slice; lane j streams the float4 columns
-// k = 4j + 128i of its 4 rows with kGemvUnroll slices of loads in flight, the
+// k = 4j + 128i of its 4 rows with gemv_unroll(TB) slices of loads in flight, the
 // CTA's X slice sits in shared memory, and the 4 x TB sums are reduced across
 // the warp by a butterfly in which every exchange halves the values a lane
 // holds (4 TB - 1 shuffles in all) and lane j ends with sum number j.
 constexpr int kGemvWarps = 8;
 constexpr int kGemvRows = 4;  // rows of W per warp
 constexpr int kGemvUnroll = 4;
+// One row: three slices per warp in flight and three CTAs per SM (registers
+// for 3 x 256 threads), so a down projection of 408 CTAs runs in one wave;
+// more rows: four slices, two CTAs per SM.
+__host__ __device__ constexpr int gemv_unroll(int TB) { return TB == 1 ? 3 : kGemvUnroll; }
+__host__ __device__ constexpr int gemv_min_blocks(int TB) { return TB == 1 ? 3 : 1; }
+__host__ __device__ constexpr int gemv_ctas_per_sm(int TB) { return TB == 1 ? 3 : 2; }
 
 template <int TB>
-__global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(
+__global__ void __launch_bounds__(kGemvWarps * 32, gemv_min_blocks(TB)) gemv_kernel(
     const float* __restrict__ W, int M, int K, int kslice, const float* __restrict__ X,
     int64_t x_row_stride, int64_t x_layer_stride, int rows_per_layer, int B, float* __restrict__ part) {
   extern __shared__ __align__(16) float Xs[];  // [TB][kslice]
@@ -505,10 +511,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(
   const int k0 = s * kslice;
   const int layer = rows_per_layer > 0 ? m_cta / rows_per_layer : 0;
   const bool rows_ok = m0 + kGemvRows <= M;
+  constexpr int kU = gemv_unroll(TB);
   // W does not depend on the kernel ahead: start its first slices now.  The
-  // register ring w holds kGemvUnroll slices (slice i in w[i % kGemvUnroll]);
-  // a slot is reloaded with slice i + kGemvUnroll as soon as slice i is used.
-  float4 w[kGemvUnroll][kGemvRows];
+  // register ring w holds kU slices (slice i in w[i % kU]);
+  // a slot is reloaded with slice i + kU as soon as slice i is used.
+  float4 w[kU][kGemvRows];
   const float* wrow = W + (size_t)m0 * K + k0 + 4 * lane;
   auto load_slice = [&](float4* dst, int i) {
 #pragma unroll
@@ -518,7 +525,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(
                    : make_float4(0.f, 0.f, 0.f, 0.f);
   };
 #pragma unroll
-  for (int u = 0; u < kGemvUnroll; ++u) load_slice(w[u], u);
+  for (int u = 0; u < kU; ++u) load_slice(w[u], u);
   grid_dependency_wait();  // X is written by the kernel ahead
   const float* xsrc = X + (size_t)layer * x_layer_stride + k0;
   for (int i = threadIdx.x; i < TB * kslice / 4; i += kGemvWarps * 32) {
@@ -532,9 +539,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(
 #pragma unroll
   for (int v = 0; v < kGemvRows * TB; ++v) acc[v] = 0.f;
   const int nslices = kslice / 128;
-  for (int i0 = 0; i0 < nslices; i0 += kGemvUnroll) {
+  for (int i0 = 0; i0 < nslices; i0 += kU) {
 #pragma unroll
-    for (int u = 0; u < kGemvUnroll; ++u) {
+    for (int u = 0; u < kU; ++u) {
       const int i = i0 + u;
       if (i >= nslices) break;
 #pragma unroll
@@ -550,7 +557,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(
           acc[r * TB + b] = a;
         }
       }
-      load_slice(w[u], i + kGemvUnroll);
+      load_slice(w[u], i + kU);
     }
   }
   // butterfly: at stride h, the lanes with bit h set keep the upper half of
@@ -868,7 +875,7 @@ fm_status launch_query_prep_gemv(fm_ctx* ctx, const float* hidden, const int64_t
   int ks = 1;
   const int row_blocks = (Md + kGemvWarps * kGemvRows - 1) / (kGemvWarps * kGemvRows);
   while (ks * 2 <= ctx->splitk_max && HID % (ks * 2 * 128) == 0 && HID / (ks * 2) >= 1024 &&
-         row_blocks * ks < 2 * ctx->num_sms)
+         row_blocks * ks < gemv_ctas_per_sm(TB) * ctx->num_sms)
     ks *= 2;
   while (sizeof(float) * TB * (size_t)(HID / ks) > 64 * 1024 && ks * 2 <= ctx->splitk_max &&
          HID % (ks * 2 * 128) == 0)
