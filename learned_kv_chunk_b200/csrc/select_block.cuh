@@ -24,7 +24,7 @@ __device__ __forceinline__ uint32_t block_order_key(float x) {
 
 // Shared scratch of the selection: s_warp holds kBlkThreads / 32 + 1 ints.
 struct BlockSelScratch {
-  uint32_t* hist;  // 2048 bins
+  uint32_t* hist;  // 2048 words: eight 256-bin histograms, one per pair of warps
   int* warp;       // kBlkThreads / 32 + 1
   uint32_t* pick;  // 2
 };
@@ -64,10 +64,16 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
 //
 // The keys share every bit above the highest bit in which their maximum and
 // minimum differ, so the passes start there: each pass histograms the next
-// (up to) 11 undecided bits of the keys that match the bits decided so far
-// and picks the digit holding the want-th largest.  Once the picked digit
-// holds at most kSelFinish keys, they are gathered and ranked directly.
+// (up to) 8 undecided bits of the keys that match the bits decided so far
+// and picks the digit holding the want-th largest.  Each pair of warps counts
+// into its own 256-bin histogram with plain shared-memory atomics, so equal
+// digits contend within two warps only (scores near the cut share their
+// leading bits); the eight histograms are summed per bin.  Once the picked
+// digit holds at most kSelFinish keys, they are gathered and ranked directly.
 constexpr int kSelFinish = 256;
+constexpr int kSelBits = 8, kSelBins = 1 << kSelBits;
+constexpr int kSelCopies = kBlkThreads / 64;  // one histogram per two warps
+static_assert(kSelCopies * kSelBins == 2048 && kSelBins <= kBlkThreads, "selection scratch");
 
 template <class KeyAt>
 __device__ __forceinline__ void block_kth_largest_of(KeyAt key_at, int n, uint32_t want, BlockSelScratch sc,
@@ -103,48 +109,30 @@ __device__ __forceinline__ void block_kth_largest_of(KeyAt key_at, int n, uint32
   }
   int lo = 32 - __clz(kmax ^ kmin);  // bits [0, lo) undecided
   uint32_t prefix = lo >= 32 ? 0u : (kmax >> lo) << lo;
-  const unsigned lane_lt = (1u << lane) - 1u;
+  uint32_t* my_hist = sc.hist + (warp >> 1) * kSelBins;
 #pragma unroll 1
   while (lo > 0) {
-    const int nbits = lo < 11 ? lo : 11, shift = lo - nbits, nb = 1 << nbits;
-    for (int i = t; i < nb; i += kBlkThreads) sc.hist[i] = 0u;
+    const int nbits = lo < kSelBits ? lo : kSelBits, shift = lo - nbits, nb = 1 << nbits;
+    for (int i = t; i < kSelCopies * kSelBins; i += kBlkThreads) sc.hist[i] = 0u;
     __syncthreads();
-    // lanes holding the same digit add to the histogram with one atomic
     for (int i0 = 0; i0 < n; i0 += kBlkThreads) {
       const int i = i0 + t;
       const uint32_t key = i < n ? key_at(i) : 0u;
-      const bool act = i < n && (lo >= 32 || (key >> lo) == (prefix >> lo));
-      const unsigned active = __ballot_sync(0xffffffffu, act);
-      if (act) {
-        const uint32_t bin = (key >> shift) & (uint32_t)(nb - 1);
-        const unsigned peers = __match_any_sync(active, bin);
-        if ((peers & lane_lt) == 0) atomicAdd(&sc.hist[bin], (uint32_t)__popc(peers));
-      }
+      if (i < n && (lo >= 32 || (key >> lo) == (prefix >> lo)))
+        atomicAdd(&my_hist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
     }
     __syncthreads();
-    // thread t owns bins [t*per, (t+1)*per) in descending digit order
-    const int per = (nb + kBlkThreads - 1) / kBlkThreads;
+    // thread t < nb owns digit nb - 1 - t (descending digit order)
     uint32_t mine = 0;
-    for (int j = 0; j < per; ++j) {
-      const int d = nb - 1 - (t * per + j);
-      if (d >= 0) mine += sc.hist[d];
-    }
+    if (t < nb)
+#pragma unroll
+      for (int c = 0; c < kSelCopies; ++c) mine += sc.hist[c * kSelBins + (nb - 1 - t)];
     int tot;
     const uint32_t before = (uint32_t)block_exclusive_scan((int)mine, sc.warp, &tot);
-    if (before < want && before + mine >= want) {
-      uint32_t acc = before;
-      for (int j = 0; j < per; ++j) {
-        const int d = nb - 1 - (t * per + j);
-        if (d < 0) break;
-        const uint32_t c = sc.hist[d];
-        if (acc + c >= want) {
-          sc.pick[0] = prefix | ((uint32_t)d << shift);
-          sc.pick[1] = want - acc;
-          sc.warp[W] = (int)c;  // keys in the picked digit
-          break;
-        }
-        acc += c;
-      }
+    if (t < nb && before < want && before + mine >= want) {
+      sc.pick[0] = prefix | ((uint32_t)(nb - 1 - t) << shift);
+      sc.pick[1] = want - before;
+      sc.warp[W] = (int)mine;  // keys in the picked digit
     }
     __syncthreads();
     prefix = sc.pick[0];
