@@ -6,7 +6,7 @@
 // The selection is an exact radix select on the order-preserving 32-bit keys
 // of select.cu (larger score -> larger key, +0 = -0, NaN lowest).  The passes
 // start at the highest bit in which the row's valid keys differ (found first,
-// with one OR over the cluster), 11 bits at a time: sigmoid scores share
+// with one OR over the cluster), 8 bits at a time: sigmoid scores share
 // their sign and most of their exponent, and a first pass over the top bits
 // would pile them into a few bins.  The passes fix the K-th largest key T and
 // how many keys equal to T are kept; the mask keeps every key > T and the
@@ -16,7 +16,7 @@
 // slice [r*S, (r+1)*S) of the row, S = ceil(N / C) <= 16384, as keys in its
 // shared memory (thread t handles keys j*512 + t), so the row is read from
 // global memory once.  Per pass: every CTA histograms its keys into its own shared
-// histogram; a cluster barrier; CTA r sums the bins b with b % C == r over the
+// histogram (a copy per pair of warps, then summed); a cluster barrier; CTA r sums the bins b with b % C == r over the
 // cluster (distributed shared memory reads); a cluster barrier; then every
 // CTA reads the C owners' sums and finds the digit itself (all CTAs compute
 // the same digit from the same sums).  Histograms and sums are double
@@ -41,7 +41,9 @@ constexpr int kBins = 2048;
 constexpr int kTargetSlice = 4096;  // keys per CTA the cluster size aims for
 
 struct ClusterSmem {
-  uint32_t hist[2][kBins];  // this CTA's histogram of the pass
+  uint32_t hist[2][kBins];  // this CTA's histogram of the pass: counted in kSelCopies
+                            // 256-bin copies (one per pair of warps), then summed into
+                            // its first kSelBins words
   uint32_t sum[2][kBins];   // bins b with b % C == rank: the cluster's total
   int warp[kCThreads / 32 + 1];
   uint32_t pick[3];         // prefix so far, want, count of keys == T (last pass)
@@ -118,29 +120,33 @@ __global__ void __launch_bounds__(kCThreads, 2) topk_cluster_kernel(const float*
   const uint32_t all_diff = S.pick[0];
   __syncthreads();
 
-  // radix passes over the bits below the highest differing bit, 11 at a time
+  // radix passes over the bits below the highest differing bit, 8 at a time:
+  // each pair of warps counts into its own 256-bin copy with plain atomics
+  // (equal digits contend within two warps only), and the copies are summed
   int top = all_diff ? 32 - __clz(all_diff) : 0;  // bits [top, 32) are the reference's
   uint32_t prefix = ref & ~low_mask(top), want = (uint32_t)k, cnt_eq = (uint32_t)nv;
-  const unsigned lane_lt = (1u << lane) - 1u;
 #pragma unroll 1
   for (int pass = 0; top > 0; ++pass) {
-    const int nbits = top < 11 ? top : 11, shift = top - nbits, nb = 1 << nbits;
+    const int nbits = top < kSelBits ? top : kSelBits, shift = top - nbits, nb = 1 << nbits;
     uint32_t* h = S.hist[pass & 1];
     uint32_t* sm = S.sum[pass & 1];
-    for (int i = t; i < nb; i += kCThreads) h[i] = 0u;
+    for (int i = t; i < kSelCopies * kSelBins; i += kCThreads) h[i] = 0u;
     __syncthreads();
+    uint32_t* my_hist = h + (t >> 6) * kSelBins;
 #pragma unroll 4
     for (int j = 0; j < kKeysPerThread; ++j) {
       if (j >= rows) break;
       const int i = base + j * kCThreads + t;
       const uint32_t kk = key[j * kCThreads + t];
-      const bool act = i < vend && (top >= 32 || (kk >> top) == (prefix >> top));
-      const unsigned active = __ballot_sync(0xffffffffu, act);
-      if (act) {
-        const uint32_t bin = (kk >> shift) & (uint32_t)(nb - 1);
-        const unsigned peers = __match_any_sync(active, bin);
-        if ((peers & lane_lt) == 0) atomicAdd(&h[bin], (uint32_t)__popc(peers));
-      }
+      if (i < vend && (top >= 32 || (kk >> top) == (prefix >> top)))
+        atomicAdd(&my_hist[(kk >> shift) & (uint32_t)(nb - 1)], 1u);
+    }
+    __syncthreads();
+    if (t < nb) {  // bin t of every copy is read and the sum written by thread t alone
+      uint32_t x = 0u;
+#pragma unroll
+      for (int c = 0; c < kSelCopies; ++c) x += h[c * kSelBins + t];
+      h[t] = x;
     }
     cl.sync();  // every CTA's histogram of this pass is complete
     // sum the owned bins over the cluster: pair p = (owned bin q, source CTA
