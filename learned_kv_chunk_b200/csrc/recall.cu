@@ -13,12 +13,16 @@
 //               resident buffer on the GPU.
 //
 // Compaction is one launch with a cluster of up to 4 CTAs per row: each CTA
-// counts the kept entries of its part of the mask, the cluster exchanges the
+// counts the kept entries of its part of the mask (landed in shared memory
+// by bulk copies when the row starts on 16 bytes), the cluster exchanges the
 // counts through distributed shared memory, and each CTA writes its indices
-// at the offset the CTAs before it leave.  The gather is a copy
-// with one warp per record and several records in flight per warp: the
-// selected records are scattered, so the copy engines (one call per
-// contiguous run) are not used.
+// at the offset the CTAs before it leave.  The gather from device memory
+// stages each record's 16-byte granules in shared memory with one bulk copy
+// per record and writes tiles of consecutive slots out with 4-byte stores;
+// from pinned host memory (or off the 4-byte grid) it is a copy with one
+// warp per record and several records in flight per warp.  The selected
+// records are scattered, so the copy engines (one call per contiguous run)
+// are not used.
 #include <cooperative_groups.h>
 
 #include "fm_internal.cuh"

@@ -496,21 +496,23 @@ __global__ void __launch_bounds__(kBlkThreads) topk_sample_kernel(Workspace w, F
 
 // Fast path, grid-wide: writes the mask of the Fast / All / Empty rows (zeros
 // for Fast rows; their kept bytes are set per row afterwards) and appends the
-// valid scores >= tau of Fast rows to the row's list.
+// valid scores >= tau of Fast rows to the row's list.  A CTA takes kThreads *
+// PER scores of one row (its own slicing: no workspace is kept per block).
+template <int PER>
 __global__ void __launch_bounds__(kThreads) topk_collect_kernel(Workspace w, FastWs f, int C,
                                                                 const float* __restrict__ ens, int N,
                                                                 uint8_t* __restrict__ keep) {
   const int b = blockIdx.y;
-  const int64_t base = (int64_t)blockIdx.x * kChunk;
+  const int64_t base = (int64_t)blockIdx.x * (kThreads * PER);
   const float* row = ens + (int64_t)b * N;
   // the scores are loaded before the row's state and threshold are read, so
   // the two latencies overlap (loads past the row's valid length are masked
   // below; every index here is inside the row).  This grid starts once the
   // sample kernel's CTAs have left, each after its wait on the kernels that
   // wrote the scores, so they may be read before waiting for it.
-  uint32_t key[kPerThread];  // the scores' bits, then their order keys
+  uint32_t key[PER];  // the scores' bits, then their order keys
 #pragma unroll
-  for (int i = 0; i < kPerThread; ++i) {
+  for (int i = 0; i < PER; ++i) {
     const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
     key[i] = n < N ? __float_as_uint(__ldg(row + n)) : 0u;
   }
@@ -522,7 +524,7 @@ __global__ void __launch_bounds__(kThreads) topk_collect_kernel(Workspace w, Fas
   uint8_t* out = keep + (int64_t)b * N;
   if ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(keep) & 3u) == 0) {
 #pragma unroll
-    for (int i = 0; i < kPerThread / 4; ++i) {
+    for (int i = 0; i < PER / 4; ++i) {
       const int64_t n = base + ((int64_t)i * kThreads + threadIdx.x) * 4;
       if (n >= N) break;
       uint32_t word = 0;
@@ -532,7 +534,7 @@ __global__ void __launch_bounds__(kThreads) topk_collect_kernel(Workspace w, Fas
       *reinterpret_cast<uint32_t*>(out + n) = word;
     }
   } else {
-    for (int i = 0; i < kPerThread; ++i) {
+    for (int i = 0; i < PER; ++i) {
       const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
       if (n >= N) break;
       out[n] = (mode == kModeAll && n < nv) ? 1 : 0;
@@ -542,7 +544,7 @@ __global__ void __launch_bounds__(kThreads) topk_collect_kernel(Workspace w, Fas
   const uint32_t tau = f.tau[b];
   uint32_t is_cand = 0;  // bit i: element i of this thread is a candidate
 #pragma unroll
-  for (int i = 0; i < kPerThread; ++i) {
+  for (int i = 0; i < PER; ++i) {
     const int64_t n = base + (int64_t)i * kThreads + threadIdx.x;
     key[i] = order_key(n < nv ? __uint_as_float(key[i]) : 0.f);
     if (n < nv && key[i] >= tau) is_cand |= 1u << i;
@@ -556,7 +558,7 @@ __global__ void __launch_bounds__(kThreads) topk_collect_kernel(Workspace w, Fas
   __syncthreads();
   int pos = s_base + before;
 #pragma unroll
-  for (int i = 0; i < kPerThread; ++i) {
+  for (int i = 0; i < PER; ++i) {
     if (is_cand & (1u << i)) {
       if (pos < C) {
         f.ckey[(size_t)b * C + pos] = key[i];
@@ -751,8 +753,11 @@ fm_status launch_topk(const float* ens, const int32_t* n_valid, int B, int N, in
     // their scores, slowed the select (ragged 32-row case: 51 us against 42)
     cudaError_t e = launch_overlapped(topk_sample_kernel, dim3(B), dim3(kBlkThreads), sizeof(uint32_t) * kSample,
                                       st, w, f, ens, N, n_valid, k);
+    // 4096 scores per CTA: three CTAs per SM, where 8192 allowed two
+    constexpr int kCollectPer = 8;
+    const dim3 cgrid((unsigned)(((int64_t)N + kThreads * kCollectPer - 1) / (kThreads * kCollectPer)), (unsigned)B);
     if (e == cudaSuccess)
-      e = launch_overlapped(topk_collect_kernel, grid, dim3(kThreads), 0, st, w, f, C, ens, N, keep);
+      e = launch_overlapped(topk_collect_kernel<kCollectPer>, cgrid, dim3(kThreads), 0, st, w, f, C, ens, N, keep);
     if (e == cudaSuccess)
       e = launch_overlapped(topk_fastsel_kernel, dim3(B), dim3(kBlkThreads), 2 * sizeof(uint32_t) * (size_t)C, st,
                             w, f, (const float*)ens, C, N, keep);
