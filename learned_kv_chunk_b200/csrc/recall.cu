@@ -346,10 +346,12 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__
 // harmless), all copies completing on one barrier; the warps then write the
 // T records out with 4-byte stores, the slots of a row being contiguous in
 // dst.  No registers hold data in flight, so the many CTAs an SM holds
-// overlap their copies' latencies.  (A persistent form with two stages per
-// CTA, writing one tile while the next one's copies fly, measured slower.)
+// overlap their copies' latencies (64 slots of 132-byte records per CTA, 16
+// CTAs per SM, measured faster than 128 slots and 11).  A persistent form
+// with two stages per CTA, writing one tile while the next one's copies fly,
+// measured slower.
 constexpr int kGThreads = 128;        // threads per CTA; T <= kGThreads
-constexpr int kGStageBytes = 18432;   // staging shared memory per CTA (T * slot at most)
+constexpr int kGStageBytes = 9216;    // staging shared memory per CTA (T * slot at most)
 
 // Bytes of a record's slot: the 16-byte granules of a record that starts
 // 0, 4, 8 or 12 bytes past a granule boundary.
