@@ -111,6 +111,32 @@ def test_host_side_argument_rejection(lib):
     assert out.value is None
 
 
+def test_recall_argument_rejection(lib):
+    """The recall calls refuse bad arguments on the host, before any CUDA
+    call: null pointers, sizes below one, strides that cannot hold a row,
+    misaligned index lists, a workspace that is too small."""
+    P, I, I64, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.fm_compact_mask.argtypes = [P, I, I, I, P, P, P, S, P]
+    lib.fm_gather_records.argtypes = [P, I64, I, I64, P, P, I, I, P, I64, P]
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails its checks first
+    INVALID, ALIGN = 1, 2
+    ws = int(lib.fm_compact_workspace_bytes(4, 1000))
+    assert ws > 0
+    assert lib.fm_compact_mask(None, 4, 1000, 64, fake, fake, fake, ws, None) == INVALID
+    assert lib.fm_compact_mask(fake, 0, 1000, 64, fake, fake, fake, ws, None) == INVALID
+    assert lib.fm_compact_mask(fake, 4, 1000, 0, fake, fake, fake, ws, None) == INVALID
+    assert lib.fm_compact_mask(fake, 70000, 1000, 64, fake, fake, fake, ws, None) == INVALID  # B > 65535
+    assert lib.fm_compact_mask(fake, 4, 1000, 64, ctypes.c_void_p(0x1002), fake, fake, ws, None) == ALIGN
+    assert lib.fm_compact_mask(fake, 4, 1000, 64, fake, fake, ctypes.c_void_p(0x1008), ws, None) == ALIGN
+    assert lib.fm_compact_mask(fake, 4, 1000, 64, fake, fake, fake, ws - 1, None) == INVALID
+    assert lib.fm_gather_records(None, 1320, 10, 132, fake, fake, 4, 8, fake, 1056, None) == INVALID
+    assert lib.fm_gather_records(fake, 1320, 10, 0, fake, fake, 4, 8, fake, 1056, None) == INVALID
+    assert lib.fm_gather_records(fake, 1319, 10, 132, fake, fake, 4, 8, fake, 1056, None) == INVALID  # row stride
+    assert lib.fm_gather_records(fake, 1320, 10, 132, fake, fake, 4, 8, fake, 1055, None) == INVALID  # dst stride
+    assert lib.fm_gather_records(fake, 1320, 10, 132, ctypes.c_void_p(0x1001), fake, 4, 8, fake, 1056,
+                                 None) == ALIGN
+
+
 def test_header_is_plain_c(tmp_path):
     """include/fm.h is a C ABI: it compiles as strict C99 (and as C++), with
     every declared type usable from C."""
